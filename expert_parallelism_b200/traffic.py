@@ -1,0 +1,48 @@
+"""Byte and flop accounting for the MoE-layer hot path (host-side only).
+
+``dispatch_combine_bytes_per_token`` is the traffic rule of "Expert
+parallelism and all-to-all", section "Traffic math": each token's hidden
+vector travels to its k experts and back, 2 * k * H * bytes per token per
+MoE layer.  The rest gives the algorithmic HBM bytes and flops of each
+kernel on one GPU, the figures the roofline fractions divide by.
+"""
+from __future__ import annotations
+
+from .workloads import ELEM_BYTES, Workload
+
+
+def dispatch_combine_bytes_per_token(k: int, H: int, bytes_per_elem: int) -> int:
+    """2 * k * H * bytes: dispatch plus combine, one token, one MoE layer."""
+    return 2 * k * H * bytes_per_elem
+
+
+def dispatch_bytes_from_layout(rank_offsets_last: int, H: int, bytes_per_elem: int) -> int:
+    """Bytes the dispatch all-to-all would move for one GPU: every routed
+    row (rank_offsets[W] of them) of H elements."""
+    return rank_offsets_last * H * bytes_per_elem
+
+
+def kernel_bytes(wl: Workload) -> dict:
+    """Algorithmic HBM bytes per launch of each step (each input read once,
+    each output written once)."""
+    N, T, H, E, k, I = wl.N, wl.T, wl.H, wl.E, wl.k, wl.I
+    xb, pb, wb = ELEM_BYTES[wl.act], ELEM_BYTES[wl.payload], ELEM_BYTES[wl.wdt]
+    scales = N * (H // 128) * 4 if wl.payload == "e4m3" else 0
+    return {
+        "route_topk": T * E * 4 + T * k * 8,
+        "dispatch_layout": N * 4 + N * 8 + (2 * E + 1) * 4 + (wl.W + 1) * 4,
+        "permute": T * H * xb + N * H * pb + scales,
+        "combine": N * H * wb + T * k * 8 + T * H * xb,
+    }
+
+
+def gemm_flops(wl: Workload, rows: int | None = None) -> dict:
+    """Dense flops of the two GEMM phases for ``rows`` routed rows."""
+    n = wl.N if rows is None else rows
+    return {"gate_up": 2 * n * wl.H * 2 * wl.I, "down": 2 * n * wl.I * wl.H,
+            "total": 6 * n * wl.H * wl.I}
+
+
+def touched_weight_bytes(wl: Workload, experts_touched: int) -> int:
+    """Expert-weight bytes a pass must read at least once."""
+    return experts_touched * 3 * wl.I * wl.H * ELEM_BYTES[wl.wdt]

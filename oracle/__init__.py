@@ -1,0 +1,193 @@
+"""CPU oracle for the MoE-layer hot path -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product library never calls it
+and shares no code with it.
+
+The arithmetic lives in ``moe_oracle.c`` (plain C, fp64, OpenMP over the
+GEMM's rows); this module compiles it on first use and marshals CPU torch
+tensors in and out.  Every function takes and returns CPU tensors; bf16
+data travels as its bit pattern.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB = os.path.join(_HERE, "libmoe_oracle.so")
+
+F32, BF16, E4M3 = 0, 1, 2
+_CODE = {"f32": F32, "bf16": BF16, "e4m3": E4M3}
+_TDT = {"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.float8_e4m3fn}
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``oracle/libmoe_oracle.so`` (gcc, -O2, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+                               "-Wall", "-Wextra", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P, I64, I32, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int
+        lib.oracle_route_topk.argtypes = [P, I64, I32, I32, P, P]
+        lib.oracle_route_topk.restype = I
+        lib.oracle_dispatch_layout.argtypes = [P, I64, I32, I32, I32, P, P, P, P, P]
+        lib.oracle_dispatch_layout.restype = I64
+        lib.oracle_permute.argtypes = [P, I, I64, I32, I32, P, I64, P, I, P]
+        lib.oracle_permute.restype = I
+        lib.oracle_grouped_gemm.argtypes = [P, I, P, P, I32, I32, I32, I32, P, P, I, P, P, P]
+        lib.oracle_grouped_gemm.restype = I64
+        lib.oracle_combine.argtypes = [P, I, P, P, I64, I32, I32, P, I]
+        lib.oracle_combine.restype = I
+        lib.oracle_e4m3_encode.argtypes = [P, I64, P]
+        lib.oracle_e4m3_decode.argtypes = [P, I64, P]
+        lib.oracle_bf16_round.argtypes = [P, I64, P]
+        _lib = lib
+    return _lib
+
+
+def _p(t: torch.Tensor | None):
+    if t is None:
+        return None
+    assert t.device.type == "cpu" and t.is_contiguous()
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _dt_name(t: torch.Tensor) -> str:
+    for k, v in _TDT.items():
+        if t.dtype == v:
+            return k
+    raise TypeError(f"oracle: unsupported dtype {t.dtype}")
+
+
+# ---------------------------------------------------------------- codecs
+def e4m3_encode(v: torch.Tensor) -> torch.Tensor:
+    """fp32 -> e4m3 code bytes (uint8), RNE with saturation to +-448."""
+    v = v.to(torch.float32).contiguous()
+    out = torch.empty(v.shape, dtype=torch.uint8)
+    _load().oracle_e4m3_encode(_p(v), v.numel(), _p(out))
+    return out
+
+
+def e4m3_decode(c: torch.Tensor) -> torch.Tensor:
+    """e4m3 code bytes -> fp64 values."""
+    c = c.contiguous().view(torch.uint8)
+    out = torch.empty(c.shape, dtype=torch.float64)
+    _load().oracle_e4m3_decode(_p(c), c.numel(), _p(out))
+    return out
+
+
+def bf16_round(v: torch.Tensor) -> torch.Tensor:
+    """fp64 -> bf16 (RNE), returned as a bfloat16 tensor."""
+    v = v.to(torch.float64).contiguous()
+    out = torch.empty(v.shape, dtype=torch.int16)
+    _load().oracle_bf16_round(_p(v), v.numel(), _p(out))
+    return out.view(torch.bfloat16)
+
+
+# ---------------------------------------------------------------- the five steps
+def route_topk(logits: torch.Tensor, k: int):
+    logits = logits.to(torch.float32).contiguous()
+    T, E = logits.shape
+    idx = torch.empty(T, k, dtype=torch.int32)
+    w = torch.empty(T, k, dtype=torch.float32)
+    _load().oracle_route_topk(_p(logits), T, E, k, _p(idx), _p(w))
+    return idx, w
+
+
+def dispatch_layout(topk_idx: torch.Tensor, E: int, W: int):
+    topk_idx = topk_idx.to(torch.int32).contiguous()
+    T, k = topk_idx.shape
+    N = T * k
+    counts = torch.empty(E, dtype=torch.int32)
+    offsets = torch.empty(E + 1, dtype=torch.int32)
+    rank_offsets = torch.empty(W + 1, dtype=torch.int32)
+    slot_of_pair = torch.empty(N, dtype=torch.int32)
+    pair_of_slot = torch.empty(N, dtype=torch.int32)
+    bad = _load().oracle_dispatch_layout(_p(topk_idx), T, k, E, W, _p(counts), _p(offsets),
+                                         _p(rank_offsets), _p(slot_of_pair), _p(pair_of_slot))
+    return dict(expert_counts=counts, expert_offsets=offsets, rank_offsets=rank_offsets,
+                slot_of_pair=slot_of_pair, pair_of_slot=pair_of_slot, skipped=int(bad))
+
+
+def permute(x: torch.Tensor, k: int, pair_of_slot: torch.Tensor, payload: str,
+            fill: float = 0.0):
+    """Returns (xp, xp_scales or None).  Slots holding -1 keep ``fill``."""
+    x = x.contiguous()
+    T, H = x.shape
+    n_slots = pair_of_slot.numel()
+    xdt = _dt_name(x)
+    if payload == "e4m3":
+        xp = torch.full((n_slots, H), 0, dtype=torch.uint8)
+        sc = torch.full((n_slots, H // 128), fill, dtype=torch.float32)
+    else:
+        xp = torch.full((n_slots, H), fill, dtype=_TDT[payload])
+        sc = None
+    rc = _load().oracle_permute(_p(x), _CODE[xdt], T, H, k, _p(pair_of_slot.contiguous()),
+                                n_slots, _p(xp), _CODE[payload], _p(sc))
+    if rc != 0:
+        raise ValueError("oracle.permute: unsupported dtype pair")
+    if payload == "e4m3":
+        xp = xp.view(torch.float8_e4m3fn)
+    return xp, sc
+
+
+def grouped_gemm(xp: torch.Tensor, xp_scales, expert_offsets: torch.Tensor,
+                 expert_begin: int, n_experts: int, w13: torch.Tensor, w2: torch.Tensor,
+                 row_mask: torch.Tensor | None = None):
+    """Returns (h, y, rows_done); rows outside the mask (or outside the
+    experts' segments) are left as NaN."""
+    xp = xp.contiguous()
+    n_rows, H = xp.shape
+    I = w2.shape[2]
+    wdt = _dt_name(w13)
+    h = torch.full((n_rows, I), float("nan"), dtype=_TDT[wdt])
+    y = torch.full((n_rows, H), float("nan"), dtype=_TDT[wdt])
+    mask = None if row_mask is None else row_mask.to(torch.uint8).contiguous()
+    xdt = _dt_name(xp)
+    done = _load().oracle_grouped_gemm(
+        _p(xp.view(torch.uint8) if xdt == "e4m3" else xp), _CODE[xdt],
+        _p(xp_scales.contiguous() if xp_scales is not None else None),
+        _p(expert_offsets.to(torch.int32).contiguous()), expert_begin, n_experts, H, I,
+        _p(w13.contiguous()), _p(w2.contiguous()), _CODE[wdt], _p(mask), _p(h), _p(y))
+    return h, y, int(done)
+
+
+def combine(y: torch.Tensor, slot_of_pair: torch.Tensor, topk_w: torch.Tensor,
+            out_dtype: str):
+    y = y.contiguous()
+    T, k = topk_w.shape
+    H = y.shape[1]
+    out = torch.empty(T, H, dtype=_TDT[out_dtype])
+    _load().oracle_combine(_p(y), _CODE[_dt_name(y)], _p(slot_of_pair.to(torch.int32).contiguous()),
+                           _p(topk_w.to(torch.float32).contiguous()), T, k, H, _p(out),
+                           _CODE[out_dtype])
+    return out
+
+
+def layer(wl, inputs, row_mask=None):
+    """The whole hot path on one workload's inputs; returns every
+    intermediate (dict).  ``row_mask`` (per slot) samples the GEMM rows;
+    combine is then only meaningful for tokens whose pairs were all
+    computed."""
+    idx, w = route_topk(inputs["logits"], wl.k)
+    lay = dispatch_layout(idx, wl.E, wl.W)
+    xp, sc = permute(inputs["x"], wl.k, lay["pair_of_slot"], wl.payload)
+    h, y, _ = grouped_gemm(xp, sc, lay["expert_offsets"], 0, wl.E, inputs["w13"], inputs["w2"],
+                           row_mask)
+    out = combine(y, lay["slot_of_pair"], w, wl.act)
+    return dict(topk_idx=idx, topk_w=w, xp=xp, xp_scales=sc, h=h, y=y, out=out, **lay)

@@ -1,0 +1,345 @@
+/*
+ * moe_oracle.c -- plain, slow CPU oracle for the single-GPU core of an
+ * expert-parallel MoE layer (router top-k -> dispatch layout -> permute ->
+ * grouped SwiGLU expert GEMM -> weighted combine).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or
+ * call this file; only the tests, the smoke check and the benchmark's CPU
+ * baseline leg do.  It shares no code, header or table with the CUDA
+ * library: every helper below (bf16 rounding, the FP8 e4m3 codec, the
+ * softmax, the counting sort) is written here from its definition.
+ *
+ * Arithmetic is fp64 except where a value is defined by a narrower type:
+ *   - router logits are compared as the fp32 values they are;
+ *   - the FP8 payload's scale and quotient are fp32 IEEE divisions, because
+ *     they decide an integer code (the quantised byte) and the CUDA side
+ *     decides it in fp32 as well;
+ *   - every stored tensor (topk weights, h, y, out) is rounded once, from
+ *     the fp64 result, to its storage type.
+ *
+ * Sources (page title, section):
+ *   "Expert parallelism and all-to-all", "Walking through one MoE layer":
+ *       route, dispatch, grouped expert matmul, weighted combine.
+ *   "Expert Parallelism" (aiwiki), "Implementation": sort by destination
+ *       (argsort), per-rank bincount, undo the sort after the experts.
+ *   "Expert parallelism" (Transformers), "Adding an implementation" and
+ *       "How the sizes combine": (hidden_states, top_k_index, top_k_weights)
+ *       in, weighted expert output per token out; rank r owns experts
+ *       [r*E/W, (r+1)*E/W).
+ *   "Expert parallelism and all-to-all", "Traffic math": 1-byte FP8
+ *       activation payload.
+ *
+ * dtype codes: 0 = fp32, 1 = bf16 (uint16 bits), 2 = FP8 e4m3 (OCP, "fn").
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define OR_F32 0
+#define OR_BF16 1
+#define OR_E4M3 2
+
+/* ------------------------------------------------------------------ */
+/* number formats, written from their definitions                      */
+/* ------------------------------------------------------------------ */
+
+/* Round a non-negative real r to the nearest integer, ties to even. */
+static double rint_half_even(double r) {
+    double n = floor(r);
+    double f = r - n;
+    if (f > 0.5) return n + 1.0;
+    if (f < 0.5) return n;
+    return (fmod(n, 2.0) == 0.0) ? n : n + 1.0;
+}
+
+/* bf16: 1 sign, 8 exponent (bias 127), 7 fraction bits; subnormal quantum
+ * 2^-133; largest finite (2 - 2^-7) * 2^127.  Round-to-nearest-even from
+ * the exact fp64 value. */
+static uint16_t bf16_from_double(double v) {
+    if (isnan(v)) return 0x7FC0;
+    uint16_t s = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (a == 0.0) return s;
+    if (isinf(a)) return s | 0x7F80;
+    int e;
+    frexp(a, &e);              /* a = f * 2^e, f in [0.5, 1): binade 2^(e-1) */
+    int be = e - 1;
+    double q = (be < -126) ? ldexp(1.0, -133) : ldexp(1.0, be - 7);
+    double val = rint_half_even(a / q) * q;
+    if (val > ldexp(255.0, 120)) return s | 0x7F80;  /* rounds past max: inf */
+    float f = (float)val;      /* exact: val has <= 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return s | (uint16_t)((u >> 16) & 0x7FFF);
+}
+
+static double bf16_to_double(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+/* OCP 8-bit float E4M3 ("fn" variant): 1 sign, 4 exponent bits (bias 7),
+ * 3 mantissa bits; no infinities; S.1111.111 is NaN; largest finite
+ * S.1111.110 = 448; smallest normal 2^-6; subnormals m * 2^-9. */
+static double e4m3_to_double(uint8_t c) {
+    int E = (c >> 3) & 15, m = c & 7;
+    if (E == 15 && m == 7) return NAN;
+    double v = (E == 0) ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, E - 7);
+    return (c & 0x80) ? -v : v;
+}
+
+/* Encode an fp32 value: round to nearest, ties to even, saturating
+ * magnitudes above 448 to 448; NaN maps to 0x7F. */
+static uint8_t e4m3_from_float(float v) {
+    if (isnan(v)) return 0x7F;
+    uint8_t s = signbit(v) ? 0x80 : 0;
+    double a = fabs((double)v);
+    if (a > 448.0) return s | 0x7E;
+    double q;
+    if (a < ldexp(1.0, -6)) {
+        q = ldexp(1.0, -9);                    /* subnormal spacing */
+    } else {
+        int e;
+        frexp(a, &e);
+        q = ldexp(1.0, (e - 1) - 3);           /* 3 mantissa bits */
+    }
+    double val = rint_half_even(a / q) * q;    /* exact, <= 448 */
+    if (val == 0.0) return s;
+    if (val < ldexp(1.0, -6)) return s | (uint8_t)(val / ldexp(1.0, -9));
+    int e;
+    frexp(val, &e);
+    int be = e - 1;                            /* val in [2^be, 2^(be+1)) */
+    int m = (int)((val / ldexp(1.0, be) - 1.0) * 8.0);
+    return s | (uint8_t)((be + 7) << 3) | (uint8_t)m;
+}
+
+static double load_elem(const void* base, int dt, int64_t i) {
+    switch (dt) {
+        case OR_F32: return (double)((const float*)base)[i];
+        case OR_BF16: return bf16_to_double(((const uint16_t*)base)[i]);
+        default: return e4m3_to_double(((const uint8_t*)base)[i]);
+    }
+}
+
+static void store_elem(void* base, int dt, int64_t i, double v) {
+    if (dt == OR_F32) ((float*)base)[i] = (float)v;
+    else ((uint16_t*)base)[i] = bf16_from_double(v);
+}
+
+/* exported codec entry points (pinned by the CPU tests) */
+void oracle_e4m3_encode(const float* v, int64_t n, uint8_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = e4m3_from_float(v[i]);
+}
+void oracle_e4m3_decode(const uint8_t* c, int64_t n, double* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = e4m3_to_double(c[i]);
+}
+void oracle_bf16_round(const double* v, int64_t n, uint16_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = bf16_from_double(v[i]);
+}
+
+/* ------------------------------------------------------------------ */
+/* S1 route: top-k of the router logits + softmax over the k picks     */
+/* ------------------------------------------------------------------ */
+/* Experts are ordered by (logit descending, expert id ascending); the k
+ * first ones are the picks, in that order.  The weights are the softmax
+ * of the k picked logits, which equals the full softmax over E restricted
+ * to the picks and renormalised.  Returns 0. */
+int oracle_route_topk(const float* logits, int64_t T, int32_t E, int32_t k,
+                      int32_t* topk_idx, float* topk_w) {
+    unsigned char* taken = (unsigned char*)malloc(E > 0 ? (size_t)E : 1u);
+    double* z = (double*)malloc(sizeof(double) * (k > 0 ? (size_t)k : 1u));
+    for (int64_t t = 0; t < T; ++t) {
+        const float* L = logits + t * E;
+        memset(taken, 0, (size_t)E);
+        for (int32_t j = 0; j < k; ++j) {          /* k rounds of argmax */
+            int32_t best = -1;
+            for (int32_t e = 0; e < E; ++e) {
+                if (taken[e]) continue;
+                if (best < 0 || L[e] > L[best]) best = e;  /* ties keep lower id */
+            }
+            taken[best] = 1;
+            topk_idx[t * k + j] = best;
+        }
+        double m = (double)L[topk_idx[t * k]];
+        double sum = 0.0;
+        for (int32_t j = 0; j < k; ++j) {
+            z[j] = exp((double)L[topk_idx[t * k + j]] - m);
+            sum += z[j];
+        }
+        for (int32_t j = 0; j < k; ++j) topk_w[t * k + j] = (float)(z[j] / sum);
+    }
+    free(taken);
+    free(z);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* S2 dispatch layout: histogram, exclusive scan, stable counting sort */
+/* ------------------------------------------------------------------ */
+/* Pair p = t*k + j goes to expert idx[p].  Slots are expert-major, ties by
+ * pair index (a stable sort by destination, as the aiwiki sketch's argsort
+ * read as stable); logical rank r's slab starts at the offset of its first
+ * expert r*E/W.  Pairs whose expert id is outside [0, E) are skipped:
+ * slot_of_pair = -1, and slots past the last valid one hold -1.  Returns
+ * the number of skipped pairs. */
+int64_t oracle_dispatch_layout(const int32_t* idx, int64_t T, int32_t k, int32_t E,
+                               int32_t W, int32_t* counts, int32_t* offsets,
+                               int32_t* rank_offsets, int32_t* slot_of_pair,
+                               int32_t* pair_of_slot) {
+    int64_t N = T * k, bad = 0;
+    for (int32_t e = 0; e < E; ++e) counts[e] = 0;
+    for (int64_t p = 0; p < N; ++p) {
+        int32_t e = idx[p];
+        if (e < 0 || e >= E) { ++bad; continue; }
+        counts[e] += 1;
+    }
+    offsets[0] = 0;
+    for (int32_t e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + counts[e];
+    for (int32_t r = 0; r <= W; ++r) rank_offsets[r] = offsets[(int64_t)r * E / W];
+    int32_t* fill = (int32_t*)calloc(E > 0 ? (size_t)E : 1u, sizeof(int32_t));
+    for (int64_t p = 0; p < N; ++p) {
+        int32_t e = idx[p];
+        if (e < 0 || e >= E) { slot_of_pair[p] = -1; continue; }
+        int32_t s = offsets[e] + fill[e]++;
+        slot_of_pair[p] = s;
+        pair_of_slot[s] = (int32_t)p;
+    }
+    for (int64_t s = offsets[E]; s < N; ++s) pair_of_slot[s] = -1;
+    free(fill);
+    return bad;
+}
+
+/* ------------------------------------------------------------------ */
+/* S3 permute: xp[s] = x[pair_of_slot[s] / k], optional FP8 payload     */
+/* ------------------------------------------------------------------ */
+/* Same-dtype payload: a bitwise row copy.  FP8 payload: for every
+ * 128-element block of the token's row, scale = amax / 448 (fp32 IEEE
+ * division; 1 when amax is 0) and q = e4m3(x / scale) (fp32 IEEE division,
+ * then round-to-nearest-even with saturation).  Slots holding -1 are not
+ * written.  Returns 0, or -1 for an unsupported dtype pair. */
+int oracle_permute(const void* x, int x_dt, int64_t T, int32_t H, int32_t k,
+                   const int32_t* pair_of_slot, int64_t n_slots, void* xp, int xp_dt,
+                   float* xp_scales) {
+    (void)T;
+    size_t eb = (x_dt == OR_F32) ? 4 : 2;
+    if (xp_dt == x_dt) {
+        for (int64_t s = 0; s < n_slots; ++s) {
+            int32_t p = pair_of_slot[s];
+            if (p < 0) continue;
+            memcpy((char*)xp + (size_t)s * H * eb, (const char*)x + (size_t)(p / k) * H * eb,
+                   (size_t)H * eb);
+        }
+        return 0;
+    }
+    if (xp_dt != OR_E4M3 || (H % 128) != 0) return -1;
+    int32_t nb = H / 128;
+    for (int64_t s = 0; s < n_slots; ++s) {
+        int32_t p = pair_of_slot[s];
+        if (p < 0) continue;
+        int64_t t = p / k;
+        for (int32_t b = 0; b < nb; ++b) {
+            float amax = 0.0f;
+            for (int32_t i = 0; i < 128; ++i) {
+                float v = (float)load_elem(x, x_dt, t * H + b * 128 + i);
+                if (fabsf(v) > amax) amax = fabsf(v);
+            }
+            float scale = amax / 448.0f;
+            if (scale == 0.0f) scale = 1.0f;
+            xp_scales[s * nb + b] = scale;
+            for (int32_t i = 0; i < 128; ++i) {
+                float v = (float)load_elem(x, x_dt, t * H + b * 128 + i);
+                float r = v / scale;
+                ((uint8_t*)xp)[s * H + b * 128 + i] = e4m3_from_float(r);
+            }
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* S4 grouped SwiGLU expert FFN                                        */
+/* ------------------------------------------------------------------ */
+/* For local expert j (global e = expert_begin + j) and every slot s in
+ * [offsets[e], offsets[e+1]):
+ *     g_i = sum_h A[s,h] W13[j, i, h],  u_i = sum_h A[s,h] W13[j, I+i, h]
+ *     h_i = silu(g_i) * u_i,  silu(g) = g / (1 + exp(-g))
+ *     y_o = sum_i h_i W2[j, o, i]
+ * A is the payload row as a real number; for the FP8 payload it is the
+ * bf16 rounding of the fp32 product decode(q) * scale.  h and y are
+ * stored (rounded once) in the weight dtype, and y is computed from the
+ * stored h.  row_mask (indexed by slot, may be NULL) restricts the work to
+ * a sample of rows.  Returns the number of rows computed. */
+int64_t oracle_grouped_gemm(const void* xp, int xp_dt, const float* xp_scales,
+                            const int32_t* offsets, int32_t expert_begin,
+                            int32_t n_experts, int32_t H, int32_t I, const void* w13,
+                            const void* w2, int w_dt, const uint8_t* row_mask, void* h,
+                            void* y) {
+    int64_t s_lo = offsets[expert_begin], s_hi = offsets[expert_begin + n_experts];
+    int64_t done = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(+ : done)
+    for (int64_t s = s_lo; s < s_hi; ++s) {
+        if (row_mask && !row_mask[s]) continue;
+        int32_t j = expert_begin;
+        while (offsets[j + 1] <= s) ++j;          /* expert owning slot s */
+        j -= expert_begin;
+        double* a = (double*)malloc(sizeof(double) * (size_t)H);
+        double* hv = (double*)malloc(sizeof(double) * (size_t)I);
+        for (int32_t c = 0; c < H; ++c) {
+            if (xp_dt == OR_E4M3) {
+                float dq = (float)e4m3_to_double(((const uint8_t*)xp)[s * H + c]);
+                float prod = dq * xp_scales[s * (H / 128) + c / 128];
+                a[c] = bf16_to_double(bf16_from_double((double)prod));
+            } else {
+                a[c] = load_elem(xp, xp_dt, s * H + c);
+            }
+        }
+        int64_t w13_base = (int64_t)j * 2 * I * H, w2_base = (int64_t)j * H * I;
+        for (int32_t i = 0; i < I; ++i) {
+            double g = 0.0, u = 0.0;
+            for (int32_t c = 0; c < H; ++c) {
+                g += a[c] * load_elem(w13, w_dt, w13_base + (int64_t)i * H + c);
+                u += a[c] * load_elem(w13, w_dt, w13_base + (int64_t)(I + i) * H + c);
+            }
+            double v = g / (1.0 + exp(-g)) * u;
+            store_elem(h, w_dt, s * I + i, v);
+            hv[i] = load_elem(h, w_dt, s * I + i);   /* y uses the stored h */
+        }
+        for (int32_t o = 0; o < H; ++o) {
+            double acc = 0.0;
+            for (int32_t i = 0; i < I; ++i)
+                acc += hv[i] * load_elem(w2, w_dt, w2_base + (int64_t)o * I + i);
+            store_elem(y, w_dt, s * H + o, acc);
+        }
+        free(a);
+        free(hv);
+        done += 1;
+    }
+    return done;
+}
+
+/* ------------------------------------------------------------------ */
+/* S5 combine: out[t] = sum_j w[t,j] * y[slot_of_pair[t*k+j]]          */
+/* ------------------------------------------------------------------ */
+/* The un-permute of the aiwiki sketch (y[order] = back) fused with the
+ * router-weighted sum into the token's home row.  Skipped pairs (slot -1)
+ * add nothing.  Returns 0. */
+int oracle_combine(const void* y, int y_dt, const int32_t* slot_of_pair,
+                   const float* topk_w, int64_t T, int32_t k, int32_t H, void* out,
+                   int out_dt) {
+    double* acc = (double*)malloc(sizeof(double) * (size_t)H);
+    for (int64_t t = 0; t < T; ++t) {
+        for (int32_t c = 0; c < H; ++c) acc[c] = 0.0;
+        for (int32_t j = 0; j < k; ++j) {
+            int32_t s = slot_of_pair[t * k + j];
+            if (s < 0) continue;
+            double w = (double)topk_w[t * k + j];
+            for (int32_t c = 0; c < H; ++c) acc[c] += w * load_elem(y, y_dt, (int64_t)s * H + c);
+        }
+        for (int32_t c = 0; c < H; ++c) store_elem(out, out_dt, t * H + c, acc[c]);
+    }
+    free(acc);
+    return 0;
+}
