@@ -21,9 +21,10 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "moe_oracle.c")
 _LIB = os.path.join(_HERE, "libmoe_oracle.so")
 
-F32, BF16, E4M3 = 0, 1, 2
-_CODE = {"f32": F32, "bf16": BF16, "e4m3": E4M3}
-_TDT = {"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.float8_e4m3fn}
+F32, BF16, E4M3, F64 = 0, 1, 2, 3
+_CODE = {"f32": F32, "bf16": BF16, "e4m3": E4M3, "f64": F64}
+_TDT = {"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.float8_e4m3fn,
+        "f64": torch.float64}
 
 _lib = None
 
@@ -49,7 +50,7 @@ def _load():
         lib.oracle_dispatch_layout.restype = I64
         lib.oracle_permute.argtypes = [P, I, I64, I32, I32, P, I64, P, I, P]
         lib.oracle_permute.restype = I
-        lib.oracle_grouped_gemm.argtypes = [P, I, P, P, I32, I32, I32, I32, P, P, I, P, P, P]
+        lib.oracle_grouped_gemm.argtypes = [P, I, P, P, I32, I32, I32, I32, P, P, I, P, P, P, I]
         lib.oracle_grouped_gemm.restype = I64
         lib.oracle_combine.argtypes = [P, I, P, P, I64, I32, I32, P, I]
         lib.oracle_combine.restype = I
@@ -148,27 +149,33 @@ def permute(x: torch.Tensor, k: int, pair_of_slot: torch.Tensor, payload: str,
 
 def grouped_gemm(xp: torch.Tensor, xp_scales, expert_offsets: torch.Tensor,
                  expert_begin: int, n_experts: int, w13: torch.Tensor, w2: torch.Tensor,
-                 row_mask: torch.Tensor | None = None):
-    """Returns (h, y, rows_done); rows outside the mask (or outside the
+                 row_mask: torch.Tensor | None = None, out: str = "f64"):
+    """Returns (h, y, rows_done).  h and y come back in ``out``: "f64" =
+    unrounded (the default: what parity compares against), or the weight
+    dtype's storage rounding.  The down projection always consumes h
+    rounded to the weight dtype.  Rows outside the mask (or outside the
     experts' segments) are left as NaN."""
     xp = xp.contiguous()
     n_rows, H = xp.shape
     I = w2.shape[2]
     wdt = _dt_name(w13)
-    h = torch.full((n_rows, I), float("nan"), dtype=_TDT[wdt])
-    y = torch.full((n_rows, H), float("nan"), dtype=_TDT[wdt])
+    h = torch.full((n_rows, I), float("nan"), dtype=_TDT[out])
+    y = torch.full((n_rows, H), float("nan"), dtype=_TDT[out])
     mask = None if row_mask is None else row_mask.to(torch.uint8).contiguous()
     xdt = _dt_name(xp)
     done = _load().oracle_grouped_gemm(
         _p(xp.view(torch.uint8) if xdt == "e4m3" else xp), _CODE[xdt],
         _p(xp_scales.contiguous() if xp_scales is not None else None),
         _p(expert_offsets.to(torch.int32).contiguous()), expert_begin, n_experts, H, I,
-        _p(w13.contiguous()), _p(w2.contiguous()), _CODE[wdt], _p(mask), _p(h), _p(y))
+        _p(w13.contiguous()), _p(w2.contiguous()), _CODE[wdt], _p(mask), _p(h), _p(y),
+        _CODE[out])
     return h, y, int(done)
 
 
 def combine(y: torch.Tensor, slot_of_pair: torch.Tensor, topk_w: torch.Tensor,
-            out_dtype: str):
+            out_dtype: str = "f64"):
+    """Weighted sum of each token's k rows of y (in y's own dtype, i.e.
+    as the path stores it), in fp64; "f64" returns it unrounded."""
     y = y.contiguous()
     T, k = topk_w.shape
     H = y.shape[1]
@@ -179,15 +186,27 @@ def combine(y: torch.Tensor, slot_of_pair: torch.Tensor, topk_w: torch.Tensor,
     return out
 
 
+def round_to(v: torch.Tensor, dtype: str) -> torch.Tensor:
+    """fp64 values rounded to a storage type with the oracle's own rounding."""
+    if dtype == "bf16":
+        return bf16_round(v)
+    if dtype == "f32":
+        return v.to(torch.float32)      # IEEE round-to-nearest-even
+    return v
+
+
 def layer(wl, inputs, row_mask=None):
     """The whole hot path on one workload's inputs; returns every
-    intermediate (dict).  ``row_mask`` (per slot) samples the GEMM rows;
-    combine is then only meaningful for tokens whose pairs were all
-    computed."""
+    intermediate (dict).  h, y and out are unrounded (fp64); ``y_stored`` is
+    y in its storage type, which is what combine consumes.  ``row_mask``
+    (per slot) samples the GEMM rows; combine is then only meaningful for
+    tokens whose pairs were all computed."""
     idx, w = route_topk(inputs["logits"], wl.k)
     lay = dispatch_layout(idx, wl.E, wl.W)
     xp, sc = permute(inputs["x"], wl.k, lay["pair_of_slot"], wl.payload)
     h, y, _ = grouped_gemm(xp, sc, lay["expert_offsets"], 0, wl.E, inputs["w13"], inputs["w2"],
                            row_mask)
-    out = combine(y, lay["slot_of_pair"], w, wl.act)
-    return dict(topk_idx=idx, topk_w=w, xp=xp, xp_scales=sc, h=h, y=y, out=out, **lay)
+    y_stored = round_to(y, wl.wdt)
+    out = combine(y_stored, lay["slot_of_pair"], w)
+    return dict(topk_idx=idx, topk_w=w, xp=xp, xp_scales=sc, h=h, y=y, y_stored=y_stored,
+                out=out, **lay)

@@ -14,8 +14,13 @@
  *   - the FP8 payload's scale and quotient are fp32 IEEE divisions, because
  *     they decide an integer code (the quantised byte) and the CUDA side
  *     decides it in fp32 as well;
- *   - every stored tensor (topk weights, h, y, out) is rounded once, from
- *     the fp64 result, to its storage type.
+ *   - a value the path stores and then consumes again is rounded, as the
+ *     path stores it, before it is consumed: h (bf16 or fp32) before the
+ *     down projection, y before the combine (the caller passes y in its
+ *     storage type);
+ *   - the results a caller compares (h, y, out) can be returned unrounded
+ *     in fp64 (dtype code 3), i.e. before their own storage rounding; the
+ *     router weights are returned in fp32, their storage type.
  *
  * Sources (page title, section):
  *   "Expert parallelism and all-to-all", "Walking through one MoE layer":
@@ -29,7 +34,8 @@
  *   "Expert parallelism and all-to-all", "Traffic math": 1-byte FP8
  *       activation payload.
  *
- * dtype codes: 0 = fp32, 1 = bf16 (uint16 bits), 2 = FP8 e4m3 (OCP, "fn").
+ * dtype codes: 0 = fp32, 1 = bf16 (uint16 bits), 2 = FP8 e4m3 (OCP, "fn"),
+ * 3 = fp64 (results only).
  */
 #include <math.h>
 #include <stdint.h>
@@ -39,6 +45,7 @@
 #define OR_F32 0
 #define OR_BF16 1
 #define OR_E4M3 2
+#define OR_F64 3
 
 /* ------------------------------------------------------------------ */
 /* number formats, written from their definitions                      */
@@ -120,12 +127,19 @@ static double load_elem(const void* base, int dt, int64_t i) {
     switch (dt) {
         case OR_F32: return (double)((const float*)base)[i];
         case OR_BF16: return bf16_to_double(((const uint16_t*)base)[i]);
+        case OR_F64: return ((const double*)base)[i];
         default: return e4m3_to_double(((const uint8_t*)base)[i]);
     }
 }
 
+/* v rounded to storage type dt (fp32 or bf16), as a double */
+static double round_to(int dt, double v) {
+    return dt == OR_F32 ? (double)(float)v : bf16_to_double(bf16_from_double(v));
+}
+
 static void store_elem(void* base, int dt, int64_t i, double v) {
-    if (dt == OR_F32) ((float*)base)[i] = (float)v;
+    if (dt == OR_F64) ((double*)base)[i] = v;
+    else if (dt == OR_F32) ((float*)base)[i] = (float)v;
     else ((uint16_t*)base)[i] = bf16_from_double(v);
 }
 
@@ -268,15 +282,16 @@ int oracle_permute(const void* x, int x_dt, int64_t T, int32_t H, int32_t k,
  *     h_i = silu(g_i) * u_i,  silu(g) = g / (1 + exp(-g))
  *     y_o = sum_i h_i W2[j, o, i]
  * A is the payload row as a real number; for the FP8 payload it is the
- * bf16 rounding of the fp32 product decode(q) * scale.  h and y are
- * stored (rounded once) in the weight dtype, and y is computed from the
- * stored h.  row_mask (indexed by slot, may be NULL) restricts the work to
- * a sample of rows.  Returns the number of rows computed. */
+ * bf16 rounding of the fp32 product decode(q) * scale.  The down
+ * projection consumes h rounded to the weight dtype (as the path stores
+ * it); h and y are written in out_dt (fp64 = unrounded, or a storage type).
+ * row_mask (indexed by slot, may be NULL) restricts the work to a sample
+ * of rows.  Returns the number of rows computed. */
 int64_t oracle_grouped_gemm(const void* xp, int xp_dt, const float* xp_scales,
                             const int32_t* offsets, int32_t expert_begin,
                             int32_t n_experts, int32_t H, int32_t I, const void* w13,
                             const void* w2, int w_dt, const uint8_t* row_mask, void* h,
-                            void* y) {
+                            void* y, int out_dt) {
     int64_t s_lo = offsets[expert_begin], s_hi = offsets[expert_begin + n_experts];
     int64_t done = 0;
 #pragma omp parallel for schedule(dynamic, 1) reduction(+ : done)
@@ -304,14 +319,14 @@ int64_t oracle_grouped_gemm(const void* xp, int xp_dt, const float* xp_scales,
                 u += a[c] * load_elem(w13, w_dt, w13_base + (int64_t)(I + i) * H + c);
             }
             double v = g / (1.0 + exp(-g)) * u;
-            store_elem(h, w_dt, s * I + i, v);
-            hv[i] = load_elem(h, w_dt, s * I + i);   /* y uses the stored h */
+            store_elem(h, out_dt, s * I + i, v);
+            hv[i] = round_to(w_dt, v);                 /* the down projection reads stored h */
         }
         for (int32_t o = 0; o < H; ++o) {
             double acc = 0.0;
             for (int32_t i = 0; i < I; ++i)
                 acc += hv[i] * load_elem(w2, w_dt, w2_base + (int64_t)o * I + i);
-            store_elem(y, w_dt, s * H + o, acc);
+            store_elem(y, out_dt, s * H + o, acc);
         }
         free(a);
         free(hv);
@@ -324,8 +339,8 @@ int64_t oracle_grouped_gemm(const void* xp, int xp_dt, const float* xp_scales,
 /* S5 combine: out[t] = sum_j w[t,j] * y[slot_of_pair[t*k+j]]          */
 /* ------------------------------------------------------------------ */
 /* The un-permute of the aiwiki sketch (y[order] = back) fused with the
- * router-weighted sum into the token's home row.  Skipped pairs (slot -1)
- * add nothing.  Returns 0. */
+ * router-weighted sum into the token's home row, in fp64; out_dt fp64
+ * returns it unrounded.  Skipped pairs (slot -1) add nothing.  Returns 0. */
 int oracle_combine(const void* y, int y_dt, const int32_t* slot_of_pair,
                    const float* topk_w, int64_t T, int32_t k, int32_t H, void* out,
                    int out_dt) {
