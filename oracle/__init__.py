@@ -174,8 +174,8 @@ def grouped_gemm(xp: torch.Tensor, xp_scales, expert_offsets: torch.Tensor,
 
 def combine(y: torch.Tensor, slot_of_pair: torch.Tensor, topk_w: torch.Tensor,
             out_dtype: str = "f64"):
-    """Weighted sum of each token's k rows of y (in y's own dtype, i.e.
-    as the path stores it), in fp64; "f64" returns it unrounded."""
+    """Weighted sum of each token's k rows of y (read in y's own dtype), in
+    fp64; "f64" returns it unrounded."""
     y = y.contiguous()
     T, k = topk_w.shape
     H = y.shape[1]
@@ -197,16 +197,14 @@ def round_to(v: torch.Tensor, dtype: str) -> torch.Tensor:
 
 def layer(wl, inputs, row_mask=None):
     """The whole hot path on one workload's inputs; returns every
-    intermediate (dict).  h, y and out are unrounded (fp64); ``y_stored`` is
-    y in its storage type, which is what combine consumes.  ``row_mask``
-    (per slot) samples the GEMM rows; combine is then only meaningful for
-    tokens whose pairs were all computed."""
+    intermediate (dict).  h, y and out are unrounded (fp64): out is the
+    weighted sum of the exact y.  ``row_mask`` (per slot) samples the GEMM
+    rows; combine is then only meaningful for tokens whose pairs were all
+    computed."""
     idx, w = route_topk(inputs["logits"], wl.k)
     lay = dispatch_layout(idx, wl.E, wl.W)
     xp, sc = permute(inputs["x"], wl.k, lay["pair_of_slot"], wl.payload)
     h, y, _ = grouped_gemm(xp, sc, lay["expert_offsets"], 0, wl.E, inputs["w13"], inputs["w2"],
                            row_mask)
-    y_stored = round_to(y, wl.wdt)
-    out = combine(y_stored, lay["slot_of_pair"], w)
-    return dict(topk_idx=idx, topk_w=w, xp=xp, xp_scales=sc, h=h, y=y, y_stored=y_stored,
-                out=out, **lay)
+    out = combine(y, lay["slot_of_pair"], w)
+    return dict(topk_idx=idx, topk_w=w, xp=xp, xp_scales=sc, h=h, y=y, out=out, **lay)

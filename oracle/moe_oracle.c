@@ -14,13 +14,13 @@
  *   - the FP8 payload's scale and quotient are fp32 IEEE divisions, because
  *     they decide an integer code (the quantised byte) and the CUDA side
  *     decides it in fp32 as well;
- *   - a value the path stores and then consumes again is rounded, as the
- *     path stores it, before it is consumed: h (bf16 or fp32) before the
- *     down projection, y before the combine (the caller passes y in its
- *     storage type);
- *   - the results a caller compares (h, y, out) can be returned unrounded
- *     in fp64 (dtype code 3), i.e. before their own storage rounding; the
- *     router weights are returned in fp32, their storage type.
+ *   - an operand the layer defines in a narrow type is rounded to it:
+ *     the expert GEMMs take bf16 (or fp32) operands, so h is rounded to the
+ *     weight dtype before the down projection;
+ *   - everything else is exact: the results a caller compares (h, y, out)
+ *     are returned unrounded in fp64 (dtype code 3), and combine sums y as
+ *     given (fp64 y from the GEMM for the exact layer output); the router
+ *     weights are returned in fp32, their storage type.
  *
  * Sources (page title, section):
  *   "Expert parallelism and all-to-all", "Walking through one MoE layer":

@@ -270,10 +270,9 @@ def test_layer_matches_plain_torch_fp64_tiny():
         y[m] = h @ w2.T
     rel = lambda a, b: float(((a - b).abs() / b.pow(2).mean(1, keepdim=True).sqrt()).max())
     assert rel(r["y"], y) < 1e-12
-    y32 = y.float().double()                                          # y as stored (fp32)
     out = torch.zeros(wl.T, wl.H, dtype=torch.float64)
-    out.index_add_(0, perm // wl.k, y32 * r["topk_w"].double().reshape(-1)[perm][:, None])
-    assert rel(r["out"], out) < 1e-6
+    out.index_add_(0, perm // wl.k, y * r["topk_w"].double().reshape(-1)[perm][:, None])
+    assert rel(r["out"], out) < 1e-12
 
 
 def test_traffic_worked_example():
