@@ -1,0 +1,381 @@
+#!/usr/bin/env python3
+"""Benchmark of the single-GPU MoE-layer hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload dsv3]
+                    [--impl ours|reference] [--no-cpu-baseline]
+
+One step = one pass of the whole hot path (router top-k -> dispatch layout
+-> permute -> grouped SwiGLU GEMM -> combine) over one batch of the
+workload, inputs resident in HBM.  L2 is flushed (a 512 MiB write) before
+every step, outside the step's CUDA events.  With N > 1 (torchrun), every
+rank runs an independent replica of the layer on its own GPU (no
+collective on the data path: weak scaling); the per-step time is the max
+over ranks.  Rank 0 prints one JSON line.
+
+``--impl reference`` times the CPU oracle instead (the only other place
+that runs it), on a bounded token sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from expert_parallelism_b200 import moe, traffic, workloads  # noqa: E402
+
+METRIC = "MoE-layer tokens/s (dispatch+grouped GEMM+combine); permute/combine HBM GB/s"
+L2_FLUSH_BYTES = 512 << 20
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p["bf16_tflops_sustained"], "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ---------------------------------------------------------------- CPU oracle leg
+def oracle_sample(wl, target_s: float = 12.0, max_tokens: int | None = None):
+    """Time the CPU oracle on a token sample of the workload: all five steps
+    for the first S tokens (route, layout, permute, GEMM, combine).  S grows
+    (doubling) until the oracle's own time reaches ``target_s``/2; expert
+    weights are drawn on the host outside the timed calls."""
+    import oracle
+    logits_all = workloads.router_logits(wl)
+    x_all = workloads.hidden_states(wl)
+    cache = {}
+
+    def run(S):
+        sub = wl.replace(T=S)
+        lg, x = logits_all[:S].contiguous(), x_all[:S].contiguous()
+        t0 = time.perf_counter()
+        idx, w = oracle.route_topk(lg, wl.k)
+        lay = oracle.dispatch_layout(idx, wl.E, wl.W)
+        xp, sc = oracle.permute(x, wl.k, lay["pair_of_slot"], wl.payload)
+        el = time.perf_counter() - t0
+        off = lay["expert_offsets"].tolist()
+        touched = [e for e in range(wl.E) if off[e + 1] > off[e]]
+        for e in touched:
+            if e not in cache:
+                cache[e] = (workloads.expert_w13(wl, e), workloads.expert_w2(wl, e))
+        y = torch.empty(sub.N, wl.H, dtype=torch.float64)
+        for i in range(0, len(touched), 32):
+            grp = touched[i:i + 32]
+            rows = torch.cat([torch.arange(off[e], off[e + 1]) for e in grp])
+            oe = torch.tensor([0] + list(torch.tensor([off[e + 1] - off[e] for e in grp])
+                                         .cumsum(0).tolist()), dtype=torch.int32)
+            a13 = torch.stack([cache[e][0] for e in grp])
+            a2 = torch.stack([cache[e][1] for e in grp])
+            t0 = time.perf_counter()
+            _, ye, _ = oracle.grouped_gemm(xp[rows].contiguous(),
+                                           sc[rows].contiguous() if sc is not None else None,
+                                           oe, 0, len(grp), a13, a2)
+            el += time.perf_counter() - t0
+            y[rows] = ye
+        t0 = time.perf_counter()
+        oracle.combine(y, lay["slot_of_pair"], w, wl.act)
+        el += time.perf_counter() - t0
+        return el
+
+    S = 4
+    el = run(S)
+    cap = wl.T if max_tokens is None else min(wl.T, max_tokens)
+    while el < target_s / 2 and S < cap:
+        S = min(cap, S * 2)
+        cache_keep = len(cache)
+        el = run(S)
+        if len(cache) > 400 and cache_keep:
+            cache.clear()
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": S / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {S} of {wl.T} tokens of workload {wl.name}, all five steps "
+                      f"(fp64 C oracle, OpenMP over GEMM rows); {el:.2f} s of oracle time"}
+
+
+def run_reference(args, wl):
+    ws, rank, local = _dist()
+    if rank != 0:
+        return
+    times = []
+    for _ in range(args.warmup):
+        oracle_sample(wl, target_s=2.0, max_tokens=8)
+    res = None
+    for _ in range(args.steps):
+        res = oracle_sample(wl, target_s=args.ref_seconds)
+        times.append(1.0 / res["value"] * wl.T)
+    v = res["value"]
+    line = {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * wl.T / v,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": _config(wl), "cpu_baseline": res,
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def _config(wl):
+    return {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "I": wl.I,
+            "logical_ranks": wl.W, "activations": wl.act, "payload": wl.payload,
+            "gemm": wl.wdt, "router": wl.router, "seed": wl.seed,
+            "l2": f"flushed ({L2_FLUSH_BYTES >> 20} MiB write) before every step",
+            "parallelism": "replicas (one independent layer per GPU)"}
+
+
+# ---------------------------------------------------------------- GPU leg
+def run_ours(args, wl):
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    lib = moe.load_library()
+    inp = workloads.layer_inputs(wl, with_weights=False, device="cpu")
+    logits, x = inp["logits"].to(dev), inp["x"].to(dev)
+    wdt = workloads.TORCH_DTYPE[wl.wdt]
+    w13 = torch.empty(wl.E, 2 * wl.I, wl.H, dtype=wdt, device=dev)
+    w2 = torch.empty(wl.E, wl.H, wl.I, dtype=wdt, device=dev)
+    workloads.fill_expert_weights(wl, w13, w2)
+    buf = moe.LayerBuffers(wl, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    names = ["route_topk", "dispatch_layout", "permute", "grouped_gemm", "combine"]
+
+    def step(evs):
+        evs[0].record(stream)
+        moe.moe_route_topk(logits, buf.topk_idx, buf.topk_w)
+        evs[1].record(stream)
+        moe.moe_dispatch_layout(buf.topk_idx, wl.E, wl.W, buf.expert_counts, buf.expert_offsets,
+                                buf.rank_offsets, buf.slot_of_pair, buf.pair_of_slot,
+                                buf.layout_ws, buf.dev_status)
+        evs[2].record(stream)
+        moe.moe_permute(x, wl.k, buf.slot_of_pair, buf.xp, buf.xp_scales)
+        evs[3].record(stream)
+        moe.moe_grouped_gemm(buf.xp, buf.xp_scales, buf.expert_offsets, 0, wl.E, w13, w2, buf.h,
+                             buf.y, buf.gemm_ws, buf.dev_status)
+        evs[4].record(stream)
+        moe.moe_combine(buf.y, buf.slot_of_pair, buf.topk_w, buf.out)
+        evs[5].record(stream)
+
+    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step(mk())
+    torch.cuda.synchronize()
+    st = moe.moe_check_status(buf.dev_status)
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {moe.STATUS.get(st, st)}")
+
+    launches0 = lib.moe_launch_count()
+    all_evs = [mk() for _ in range(args.steps)]
+    if ws > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.fill_(1)
+            step(all_evs[i])
+        torch.cuda.synchronize()
+    if ws > 1:
+        torch.distributed.barrier()
+    launches = (lib.moe_launch_count() - launches0) // max(args.steps, 1)
+    per = {n: [] for n in names}
+    step_ms = []
+    for evs in all_evs:
+        for j, n in enumerate(names):
+            per[n].append(evs[j].elapsed_time(evs[j + 1]))
+        step_ms.append(evs[0].elapsed_time(evs[5]))
+    ms = statistics.mean(step_ms)
+    layer_ms = ms - statistics.mean(per["route_topk"])      # dispatch + GEMM + combine
+    if ws > 1:
+        t = torch.tensor([ms, layer_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms, layer_ms = float(t[0]), float(t[1])
+
+    # end to end through the C ABI from pinned host buffers
+    h_logits = inp["logits"].pin_memory()
+    h_x = inp["x"].pin_memory()
+    h_out = torch.empty(buf.out.shape, dtype=buf.out.dtype).pin_memory()
+    e2e_ms = []
+    for i in range(args.warmup + args.steps):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        logits.copy_(h_logits, non_blocking=True)
+        x.copy_(h_x, non_blocking=True)
+        moe.layer_forward(wl, logits, x, w13, w2, buf)
+        h_out.copy_(buf.out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(e0.elapsed_time(e1))
+    e2e = statistics.mean(e2e_ms)
+    if ws > 1:
+        t = torch.tensor([e2e], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e = float(t[0])
+    st = moe.moe_check_status(buf.dev_status)
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {moe.STATUS.get(st, st)}")
+
+    if rank == 0:
+        peaks = _peaks()
+        kb = traffic.kernel_bytes(wl)
+        fl = traffic.gemm_flops(wl)
+        avg = {n: statistics.mean(v) for n, v in per.items()}
+        gemm_tflops = fl["total"] / (avg["grouped_gemm"] * 1e-3) / 1e12
+        counts = buf.expert_counts.cpu()
+        touched = int((counts > 0).sum())
+        kernels = {
+            "route_topk": {"us": avg["route_topk"] * 1e3,
+                           "gbs": kb["route_topk"] / (avg["route_topk"] * 1e-3) / 1e9},
+            "dispatch_layout": {"us": avg["dispatch_layout"] * 1e3},
+            "permute": {"us": avg["permute"] * 1e3, "bytes": kb["permute"],
+                        "gbs": kb["permute"] / (avg["permute"] * 1e-3) / 1e9},
+            "grouped_gemm": {"us": avg["grouped_gemm"] * 1e3, "flops": fl["total"],
+                             "tflops": gemm_tflops,
+                             "weight_gbs": traffic.touched_weight_bytes(wl, touched)
+                             / (avg["grouped_gemm"] * 1e-3) / 1e9,
+                             "experts_touched": touched},
+            "combine": {"us": avg["combine"] * 1e3, "bytes": kb["combine"],
+                        "gbs": kb["combine"] / (avg["combine"] * 1e-3) / 1e9},
+        }
+        for n in ["permute", "combine", "route_topk"]:
+            kernels[n]["hbm_frac"] = kernels[n]["gbs"] / peaks["hbm_gbs"]
+        prof = _profile_traffic()
+        roof = {"kernel": "grouped_gemm (gate/up + SwiGLU, then down)", "bound": "tensor",
+                "achieved": gemm_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": gemm_tflops / peaks["bf16_tflops"], "traffic": prof,
+                "peak_source": peaks["source"] + " burst bf16 (timed per call)"}
+        line = {
+            "metric": METRIC, "value": ws * wl.T / (ms * 1e-3), "unit": "tokens/s",
+            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": _config(wl),
+            "layer_tokens_per_s": ws * wl.T / (layer_ms * 1e-3),
+            "layer_ms_excl_route": layer_ms,
+            "kernels": kernels, "roofline": roof,
+            "e2e": {"value": ws * wl.T / (e2e * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h_logits.numel() * 4 + h_x.numel() * h_x.element_size(),
+                    "d2h_bytes_per_step": h_out.numel() * h_out.element_size(),
+                    "ms_per_step": e2e},
+            "gpu_launches": int(launches), "clocks": clk.summary(),
+        }
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = oracle_sample(wl)
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+def _profile_traffic():
+    """DRAM bytes per launch of the GEMM from the committed ncu summary, if
+    one matching the current kernel is recorded there."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            return json.load(f).get("grouped_gemm_bytes_per_launch")
+    except Exception:
+        return None
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="dsv3", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    wl = workloads.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    main()

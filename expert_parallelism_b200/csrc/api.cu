@@ -1,0 +1,191 @@
+// api.cu -- the extern "C" boundary of libmoe (declared in include/moe.h).
+//
+// Every entry point validates its arguments on the host first and returns
+// MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED before anything is enqueued,
+// then launches its kernels on the caller's stream and returns without
+// waiting.  Nothing here allocates or frees device memory.
+#include <stdio.h>
+
+#include <atomic>
+
+#include "common.cuh"
+
+namespace moe {
+cudaError_t launch_route_topk(const float*, int64_t, int, int, int32_t*, float*, cudaStream_t);
+size_t layout_workspace_bytes(int64_t T, int k, int E);
+cudaError_t launch_dispatch_layout(const int32_t*, int64_t, int, int, int, int32_t*, int32_t*,
+                                   int32_t*, int32_t*, int32_t*, void*, int32_t*, cudaStream_t);
+cudaError_t launch_permute(const void*, moe_dtype, int64_t, int, int, const int32_t*, void*,
+                           moe_dtype, float*, cudaStream_t);
+cudaError_t launch_combine(const void*, moe_dtype, const int32_t*, const float*, int64_t, int,
+                           int, void*, moe_dtype, cudaStream_t);
+cudaError_t launch_dequant_e4m3(const uint8_t*, const float*, const int32_t*, int, int, int64_t,
+                                int, __nv_bfloat16*, cudaStream_t);
+cudaError_t launch_grouped_gemm_simt_f32(const float*, const int32_t*, int, int, int64_t, int,
+                                         int, const float*, const float*, float*, float*,
+                                         cudaStream_t);
+cudaError_t launch_grouped_gemm_tc(const __nv_bfloat16*, const int32_t*, int, int, int64_t, int,
+                                   int, const __nv_bfloat16*, const __nv_bfloat16*,
+                                   __nv_bfloat16*, __nv_bfloat16*, int32_t*, cudaStream_t);
+}  // namespace moe
+
+namespace moe {
+static std::atomic<uint64_t> g_launches{0};
+void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+bool is_act_dtype(moe_dtype d) { return d == MOE_F32 || d == MOE_BF16; }
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+moe_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return MOE_OK;
+    fprintf(stderr, "libmoe: CUDA error: %s\n", cudaGetErrorString(e));
+    return MOE_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_route_topk(const float* logits, int64_t T, int32_t E, int32_t k,
+                          int32_t* topk_idx, float* topk_w, void* stream) {
+    if (T < 0 || E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
+    if (E > MOE_MAX_EXPERTS || k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
+    if (T == 0) return MOE_OK;
+    if (!logits || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+    return cuda_status(
+        launch_route_topk(logits, T, E, k, topk_idx, topk_w, (cudaStream_t)stream));
+}
+
+size_t moe_dispatch_layout_workspace_bytes(int64_t T, int32_t k, int32_t E) {
+    if (T < 0 || k < 1 || E < 1) return 0;
+    return layout_workspace_bytes(T, k, E);
+}
+
+moe_status moe_dispatch_layout(const int32_t* topk_idx, int64_t T, int32_t k, int32_t E,
+                               int32_t W, int32_t* expert_counts, int32_t* expert_offsets,
+                               int32_t* rank_offsets, int32_t* slot_of_pair,
+                               int32_t* pair_of_slot, void* workspace, size_t workspace_bytes,
+                               int32_t* dev_status, void* stream) {
+    if (T < 0 || k < 1 || E < 1 || W < 1 || W > E || (E % W) != 0) return MOE_ERR_INVALID_ARG;
+    if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+    if (T * (int64_t)k >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
+    if (!expert_counts || !expert_offsets || !rank_offsets || !workspace || !dev_status)
+        return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!topk_idx || !slot_of_pair || !pair_of_slot)) return MOE_ERR_INVALID_ARG;
+    if (workspace_bytes < layout_workspace_bytes(T, k, E) || !aligned16(workspace))
+        return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_dispatch_layout(topk_idx, T, k, E, W, expert_counts,
+                                              expert_offsets, rank_offsets, slot_of_pair,
+                                              pair_of_slot, workspace, dev_status,
+                                              (cudaStream_t)stream));
+}
+
+moe_status moe_permute(const void* x, moe_dtype x_dtype, int64_t T, int32_t H, int32_t k,
+                       const int32_t* slot_of_pair, void* xp, moe_dtype xp_dtype,
+                       float* xp_scales, void* stream) {
+    if (T < 0 || H < 1 || k < 1 || (H % 8) != 0) return MOE_ERR_INVALID_ARG;
+    if (!is_act_dtype(x_dtype)) return MOE_ERR_INVALID_ARG;
+    if (xp_dtype != x_dtype && xp_dtype != MOE_E4M3) return MOE_ERR_INVALID_ARG;
+    if (xp_dtype == MOE_E4M3 && ((H % 128) != 0 || !xp_scales)) return MOE_ERR_INVALID_ARG;
+    if (k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
+    if (T == 0) return MOE_OK;
+    if (!x || !slot_of_pair || !xp || !aligned16(x) || !aligned16(xp)) return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_permute(x, x_dtype, T, H, k, slot_of_pair, xp, xp_dtype, xp_scales,
+                                      (cudaStream_t)stream));
+}
+
+size_t moe_grouped_gemm_workspace_bytes(int64_t n_rows, int32_t H, int32_t I, moe_dtype xp_dtype,
+                                        moe_dtype w_dtype) {
+    (void)I;
+    (void)w_dtype;
+    if (n_rows < 0 || H < 1) return 0;
+    // FP8 payload: a bf16 copy of the dequantised rows for the GEMM's A.
+    return xp_dtype == MOE_E4M3 ? (size_t)n_rows * H * 2 : 0;
+}
+
+moe_status moe_grouped_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_scales,
+                            const int32_t* expert_offsets, int32_t expert_begin,
+                            int32_t n_experts, int64_t n_rows, int32_t H, int32_t I,
+                            const void* w13, const void* w2, moe_dtype w_dtype, void* h, void* y,
+                            void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                            void* stream) {
+    if (n_rows < 0 || H < 1 || I < 1 || (H % 8) != 0 || (I % 8) != 0) return MOE_ERR_INVALID_ARG;
+    if (expert_begin < 0 || n_experts < 1) return MOE_ERR_INVALID_ARG;
+    if (n_experts > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+    const bool f32 = (w_dtype == MOE_F32 && xp_dtype == MOE_F32);
+    const bool bf16 = (w_dtype == MOE_BF16 && (xp_dtype == MOE_BF16 || xp_dtype == MOE_E4M3));
+    if (!f32 && !bf16) return MOE_ERR_INVALID_ARG;
+    if (xp_dtype == MOE_E4M3 && ((H % 128) != 0 || !xp_scales)) return MOE_ERR_INVALID_ARG;
+    if (!expert_offsets || !w13 || !w2 || !dev_status) return MOE_ERR_INVALID_ARG;
+    if (n_rows == 0) return MOE_OK;
+    if (!xp || !h || !y) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(xp) || !aligned16(w13) || !aligned16(w2) || !aligned16(h) || !aligned16(y))
+        return MOE_ERR_INVALID_ARG;
+    const size_t need = moe_grouped_gemm_workspace_bytes(n_rows, H, I, xp_dtype, w_dtype);
+    if (need > 0 && (workspace_bytes < need || !workspace || ((uintptr_t)workspace & 127u)))
+        return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (f32)
+        return cuda_status(launch_grouped_gemm_simt_f32(
+            (const float*)xp, expert_offsets, expert_begin, n_experts, n_rows, H, I,
+            (const float*)w13, (const float*)w2, (float*)h, (float*)y, s));
+    const __nv_bfloat16* a = (const __nv_bfloat16*)xp;
+    if (xp_dtype == MOE_E4M3) {
+        cudaError_t e = launch_dequant_e4m3((const uint8_t*)xp, xp_scales, expert_offsets,
+                                            expert_begin, n_experts, n_rows, H,
+                                            (__nv_bfloat16*)workspace, s);
+        if (e != cudaSuccess) return cuda_status(e);
+        a = (const __nv_bfloat16*)workspace;
+    }
+    return cuda_status(launch_grouped_gemm_tc(
+        a, expert_offsets, expert_begin, n_experts, n_rows, H, I, (const __nv_bfloat16*)w13,
+        (const __nv_bfloat16*)w2, (__nv_bfloat16*)h, (__nv_bfloat16*)y, dev_status, s));
+}
+
+moe_status moe_combine(const void* y, moe_dtype y_dtype, const int32_t* slot_of_pair,
+                       const float* topk_w, int64_t T, int32_t k, int32_t H, void* out,
+                       moe_dtype out_dtype, void* stream) {
+    if (T < 0 || H < 1 || k < 1 || (H % 8) != 0) return MOE_ERR_INVALID_ARG;
+    if (!is_act_dtype(y_dtype) || !is_act_dtype(out_dtype)) return MOE_ERR_INVALID_ARG;
+    if (k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
+    if (T == 0) return MOE_OK;
+    if (!y || !slot_of_pair || !topk_w || !out || !aligned16(y) || !aligned16(out))
+        return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_combine(y, y_dtype, slot_of_pair, topk_w, T, k, H, out, out_dtype,
+                                      (cudaStream_t)stream));
+}
+
+moe_status moe_check_status(int32_t* dev_status, void* stream) {
+    if (!dev_status) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    int32_t v = 0;
+    cudaError_t e = cudaMemcpyAsync(&v, dev_status, sizeof(v), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_status(e);
+    if (v & MOE_DEV_TIMEOUT) return MOE_ERR_TIMEOUT;
+    if (v & MOE_DEV_BAD_INDEX) return MOE_ERR_BAD_INDEX;
+    return MOE_OK;
+}
+
+uint64_t moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* moe_status_str(moe_status s) {
+    switch (s) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+        case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+        case MOE_ERR_BAD_INDEX: return "MOE_ERR_BAD_INDEX";
+        case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+        case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    }
+    return "MOE_ERR_UNKNOWN";
+}
+
+}  // extern "C"

@@ -1,0 +1,117 @@
+// combine.cu -- un-permute plus the router-weighted sum of each token's k
+// expert outputs back into its home row.
+//
+// Source: "Expert Parallelism" (aiwiki), "Implementation" (y[order] =
+// back); "Expert parallelism and all-to-all", "Walking through one MoE
+// layer", step 4 (the home GPU takes a weighted sum into the residual
+// stream).
+//
+// One CTA per token (grid-stride).  Each thread owns 8 consecutive output
+// elements; for every pick j it loads that piece of row y[slot_of_pair[t*k
+// + j]] (16-byte vector loads, all k issued before the sums), accumulates
+// w_j * y in fp32 with fused multiply-adds in j order, and rounds once.
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kCombineMaxTopK = MOE_MAX_TOPK;
+
+__device__ __forceinline__ void load8_row(const float* p, float (&f)[8]) {
+    float a[4], b[4];
+    unpack16(ld_nc_v4(p), a);
+    unpack16(ld_nc_v4(p + 4), b);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[i] = a[i];
+        f[4 + i] = b[i];
+    }
+}
+__device__ __forceinline__ void load8_row(const __nv_bfloat16* p, float (&f)[8]) {
+    unpack16(ld_nc_v4(p), f);
+}
+
+__device__ __forceinline__ void store8(float* p, const float (&f)[8]) {
+    st_v4(p, make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                        __float_as_uint(f[3])));
+    st_v4(p + 4, make_uint4(__float_as_uint(f[4]), __float_as_uint(f[5]), __float_as_uint(f[6]),
+                            __float_as_uint(f[7])));
+}
+__device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&f)[8]) {
+    st_v4(p, make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                        pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7])));
+}
+
+template <typename TY, typename TO>
+__global__ void __launch_bounds__(256) combine_kernel(const TY* __restrict__ y,
+                                                      const int32_t* __restrict__ slot_of_pair,
+                                                      const float* __restrict__ topk_w, int64_t T,
+                                                      int k, int H, TO* __restrict__ out) {
+    __shared__ int32_t s_slot[kCombineMaxTopK];
+    __shared__ float s_w[kCombineMaxTopK];
+    const int nchunk = H / 8;
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        if (threadIdx.x < k) {
+            s_slot[threadIdx.x] = slot_of_pair[t * k + threadIdx.x];
+            s_w[threadIdx.x] = topk_w[t * k + threadIdx.x];
+        }
+        __syncthreads();
+        for (int c = threadIdx.x; c < nchunk; c += blockDim.x) {
+            float acc[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+            int j = 0;
+            // four picks at a time: their loads are in flight together
+            for (; j + 4 <= k; j += 4) {
+                float v[4][8];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int32_t s = s_slot[j + u];
+                    if (s >= 0) load8_row(y + (int64_t)s * H + c * 8, v[u]);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    if (s_slot[j + u] < 0) continue;
+                    const float w = s_w[j + u];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc[i] = fmaf(w, v[u][i], acc[i]);
+                }
+            }
+            for (; j < k; ++j) {
+                const int32_t s = s_slot[j];
+                if (s < 0) continue;
+                float v[8];
+                load8_row(y + (int64_t)s * H + c * 8, v);
+                const float w = s_w[j];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = fmaf(w, v[i], acc[i]);
+            }
+            store8(out + t * H + c * 8, acc);
+        }
+        __syncthreads();
+    }
+}
+
+cudaError_t launch_combine(const void* y, moe_dtype ydt, const int32_t* slot_of_pair,
+                           const float* topk_w, int64_t T, int k, int H, void* out,
+                           moe_dtype odt, cudaStream_t s) {
+    if (T == 0) return cudaSuccess;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t cap = (int64_t)sms * 8;
+    const unsigned grid = (unsigned)(T < cap ? T : cap);
+    int threads = ((H / 8 + 31) / 32) * 32;
+    threads = threads < 32 ? 32 : (threads > 256 ? 256 : threads);
+#define MOE_COMBINE(TY, TO)                                                                    \
+    combine_kernel<TY, TO><<<grid, threads, 0, s>>>((const TY*)y, slot_of_pair, topk_w, T, k, \
+                                                    H, (TO*)out)
+    if (ydt == MOE_BF16 && odt == MOE_BF16) MOE_COMBINE(__nv_bfloat16, __nv_bfloat16);
+    else if (ydt == MOE_BF16) MOE_COMBINE(__nv_bfloat16, float);
+    else if (odt == MOE_BF16) MOE_COMBINE(float, __nv_bfloat16);
+    else MOE_COMBINE(float, float);
+#undef MOE_COMBINE
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

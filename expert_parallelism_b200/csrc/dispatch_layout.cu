@@ -1,0 +1,269 @@
+// dispatch_layout.cu -- per-expert histogram, exclusive scan and stable
+// expert-major slot assignment of the routed (token, expert) pairs.
+//
+// Source: "Expert Parallelism" (aiwiki), "Implementation": sort the local
+// tokens by destination so each peer's rows form one slab, and count rows
+// per rank; the sort is stable (ties by pair index).  Ranks own
+// consecutive expert blocks ("Expert parallelism" (Transformers docs),
+// "How the sizes combine"), so expert-major order is rank-major.
+//
+// Three launches on the caller's stream, no host synchronisation:
+//   1. layout_hist     one CTA per tile of kTilePairs pairs: shared-memory
+//                      atomic histogram -> counts[e * nt + b] (expert-major).
+//   2. layout_scan     single-pass exclusive scan of counts[] in that
+//                      expert-major order with decoupled look-back between
+//                      chunks: base[e * nt + b] = slot of tile b's first
+//                      pair routed to expert e.
+//   3. layout_scatter  one CTA per tile: a stable in-tile rank per pair
+//                      (warps walk their pairs in order, __match_any_sync
+//                      groups equal experts inside each 32-pair step, warp
+//                      counts are scanned across warps), slot = base +
+//                      rank; writes slot_of_pair / pair_of_slot, and CTA 0
+//                      writes the counts, offsets and rank offsets.
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kLayoutThreads = 256;                       // 8 warps
+constexpr int kLayoutWarps = kLayoutThreads / kWarp;
+constexpr int kGroupsPerWarp = 8;                          // 8 x 32 pairs per warp
+constexpr int kTilePairs = kLayoutWarps * kGroupsPerWarp * kWarp;  // 2048
+constexpr int kScanThreads = 256;
+constexpr int kScanItems = 16;
+constexpr int kScanChunk = kScanThreads * kScanItems;      // 4096
+
+// look-back status word: flag in the high 32 bits, value in the low 32
+constexpr unsigned long long kFlagAggregate = 1ull << 32;
+constexpr unsigned long long kFlagInclusive = 2ull << 32;
+
+struct LayoutWorkspace {
+    unsigned long long* status;  // [nchunks]
+    int32_t* ticket;             // [1]
+    int32_t* counts;             // [L]
+    int32_t* base;               // [L]
+    int64_t nt, L, nchunks;
+};
+
+static inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+static LayoutWorkspace carve(void* ws, int64_t T, int k, int E) {
+    LayoutWorkspace w;
+    const int64_t N = T * k;
+    w.nt = N > 0 ? (N + kTilePairs - 1) / kTilePairs : 1;
+    w.L = (int64_t)E * w.nt;
+    w.nchunks = (w.L + kScanChunk - 1) / kScanChunk;
+    char* p = (char*)ws;
+    w.status = (unsigned long long*)p;
+    p += align_up((size_t)w.nchunks * 8, 16);
+    w.ticket = (int32_t*)p;
+    p += 16;
+    w.counts = (int32_t*)p;
+    p += align_up((size_t)w.L * 4, 16);
+    w.base = (int32_t*)p;
+    return w;
+}
+
+size_t layout_workspace_bytes(int64_t T, int k, int E) {
+    LayoutWorkspace w = carve(nullptr, T, k, E);
+    return align_up((size_t)w.nchunks * 8, 16) + 16 + 2 * align_up((size_t)w.L * 4, 16);
+}
+
+__global__ void __launch_bounds__(kLayoutThreads) layout_hist_kernel(
+    const int32_t* __restrict__ idx, int64_t N, int E, int64_t nt,
+    int32_t* __restrict__ counts, unsigned long long* __restrict__ status, int64_t nchunks,
+    int32_t* __restrict__ ticket, int32_t* __restrict__ dev_status) {
+    extern __shared__ int32_t hist[];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+    if (blockIdx.x == 0) {
+        for (int64_t c = threadIdx.x; c < nchunks; c += blockDim.x) status[c] = 0ull;
+        if (threadIdx.x == 0) *ticket = 0;
+    }
+    __syncthreads();
+    const int64_t b = blockIdx.x;
+    const int64_t p0 = b * kTilePairs, p1 = min(N, p0 + kTilePairs);
+    int bad = 0;
+    for (int64_t p = p0 + threadIdx.x; p < p1; p += blockDim.x) {
+        const int e = __ldg(idx + p);
+        if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
+        else bad = 1;
+    }
+    if (__syncthreads_or(bad) && threadIdx.x == 0) flag_status(dev_status, MOE_DEV_BAD_INDEX);
+    for (int e = threadIdx.x; e < E; e += blockDim.x) counts[(int64_t)e * nt + b] = hist[e];
+}
+
+__global__ void __launch_bounds__(kScanThreads) layout_scan_kernel(
+    const int32_t* __restrict__ counts, int32_t* __restrict__ base, int64_t L,
+    unsigned long long* status, int32_t* ticket, int32_t* dev_status) {
+    __shared__ int32_t s_chunk, s_prefix;
+    __shared__ int32_t s_warp[kScanThreads / kWarp];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // chunks are numbered in the order CTAs start, so every predecessor a
+    // chunk waits for is already running: the look-back cannot deadlock
+    if (tid == 0) s_chunk = atomicAdd(ticket, 1);
+    __syncthreads();
+    const int64_t c = s_chunk;
+    const int64_t i0 = c * kScanChunk + (int64_t)tid * kScanItems;
+    int32_t v[kScanItems];
+    int32_t mine = 0;
+#pragma unroll
+    for (int i = 0; i < kScanItems; ++i) {
+        v[i] = (i0 + i < L) ? counts[i0 + i] : 0;
+        mine += v[i];
+    }
+    // block-wide exclusive scan of the per-thread sums
+    int32_t incl = mine;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    int32_t warp_excl = 0, total = 0;
+    for (int w = 0; w < kScanThreads / kWarp; ++w) {
+        if (w < warp) warp_excl += s_warp[w];
+        total += s_warp[w];
+    }
+    if (tid == 0) {
+        int32_t excl = 0;
+        if (c == 0) {
+            atomicExch(&status[0], kFlagInclusive | (uint32_t)total);
+        } else {
+            atomicExch(&status[c], kFlagAggregate | (uint32_t)total);
+            const uint64_t deadline = global_timer_ns() + kSpinLimitNs;
+            int64_t j = c - 1;
+            while (j >= 0) {
+                const unsigned long long st = *((volatile unsigned long long*)&status[j]);
+                const unsigned long long flag = st & 0xFFFFFFFF00000000ull;
+                if (flag == 0ull) {
+                    if (global_timer_ns() > deadline) {
+                        flag_status(dev_status, MOE_DEV_TIMEOUT);
+                        break;
+                    }
+                    __nanosleep(64);
+                    continue;
+                }
+                excl += (int32_t)(st & 0xFFFFFFFFull);
+                if (flag == kFlagInclusive) break;
+                --j;
+            }
+            atomicExch(&status[c], kFlagInclusive | (uint32_t)(excl + total));
+        }
+        s_prefix = excl;
+    }
+    __syncthreads();
+    int32_t run = s_prefix + warp_excl + (incl - mine);
+#pragma unroll
+    for (int i = 0; i < kScanItems; ++i) {
+        if (i0 + i < L) base[i0 + i] = run;
+        run += v[i];
+    }
+}
+
+__global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(
+    const int32_t* __restrict__ idx, int64_t N, int E, int W, int64_t nt,
+    const int32_t* __restrict__ counts, const int32_t* __restrict__ base, int64_t L,
+    int32_t* __restrict__ expert_counts, int32_t* __restrict__ expert_offsets,
+    int32_t* __restrict__ rank_offsets, int32_t* __restrict__ slot_of_pair,
+    int32_t* __restrict__ pair_of_slot) {
+    extern __shared__ int32_t sm[];
+    int32_t* wcount = sm;                      // [warps][E]: counts, then warp prefixes
+    int32_t* s_base = sm + kLayoutWarps * E;   // [E]: base of this tile per expert
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t b = blockIdx.x;
+    const int32_t total = base[L - 1] + counts[L - 1];
+
+    for (int i = tid; i < kLayoutWarps * E; i += blockDim.x) wcount[i] = 0;
+    for (int e = tid; e < E; e += blockDim.x) s_base[e] = base[(int64_t)e * nt + b];
+    __syncthreads();
+
+    // pass 1: each warp walks its pairs in order; equal experts inside a
+    // 32-pair step are ranked by lane, steps are ranked by a running count
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    const int64_t pw = b * kTilePairs + (int64_t)warp * (kGroupsPerWarp * kWarp);
+    int32_t rank[kGroupsPerWarp];
+    int32_t ex[kGroupsPerWarp];
+#pragma unroll
+    for (int g = 0; g < kGroupsPerWarp; ++g) {
+        const int64_t p = pw + g * kWarp + lane;
+        int e = (p < N) ? __ldg(idx + p) : -1;
+        if (e < 0 || e >= E) e = -1;
+        const uint32_t peers = __match_any_sync(0xffffffffu, e);
+        const int32_t c = (e >= 0) ? wcount[warp * E + e] : 0;
+        __syncwarp();
+        if (e >= 0 && lane == __ffs(peers) - 1) wcount[warp * E + e] = c + __popc(peers);
+        __syncwarp();
+        rank[g] = c + __popc(peers & lt_mask);
+        ex[g] = e;
+    }
+    __syncthreads();
+    // exclusive prefix of the warp counts, per expert
+    for (int e = tid; e < E; e += blockDim.x) {
+        int32_t run = 0;
+        for (int w = 0; w < kLayoutWarps; ++w) {
+            const int32_t t = wcount[w * E + e];
+            wcount[w * E + e] = run;
+            run += t;
+        }
+    }
+    __syncthreads();
+    // pass 2: slots
+#pragma unroll
+    for (int g = 0; g < kGroupsPerWarp; ++g) {
+        const int64_t p = pw + g * kWarp + lane;
+        if (p >= N) continue;
+        const int e = ex[g];
+        if (e < 0) {
+            slot_of_pair[p] = -1;
+            continue;
+        }
+        const int32_t s = s_base[e] + wcount[warp * E + e] + rank[g];
+        slot_of_pair[p] = s;
+        pair_of_slot[s] = (int32_t)p;
+    }
+    // slots past the last routed row (only when ids were skipped)
+    for (int64_t s = (int64_t)total + b * blockDim.x + tid; s < N; s += nt * blockDim.x)
+        pair_of_slot[s] = -1;
+    if (b == 0) {
+        for (int e = tid; e <= E; e += blockDim.x) {
+            const int32_t lo = (e < E) ? base[(int64_t)e * nt] : total;
+            expert_offsets[e] = lo;
+            if (e < E) {
+                const int32_t hi = (e + 1 < E) ? base[(int64_t)(e + 1) * nt] : total;
+                expert_counts[e] = hi - lo;
+            }
+        }
+        for (int r = tid; r <= W; r += blockDim.x) {
+            const int e = (int)((int64_t)r * E / W);
+            rank_offsets[r] = (e < E) ? base[(int64_t)e * nt] : total;
+        }
+    }
+}
+
+cudaError_t launch_dispatch_layout(const int32_t* idx, int64_t T, int k, int E, int W,
+                                   int32_t* expert_counts, int32_t* expert_offsets,
+                                   int32_t* rank_offsets, int32_t* slot_of_pair,
+                                   int32_t* pair_of_slot, void* workspace,
+                                   int32_t* dev_status, cudaStream_t s) {
+    const int64_t N = T * k;
+    LayoutWorkspace w = carve(workspace, T, k, E);
+    const size_t hist_smem = (size_t)E * 4;
+    const size_t scatter_smem = (size_t)(kLayoutWarps + 1) * E * 4;
+    if (scatter_smem > 48 * 1024) {
+        cudaError_t err = cudaFuncSetAttribute(
+            layout_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scatter_smem);
+        if (err != cudaSuccess) return err;
+    }
+    layout_hist_kernel<<<(unsigned)w.nt, kLayoutThreads, hist_smem, s>>>(
+        idx, N, E, w.nt, w.counts, w.status, w.nchunks, w.ticket, dev_status);
+    layout_scan_kernel<<<(unsigned)w.nchunks, kScanThreads, 0, s>>>(w.counts, w.base, w.L,
+                                                                    w.status, w.ticket,
+                                                                    dev_status);
+    layout_scatter_kernel<<<(unsigned)w.nt, kLayoutThreads, scatter_smem, s>>>(
+        idx, N, E, W, w.nt, w.counts, w.base, w.L, expert_counts, expert_offsets, rank_offsets,
+        slot_of_pair, pair_of_slot);
+    note_launches(3);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,195 @@
+"""Python binding of libmoe's C ABI (include/moe.h): argument marshalling only.
+
+Each ``moe_*`` function mirrors the C entry point of the same name: it
+takes CUDA torch tensors (PyTorch supplies device memory and the current
+stream), passes their raw pointers and sizes through ctypes, and raises
+``MoEError`` for any status other than MOE_OK.  All computation happens in
+the library's CUDA kernels; there is no Python or CPU fallback, and
+loading fails loudly when ``libmoe.so`` has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+
+MOE_F32, MOE_BF16, MOE_E4M3 = 0, 1, 2
+MOE_DEV_BAD_INDEX, MOE_DEV_TIMEOUT = 0x1, 0x2
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_BAD_INDEX",
+          4: "MOE_ERR_TIMEOUT", 5: "MOE_ERR_CUDA"}
+_DT = {torch.float32: MOE_F32, torch.bfloat16: MOE_BF16, torch.float8_e4m3fn: MOE_E4M3}
+
+# exported symbols and their ctypes signatures (P = pointer, I64/I32 = ints)
+_P, _I64, _I32, _SZ, _I = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t,
+                           ctypes.c_int)
+SIGNATURES = {
+    "moe_route_topk": ([_P, _I64, _I32, _I32, _P, _P, _P], _I),
+    "moe_dispatch_layout_workspace_bytes": ([_I64, _I32, _I32], _SZ),
+    "moe_dispatch_layout": ([_P, _I64, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _SZ, _P, _P], _I),
+    "moe_permute": ([_P, _I, _I64, _I32, _I32, _P, _P, _I, _P, _P], _I),
+    "moe_grouped_gemm_workspace_bytes": ([_I64, _I32, _I32, _I, _I], _SZ),
+    "moe_grouped_gemm": ([_P, _I, _P, _P, _I32, _I32, _I64, _I32, _I32, _P, _P, _I, _P, _P, _P,
+                          _SZ, _P, _P], _I),
+    "moe_combine": ([_P, _I, _P, _P, _I64, _I32, _I32, _P, _I, _P], _I),
+    "moe_check_status": ([_P, _P], _I),
+    "moe_status_str": ([_I], ctypes.c_char_p),
+    "moe_launch_count": ([], ctypes.c_uint64),
+}
+
+
+class MoEError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn}: {STATUS.get(code, code)}")
+        self.code = code
+        self.status = STATUS.get(code, str(code))
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libmoe.so once; raises if it is missing (no fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise ImportError(f"libmoe.so not built at {path}: run "
+                              "`python -m expert_parallelism_b200.build`")
+        lib = ctypes.CDLL(path)
+        for name, (args, res) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.argtypes, fn.restype = args, res
+        _lib = lib
+    return _lib
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(name, rc):
+    if rc != 0:
+        raise MoEError(name, rc)
+
+
+def dtype_code(t: torch.Tensor) -> int:
+    return _DT[t.dtype]
+
+
+# ----------------------------------------------------------------- the C ABI
+def moe_route_topk(logits, topk_idx, topk_w, stream=None):
+    T, E = logits.shape
+    k = topk_idx.shape[1]
+    _check("moe_route_topk", load_library().moe_route_topk(
+        _ptr(logits), T, E, k, _ptr(topk_idx), _ptr(topk_w), _stream(stream)))
+
+
+def moe_dispatch_layout_workspace_bytes(T, k, E) -> int:
+    return int(load_library().moe_dispatch_layout_workspace_bytes(T, k, E))
+
+
+def moe_dispatch_layout(topk_idx, E, W, expert_counts, expert_offsets, rank_offsets,
+                        slot_of_pair, pair_of_slot, workspace, dev_status, stream=None):
+    T, k = topk_idx.shape
+    _check("moe_dispatch_layout", load_library().moe_dispatch_layout(
+        _ptr(topk_idx), T, k, E, W, _ptr(expert_counts), _ptr(expert_offsets),
+        _ptr(rank_offsets), _ptr(slot_of_pair), _ptr(pair_of_slot), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
+
+
+def moe_permute(x, k, slot_of_pair, xp, xp_scales=None, stream=None):
+    T, H = x.shape
+    _check("moe_permute", load_library().moe_permute(
+        _ptr(x), dtype_code(x), T, H, k, _ptr(slot_of_pair), _ptr(xp), dtype_code(xp),
+        _ptr(xp_scales), _stream(stream)))
+
+
+def moe_grouped_gemm_workspace_bytes(n_rows, H, I, xp_dtype, w_dtype) -> int:
+    return int(load_library().moe_grouped_gemm_workspace_bytes(n_rows, H, I, _DT[xp_dtype],
+                                                                _DT[w_dtype]))
+
+
+def moe_grouped_gemm(xp, xp_scales, expert_offsets, expert_begin, n_experts, w13, w2, h, y,
+                     workspace, dev_status, stream=None):
+    n_rows, H = xp.shape
+    I = w2.shape[2]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("moe_grouped_gemm", load_library().moe_grouped_gemm(
+        _ptr(xp), dtype_code(xp), _ptr(xp_scales), _ptr(expert_offsets), expert_begin,
+        n_experts, n_rows, H, I, _ptr(w13), _ptr(w2), dtype_code(w13), _ptr(h), _ptr(y),
+        _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream)))
+
+
+def moe_combine(y, slot_of_pair, topk_w, out, stream=None):
+    T, k = topk_w.shape
+    H = y.shape[1]
+    _check("moe_combine", load_library().moe_combine(
+        _ptr(y), dtype_code(y), _ptr(slot_of_pair), _ptr(topk_w), T, k, H, _ptr(out),
+        dtype_code(out), _stream(stream)))
+
+
+def moe_check_status(dev_status, stream=None) -> int:
+    """Synchronises the stream; returns the raw status code (0 = OK)."""
+    return int(load_library().moe_check_status(_ptr(dev_status), _stream(stream)))
+
+
+def moe_status_str(code: int) -> str:
+    return load_library().moe_status_str(code).decode()
+
+
+# ----------------------------------------------------------------- buffers
+class LayerBuffers:
+    """Device buffers for one layer of a workload (outputs and workspaces).
+
+    Plain torch allocations made once; every step reuses them.
+    """
+
+    def __init__(self, wl, device="cuda"):
+        from .workloads import TORCH_DTYPE
+        T, H, E, k, I, W, N = wl.T, wl.H, wl.E, wl.k, wl.I, wl.W, wl.N
+        dev = torch.device(device)
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.wl = wl
+        self.topk_idx = torch.empty(T, k, **i32)
+        self.topk_w = torch.empty(T, k, dtype=torch.float32, device=dev)
+        self.expert_counts = torch.empty(E, **i32)
+        self.expert_offsets = torch.empty(E + 1, **i32)
+        self.rank_offsets = torch.empty(W + 1, **i32)
+        self.slot_of_pair = torch.empty(max(N, 1), **i32)
+        self.pair_of_slot = torch.empty(max(N, 1), **i32)
+        self.layout_ws = torch.empty(max(moe_dispatch_layout_workspace_bytes(T, k, E), 16),
+                                     dtype=torch.uint8, device=dev)
+        self.dev_status = torch.zeros(1, **i32)
+        pdt = TORCH_DTYPE[wl.payload]
+        self.xp = torch.empty(N, H, dtype=pdt, device=dev)
+        self.xp_scales = (torch.empty(N, H // 128, dtype=torch.float32, device=dev)
+                          if wl.payload == "e4m3" else None)
+        wdt = TORCH_DTYPE[wl.wdt]
+        self.h = torch.empty(N, I, dtype=wdt, device=dev)
+        self.y = torch.empty(N, H, dtype=wdt, device=dev)
+        gb = moe_grouped_gemm_workspace_bytes(N, H, I, pdt, wdt)
+        self.gemm_ws = torch.empty(gb, dtype=torch.uint8, device=dev) if gb else None
+        self.out = torch.empty(T, H, dtype=TORCH_DTYPE[wl.act], device=dev)
+
+
+def layer_forward(wl, logits, x, w13, w2, buf: LayerBuffers, stream=None):
+    """The whole hot path: route -> layout -> permute -> grouped GEMM -> combine."""
+    moe_route_topk(logits, buf.topk_idx, buf.topk_w, stream)
+    moe_dispatch_layout(buf.topk_idx, wl.E, wl.W, buf.expert_counts, buf.expert_offsets,
+                        buf.rank_offsets, buf.slot_of_pair, buf.pair_of_slot, buf.layout_ws,
+                        buf.dev_status, stream)
+    moe_permute(x, wl.k, buf.slot_of_pair, buf.xp, buf.xp_scales, stream)
+    moe_grouped_gemm(buf.xp, buf.xp_scales, buf.expert_offsets, 0, wl.E, w13, w2, buf.h, buf.y,
+                     buf.gemm_ws, buf.dev_status, stream)
+    moe_combine(buf.y, buf.slot_of_pair, buf.topk_w, buf.out, stream)
+    return buf.out

@@ -1,0 +1,242 @@
+/*
+ * moe.h -- C ABI of libmoe: the single-GPU core of an expert-parallel
+ * mixture-of-experts layer on NVIDIA B200 (sm_100a).
+ *
+ * One MoE layer, as "Expert parallelism and all-to-all" walks through it
+ * (section "Walking through one MoE layer"): the router gives every token
+ * k (expert, weight) picks; dispatch sends each token's hidden vector to
+ * the owners of its experts; each owner runs its local experts on what it
+ * received as one grouped matrix multiply; combine returns the outputs to
+ * the token's home row as a router-weighted sum.  On one GPU, the logical
+ * expert-parallel ranks ("Expert parallelism" (Transformers docs), section
+ * "How the sizes combine": rank r of W owns experts [r*E/W, (r+1)*E/W))
+ * only fix the slab layout of the permuted buffer; no collective is issued.
+ *
+ *   moe_route_topk       logits[T,E]                 -> topk_idx[T,k], topk_w[T,k]
+ *   moe_dispatch_layout  topk_idx[T,k]               -> counts, offsets, rank slabs,
+ *                                                       slot_of_pair[N], pair_of_slot[N]
+ *   moe_permute          x[T,H], slot_of_pair        -> xp[N,H] (+ FP8 block scales)
+ *   moe_grouped_gemm     xp, offsets, W13, W2        -> h[N,I], y[N,H]  (SwiGLU FFN)
+ *   moe_combine          y, slot_of_pair, topk_w     -> out[T,H]
+ *
+ * with N = T*k routed pairs; pair p = t*k + j is token t's j-th pick.
+ *
+ * Conventions shared by every call:
+ *  - All arrays are dense, row-major, and live in device memory (except
+ *    where a call says otherwise).  Index arrays are int32.
+ *  - The caller allocates and owns every buffer, including workspaces and
+ *    the device status word.  The library allocates nothing, frees
+ *    nothing and never synchronises, except moe_check_status.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *    call only enqueues work on it and returns; the chain of calls has no
+ *    host synchronisation, so it can be captured in a CUDA graph.
+ *  - Arguments are validated on the host before anything is enqueued.  An
+ *    invalid call returns MOE_ERR_INVALID_ARG (or MOE_ERR_UNSUPPORTED for a
+ *    valid request beyond the kernels' limits) and touches no output.  This
+ *    follows the pages' own rule of refusing a bad configuration up front
+ *    rather than silently falling back ("Expert parallelism" (Transformers
+ *    docs), "Overriding the plans"; the expert-parallel-plan ValueError of
+ *    transformers' distributed mixin).
+ *  - T == 0 is a valid, empty batch ("token slices may be uneven or
+ *    empty", Transformers docs, "With tensor parallelism"); experts that
+ *    receive no rows are valid too.
+ *  - Errors found on the device (an expert id outside [0, E); a bounded
+ *    wait that ran out) are OR-ed into the caller's int32 status word
+ *    `dev_status` and the call still returns MOE_OK; moe_check_status
+ *    reports them.  A failed kernel launch returns MOE_ERR_CUDA.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum moe_status {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1, /* null pointer, bad size, bad dtype combination */
+    MOE_ERR_UNSUPPORTED = 2, /* valid but beyond the kernels' limits (E > 1024, k > 16) */
+    MOE_ERR_BAD_INDEX = 3,   /* device: an expert id outside [0, E) was skipped */
+    MOE_ERR_TIMEOUT = 4,     /* device: a bounded wait ran out; results invalid */
+    MOE_ERR_CUDA = 5         /* a CUDA runtime call or kernel launch failed */
+} moe_status;
+
+typedef enum moe_dtype {
+    MOE_F32 = 0,  /* IEEE binary32 */
+    MOE_BF16 = 1, /* bfloat16 */
+    MOE_E4M3 = 2  /* OCP FP8 E4M3 (no infinities, max 448), payload only */
+} moe_dtype;
+
+/* Bits of the device status word. */
+#define MOE_DEV_BAD_INDEX 0x1
+#define MOE_DEV_TIMEOUT 0x2
+
+/* Kernel limits (MOE_ERR_UNSUPPORTED beyond them). */
+#define MOE_MAX_EXPERTS 1024
+#define MOE_MAX_TOPK 16
+
+/*
+ * moe_route_topk -- router top-k with softmax weights.
+ * Source: "Expert parallelism and all-to-all", "Walking through one MoE
+ * layer", step 1 (every token gets a list of (expert, weight) picks); the
+ * Transformers docs' (top_k_index, top_k_weights) pair ("Adding an
+ * implementation").
+ *
+ *   logits   [T, E] fp32, device, read only.
+ *   topk_idx [T, k] int32, device, written: token t's picks in order of
+ *            (logit descending, expert id ascending); ties go to the
+ *            lower expert id, -0 and +0 compare equal.
+ *   topk_w   [T, k] fp32, device, written: softmax over the k picked
+ *            logits (equal to the full softmax over E, restricted to the
+ *            picks and renormalised).
+ * Requires 1 <= k <= E, E <= MOE_MAX_EXPERTS, k <= MOE_MAX_TOPK.  Logits
+ * must be finite (NaN ordering is not defined).
+ */
+moe_status moe_route_topk(const float* logits, int64_t T, int32_t E, int32_t k,
+                          int32_t* topk_idx, float* topk_w, void* stream);
+
+/*
+ * moe_dispatch_layout -- the dispatch plan: a per-expert histogram, its
+ * exclusive scan, and a stable expert-major permutation of the pairs.
+ * Source: "Expert Parallelism" (aiwiki), "Implementation": sort the tokens
+ * by destination so each peer's rows are one contiguous slab, and count
+ * them per rank (bincount of idx // per_rank); the sort is taken as stable
+ * (ties by pair index).  Ownership: rank r owns experts [r*E/W, (r+1)*E/W)
+ * (Transformers docs, "How the sizes combine"), so the expert-major order
+ * is also rank-major and rank r's slab is [rank_offsets[r],
+ * rank_offsets[r+1]) -- exactly the send buffer of a dispatch all-to-all.
+ *
+ *   topk_idx       [T, k] int32, device, read only.
+ *   expert_counts  [E] int32, written: rows routed to each expert.
+ *   expert_offsets [E+1] int32, written: exclusive scan of the counts.
+ *   rank_offsets   [W+1] int32, written: expert_offsets[r*E/W].
+ *   slot_of_pair   [T*k] int32, written: the slot (row of the permuted
+ *                  buffer) of pair p; -1 for a pair with a bad expert id.
+ *   pair_of_slot   [T*k] int32, written: inverse map; slots past
+ *                  expert_offsets[E] hold -1.
+ *   workspace      device scratch of at least
+ *                  moe_dispatch_layout_workspace_bytes(T, k, E) bytes, 16-byte
+ *                  aligned; no initial contents needed; clobbered.
+ *   dev_status     int32 device word; MOE_DEV_BAD_INDEX is OR-ed in when a
+ *                  pair's expert id is outside [0, E) (the pair is skipped),
+ *                  MOE_DEV_TIMEOUT if the scan's bounded wait ran out.
+ * Requires 1 <= k, 1 <= W <= E, E % W == 0 (ep_size must divide the number
+ * of experts, Transformers docs, "Adding an implementation"), E <=
+ * MOE_MAX_EXPERTS, T*k < 2^31.
+ */
+size_t moe_dispatch_layout_workspace_bytes(int64_t T, int32_t k, int32_t E);
+moe_status moe_dispatch_layout(const int32_t* topk_idx, int64_t T, int32_t k, int32_t E,
+                               int32_t W, int32_t* expert_counts, int32_t* expert_offsets,
+                               int32_t* rank_offsets, int32_t* slot_of_pair,
+                               int32_t* pair_of_slot, void* workspace,
+                               size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * moe_permute -- write every token's hidden vector into the slots of its
+ * k pairs: xp[slot_of_pair[t*k + j]] = x[t] (the "sent = x[order]" of the
+ * aiwiki sketch, done as a scatter so each x row is read once).
+ * Source: aiwiki, "Implementation"; FP8 payload: "Expert parallelism and
+ * all-to-all", "Traffic math" (FP8 activations, 1 byte per element).
+ *
+ *   x         [T, H] in x_dtype (MOE_F32 or MOE_BF16), device, read only.
+ *   slot_of_pair [T*k] int32 from moe_dispatch_layout; pairs holding -1
+ *             are skipped.
+ *   xp        [T*k, H] in xp_dtype, device, written at the pairs' slots.
+ *             xp_dtype == x_dtype: a bitwise copy.
+ *             xp_dtype == MOE_E4M3: for each 128-element block of a token
+ *             row, scale = amax/448 (fp32 IEEE division; 1 if amax == 0)
+ *             and q = e4m3(x/scale) (fp32 IEEE division, round to nearest
+ *             even, saturating to +-448).  Requires H % 128 == 0.
+ *   xp_scales [T*k, H/128] fp32, written for MOE_E4M3, else ignored (may
+ *             be NULL).
+ * Requires H % 8 == 0, H > 0, k >= 1.
+ */
+moe_status moe_permute(const void* x, moe_dtype x_dtype, int64_t T, int32_t H, int32_t k,
+                       const int32_t* slot_of_pair, void* xp, moe_dtype xp_dtype,
+                       float* xp_scales, void* stream);
+
+/*
+ * moe_grouped_gemm -- every local expert's SwiGLU FFN over its rows, as
+ * one grouped GEMM ("Expert parallelism and all-to-all", "Walking through
+ * one MoE layer", step 3; the Transformers docs' experts_forward; expert
+ * weights stacked along the expert dimension, "GroupedGemmParallel").
+ *
+ * For local expert j (global expert e = expert_begin + j) and every slot s
+ * in [expert_offsets[e], expert_offsets[e+1]):
+ *     g = A_s W13[j, 0:I, :]^T,  u = A_s W13[j, I:2I, :]^T,
+ *     h_s = silu(g) * u  (silu(g) = g / (1 + exp(-g))),
+ *     y_s = h_s W2[j]^T,
+ * accumulated in fp32.  A_s is the xp row; for an FP8 payload it is
+ * bf16(decode(q) * scale) (fp32 product, rounded to bf16).
+ *
+ *   xp             [n_rows, H] in xp_dtype, device.
+ *   xp_scales      [n_rows, H/128] fp32 when xp_dtype == MOE_E4M3, else NULL.
+ *   expert_offsets [>= expert_begin + n_experts + 1] int32, DEVICE memory:
+ *                  read by the kernels, never by the host.
+ *   w13            [n_experts, 2I, H] in w_dtype (gate rows, then up rows).
+ *   w2             [n_experts, H, I] in w_dtype.
+ *   h              [n_rows, I] in w_dtype, written for the experts' rows.
+ *   y              [n_rows, H] in w_dtype, written for the experts' rows.
+ *   workspace      device scratch of moe_grouped_gemm_workspace_bytes(...)
+ *                  bytes (may be 0 / NULL when that is 0), 128-byte aligned.
+ *   dev_status     int32 device word (MOE_DEV_TIMEOUT on a bounded wait
+ *                  running out).
+ * Dtypes: w_dtype MOE_F32 with xp MOE_F32 (CUDA-core fp32 path), or w_dtype
+ * MOE_BF16 with xp MOE_BF16 or MOE_E4M3 (tensor-core path).  Requires H % 8
+ * == 0, I % 8 == 0 (H % 128 == 0 for E4M3), and the offsets to be
+ * non-decreasing with expert_offsets[expert_begin + n_experts] <= n_rows.
+ * xp, h, y, w13, w2 must be 16-byte aligned.
+ */
+size_t moe_grouped_gemm_workspace_bytes(int64_t n_rows, int32_t H, int32_t I,
+                                        moe_dtype xp_dtype, moe_dtype w_dtype);
+moe_status moe_grouped_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_scales,
+                            const int32_t* expert_offsets, int32_t expert_begin,
+                            int32_t n_experts, int64_t n_rows, int32_t H, int32_t I,
+                            const void* w13, const void* w2, moe_dtype w_dtype, void* h,
+                            void* y, void* workspace, size_t workspace_bytes,
+                            int32_t* dev_status, void* stream);
+
+/*
+ * moe_combine -- un-permute plus the router-weighted sum of each token's k
+ * expert outputs into its home row:
+ *     out[t] = sum_{j=0..k-1} topk_w[t,j] * y[slot_of_pair[t*k+j]],
+ * fp32 accumulation in j order, rounded once to out_dtype; pairs holding
+ * slot -1 add nothing.
+ * Source: aiwiki, "Implementation" (y[order] = back, undoing the sort);
+ * "Expert parallelism and all-to-all", step 4 (the home GPU takes a
+ * weighted sum into the residual stream); Transformers docs (the weighted
+ * expert output for each token).
+ *
+ *   y            [>= max slot + 1, H] in y_dtype (MOE_F32 / MOE_BF16), device.
+ *   slot_of_pair [T*k] int32, device.
+ *   topk_w       [T, k] fp32, device.
+ *   out          [T, H] in out_dtype (MOE_F32 / MOE_BF16), device, written.
+ * Requires H % 8 == 0, k >= 1.
+ */
+moe_status moe_combine(const void* y, moe_dtype y_dtype, const int32_t* slot_of_pair,
+                       const float* topk_w, int64_t T, int32_t k, int32_t H, void* out,
+                       moe_dtype out_dtype, void* stream);
+
+/*
+ * moe_check_status -- synchronise `stream`, read the device status word,
+ * clear it, and map it to a status: MOE_ERR_TIMEOUT if a wait ran out,
+ * else MOE_ERR_BAD_INDEX if an id was skipped, else MOE_OK (MOE_ERR_CUDA if
+ * the synchronisation itself failed).  The only call that blocks.
+ */
+moe_status moe_check_status(int32_t* dev_status, void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* moe_status_str(moe_status s);
+
+/* Diagnostics: total number of kernels this library has launched in this
+ * process (all devices, all streams), counted on the host at launch. */
+uint64_t moe_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

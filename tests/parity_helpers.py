@@ -1,0 +1,140 @@
+"""Shared helpers for the GPU parity tests: run the hot path through the
+C ABI and compare with the CPU oracle on the same seeded inputs.
+
+The oracle's floating-point results are exact (fp64, unrounded); the only
+narrow type inside its chain is h, the bf16 (or fp32) operand of the down
+projection.  Tolerances:
+  y, out (bf16):  per row, max |gpu - oracle| <= 2e-2 * RMS(oracle row)
+  y, out, h (fp32): per row, max |gpu - oracle| <= 1e-5 * RMS(oracle row)
+  h (bf16, the GEMM's internal activation): per element,
+                  |gpu - oracle| <= 2^-8 * |oracle| + 1e-3 * RMS(oracle row),
+                  i.e. the bf16 rounding of that element (at most half an
+                  ulp, 2^-8 relative) plus a floor for fp32 accumulation
+                  order; h is heavy-tailed (silu(g) * u), so a row-RMS bound
+                  would be smaller than the rounding of its largest entries
+  router weights: elementwise |dw| <= 1e-5 * |w|.
+Everything integer (indices, counts, offsets, permutation order, FP8 codes
+and their fp32 scales, same-dtype payload copies) must match bit for bit.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from expert_parallelism_b200 import moe, workloads
+
+BF16_TOL = 2e-2
+F32_TOL = 1e-5
+
+EXTRA = {
+    # sizes the oracle finishes in seconds that still span several tiles
+    # and ragged tails of the GEMM (partial M, N and K tiles)
+    "small_bf16": workloads.Workload("small_bf16", 300, 256, 8, 2, 192, 2, "bf16", "bf16", "bf16"),
+    "small_fp8": workloads.Workload("small_fp8", 200, 384, 16, 4, 320, 4, "bf16", "e4m3", "bf16"),
+    "ragged_bf16": workloads.Workload("ragged_bf16", 777, 200, 6, 3, 136, 3, "bf16", "bf16",
+                                      "bf16"),
+    "small_f32": workloads.Workload("small_f32", 130, 72, 5, 3, 40, 5, "f32", "f32", "f32"),
+}
+
+
+def workload(name):
+    return workloads.WORKLOADS.get(name) or EXTRA[name]
+
+
+def tol_for(dtype: torch.dtype) -> float:
+    return F32_TOL if dtype == torch.float32 else BF16_TOL
+
+
+def rowwise_ok(got: torch.Tensor, ref: torch.Tensor, tol: float):
+    """Per-row max abs error <= tol * RMS(ref row); returns (ok, worst ratio)."""
+    g, r = got.double(), ref.double()
+    rms = r.pow(2).mean(dim=1).sqrt()
+    err = (g - r).abs().amax(dim=1)
+    ratio = torch.where(rms > 0, err / rms, err)
+    worst = float(ratio.max()) if ratio.numel() else 0.0
+    return bool((ratio <= tol).all()), worst
+
+
+def h_ok(got: torch.Tensor, ref: torch.Tensor, dtype: torch.dtype):
+    """The h check above; returns (ok, worst excess over the bound / RMS)."""
+    if dtype == torch.float32:
+        return rowwise_ok(got, ref, F32_TOL)
+    g, r = got.double(), ref.double()
+    rms = r.pow(2).mean(dim=1, keepdim=True).sqrt()
+    bound = 2.0 ** -8 * r.abs() + 1e-3 * rms
+    excess = ((g - r).abs() - bound) / rms
+    worst = float(excess.max()) if excess.numel() else 0.0
+    return bool((excess <= 0).all()), worst
+
+
+def bits(t: torch.Tensor) -> torch.Tensor:
+    t = t.detach().cpu().contiguous()
+    return t.view({4: torch.int32, 2: torch.int16, 1: torch.uint8}[t.element_size()])
+
+
+class GpuLayer:
+    """Device copies of a workload's inputs plus the layer's buffers."""
+
+    def __init__(self, wl, device, inputs=None):
+        self.wl = wl
+        self.inputs = inputs if inputs is not None else workloads.layer_inputs(wl)
+        self.logits = self.inputs["logits"].to(device)
+        self.x = self.inputs["x"].to(device)
+        self.w13 = self.inputs["w13"].to(device)
+        self.w2 = self.inputs["w2"].to(device)
+        self.buf = moe.LayerBuffers(wl, device)
+
+    def run(self):
+        b, wl = self.buf, self.wl
+        moe.layer_forward(wl, self.logits, self.x, self.w13, self.w2, b)
+        torch.cuda.synchronize()
+        return moe.moe_check_status(b.dev_status)
+
+
+def sample_rows(lay: dict, T: int, k: int, n_tokens: int, seed: int = 0):
+    """Slots of a seeded token sample (all k pairs of each), plus the first
+    and last slot of every non-empty expert (the ragged M tails)."""
+    rng = np.random.default_rng(seed)
+    toks = np.sort(rng.choice(T, size=min(n_tokens, T), replace=False))
+    sop = lay["slot_of_pair"].numpy().reshape(T, k)
+    mask = np.zeros(T * k, dtype=bool)
+    mask[sop[toks].reshape(-1)] = True
+    off = lay["expert_offsets"].numpy()
+    for e in range(len(off) - 1):
+        if off[e + 1] > off[e]:
+            mask[off[e]] = True
+            mask[off[e + 1] - 1] = True
+    return torch.from_numpy(toks), torch.from_numpy(mask)
+
+
+def oracle_gemm_rows(wl, xp, sc, offsets, mask, w13=None, w2=None, batch=16):
+    """Oracle h and y for the masked slots.  Every output row depends only
+    on its own input row and its expert's weights, so the oracle runs on a
+    compact sub-problem: the sampled rows of up to ``batch`` experts at a
+    time, with those experts' weights (re-drawn per expert on the host
+    unless given).  Returns (slots, h, y), rows in ascending slot order."""
+    off = offsets.tolist()
+    todo = []
+    for e in range(wl.E):
+        lo, hi = off[e], off[e + 1]
+        sel = torch.nonzero(mask[lo:hi]).flatten() + lo
+        if sel.numel():
+            todo.append((e, sel))
+    slots, hs, ys = [], [], []
+    for i in range(0, len(todo), batch):
+        chunk = todo[i:i + batch]
+        sel = torch.cat([s for _, s in chunk])
+        a13 = torch.stack([w13[e] if w13 is not None else workloads.expert_w13(wl, e)
+                           for e, _ in chunk]).contiguous()
+        a2 = torch.stack([w2[e] if w2 is not None else workloads.expert_w2(wl, e)
+                          for e, _ in chunk]).contiguous()
+        xe = xp[sel].contiguous()
+        se = sc[sel].contiguous() if sc is not None else None
+        oe = torch.tensor([0] + list(np.cumsum([s.numel() for _, s in chunk])), dtype=torch.int32)
+        he, ye, done = oracle.grouped_gemm(xe, se, oe, 0, len(chunk), a13, a2)
+        assert done == sel.numel()
+        slots.append(sel)
+        hs.append(he)
+        ys.append(ye)
+    return torch.cat(slots), torch.cat(hs), torch.cat(ys)

@@ -1,0 +1,123 @@
+"""The C-ABI library loads, exports every symbol include/moe.h declares,
+and rejects invalid arguments on the host before launching anything.
+
+These run without a GPU: invalid calls return before any CUDA call, and
+the workspace-size queries are pure host arithmetic.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from expert_parallelism_b200 import moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+FAKE = ctypes.c_void_p(4096)   # never dereferenced: validation fails first
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from expert_parallelism_b200 import build
+    build.build()
+    return moe.load_library()
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_five_steps():
+    names = _declared()
+    for n in ["moe_route_topk", "moe_dispatch_layout", "moe_permute", "moe_grouped_gemm",
+              "moe_combine", "moe_check_status", "moe_status_str"]:
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported_and_bound(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+        assert name in moe.SIGNATURES, f"binding lacks {name}"
+
+
+def test_status_strings(lib):
+    assert moe.moe_status_str(0) == "MOE_OK"
+    assert moe.moe_status_str(1) == "MOE_ERR_INVALID_ARG"
+    assert moe.moe_status_str(4) == "MOE_ERR_TIMEOUT"
+
+
+def test_workspace_queries(lib):
+    n = lib.moe_dispatch_layout_workspace_bytes(8192, 8, 256)
+    assert n > 0 and n % 16 == 0
+    assert lib.moe_dispatch_layout_workspace_bytes(0, 8, 256) > 0     # T=0 still writes offsets
+    assert lib.moe_dispatch_layout_workspace_bytes(-1, 8, 256) == 0
+    assert lib.moe_grouped_gemm_workspace_bytes(100, 256, 64, moe.MOE_BF16, moe.MOE_BF16) == 0
+
+
+def test_route_rejects_before_launch(lib):
+    f = lib.moe_route_topk
+    assert f(FAKE, 10, 8, 9, FAKE, FAKE, None) == 1          # k > E
+    assert f(FAKE, 10, 8, 0, FAKE, FAKE, None) == 1          # k < 1
+    assert f(FAKE, -1, 8, 2, FAKE, FAKE, None) == 1          # T < 0
+    assert f(None, 10, 8, 2, FAKE, FAKE, None) == 1          # null input
+    assert f(FAKE, 10, 2048, 2, FAKE, FAKE, None) == 2       # E > 1024
+    assert f(FAKE, 10, 64, 17, FAKE, FAKE, None) == 2        # k > 16
+    assert f(None, 0, 8, 2, None, None, None) == 0           # empty batch: no-op
+
+
+def test_layout_rejects_before_launch(lib):
+    f = lib.moe_dispatch_layout
+    ws = lib.moe_dispatch_layout_workspace_bytes(10, 2, 8)
+    args = lambda **kw: [kw.get("idx", FAKE), 10, kw.get("k", 2), kw.get("E", 8), kw.get("W", 2),
+                         FAKE, FAKE, FAKE, FAKE, FAKE, kw.get("ws", FAKE),
+                         kw.get("wsb", ws), kw.get("st", FAKE), None]
+    assert f(*args(W=3)) == 1                 # ep_size must divide the number of experts
+    assert f(*args(W=16)) == 1                # more ranks than experts
+    assert f(*args(W=0)) == 1
+    assert f(*args(wsb=ws - 1)) == 1          # workspace too small
+    assert f(*args(ws=ctypes.c_void_p(4100))) == 1   # misaligned workspace
+    assert f(*args(st=None)) == 1             # no status word
+    assert f(*args(idx=None)) == 1
+    assert f(*args(E=2048, W=2)) == 2
+
+
+def test_permute_combine_gemm_reject_before_launch(lib):
+    p = lib.moe_permute
+    assert p(FAKE, moe.MOE_BF16, 10, 100, 2, FAKE, FAKE, moe.MOE_BF16, None, None) == 1   # H % 8
+    assert p(FAKE, moe.MOE_BF16, 10, 136, 2, FAKE, FAKE, moe.MOE_E4M3, FAKE, None) == 1   # H % 128
+    assert p(FAKE, moe.MOE_BF16, 10, 128, 2, FAKE, FAKE, moe.MOE_E4M3, None, None) == 1   # scales
+    assert p(FAKE, moe.MOE_E4M3, 10, 128, 2, FAKE, FAKE, moe.MOE_E4M3, FAKE, None) == 1   # x dtype
+    assert p(FAKE, moe.MOE_BF16, 10, 128, 2, FAKE, FAKE, moe.MOE_F32, None, None) == 1    # cast
+    assert p(ctypes.c_void_p(4098), moe.MOE_BF16, 10, 128, 2, FAKE, FAKE, moe.MOE_BF16, None,
+             None) == 1                                                                 # align
+    c = lib.moe_combine
+    assert c(FAKE, moe.MOE_E4M3, FAKE, FAKE, 10, 2, 128, FAKE, moe.MOE_BF16, None) == 1
+    assert c(FAKE, moe.MOE_BF16, FAKE, FAKE, 10, 0, 128, FAKE, moe.MOE_BF16, None) == 1
+    assert c(FAKE, moe.MOE_BF16, FAKE, FAKE, 10, 17, 128, FAKE, moe.MOE_BF16, None) == 2
+    g = lib.moe_grouped_gemm
+    base = [FAKE, moe.MOE_BF16, None, FAKE, 0, 8, 100, 256, 64, FAKE, FAKE, moe.MOE_BF16, FAKE,
+            FAKE, None, 0, FAKE, None]
+    bad = list(base); bad[8] = 60                      # I % 8
+    assert g(*bad) == 1
+    bad = list(base); bad[1] = moe.MOE_F32             # f32 payload with bf16 weights
+    assert g(*bad) == 1
+    bad = list(base); bad[1] = moe.MOE_E4M3            # FP8 payload needs scales
+    assert g(*bad) == 1
+    bad = list(base); bad[16] = None                   # status word
+    assert g(*bad) == 1
+    bad = list(base); bad[5] = 0                       # no experts
+    assert g(*bad) == 1
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    saved = moe._lib
+    moe._lib = None
+    try:
+        with pytest.raises(ImportError):
+            moe.load_library(str(tmp_path / "nope.so"))
+    finally:
+        moe._lib = saved

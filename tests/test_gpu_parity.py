@@ -1,0 +1,98 @@
+"""GPU parity: every step of the hot path, called through the C ABI, against
+the CPU oracle on the same seeded inputs.
+
+Small workloads (tiny and the extra ragged ones) are compared in full.
+The full-size workloads (mid, dsv3, skew, decode) are compared in full for
+routing, layout and the FP8/bf16 permute of a token sample, and on a
+seeded sample of rows for the GEMM and combine (all k rows of sampled
+tokens, plus the first and last row of every expert), with the same
+launches and sizes the benchmark times.  Full-size combine is also checked
+against a property that holds at any size: with identity experts it
+returns x bit for bit.
+"""
+import pytest
+import torch
+
+import oracle
+from expert_parallelism_b200 import moe, workloads
+
+from parity_helpers import (BF16_TOL, F32_TOL, GpuLayer, bits, h_ok, oracle_gemm_rows,
+                            rowwise_ok, sample_rows, tol_for, workload)
+
+SMALL = ["tiny", "small_f32", "small_bf16", "small_fp8", "ragged_bf16"]
+FULL = {"decode": 64, "mid": 192, "skew": 128, "dsv3": 96}   # name -> sampled tokens
+
+
+def _check_route_layout(wl, g: GpuLayer):
+    b = g.buf
+    idx_o, w_o = oracle.route_topk(g.inputs["logits"], wl.k)
+    assert torch.equal(b.topk_idx.cpu(), idx_o), "topk_idx differs"
+    wg = b.topk_w.cpu().double()
+    assert bool(((wg - w_o.double()).abs() <= 1e-5 * w_o.double().abs()).all()), "topk_w"
+    lay = oracle.dispatch_layout(idx_o, wl.E, wl.W)
+    for key in ["expert_counts", "expert_offsets", "rank_offsets", "slot_of_pair",
+                "pair_of_slot"]:
+        got = getattr(b, key).cpu()[:lay[key].numel()]
+        assert torch.equal(got, lay[key]), f"{key} differs"
+    return idx_o, w_o, lay
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name", SMALL)
+def test_small_layer_full_parity(name, cuda_device):
+    wl = workload(name)
+    g = GpuLayer(wl, cuda_device)
+    assert g.run() == 0
+    idx_o, w_o, lay = _check_route_layout(wl, g)
+    b = g.buf
+    xp_o, sc_o = oracle.permute(g.inputs["x"], wl.k, lay["pair_of_slot"], wl.payload)
+    assert torch.equal(bits(b.xp), bits(xp_o)), "xp differs"
+    if sc_o is not None:
+        assert torch.equal(bits(b.xp_scales), bits(sc_o)), "xp_scales differ"
+    h_o, y_o, done = oracle.grouped_gemm(xp_o, sc_o, lay["expert_offsets"], 0, wl.E,
+                                         g.inputs["w13"], g.inputs["w2"])
+    assert done == wl.N
+    wdt = workloads.TORCH_DTYPE[wl.wdt]
+    ok, worst = h_ok(b.h.cpu(), h_o, wdt)
+    assert ok, f"h: worst excess {worst:.3g}"
+    ok, worst = rowwise_ok(b.y.cpu(), y_o, tol_for(wdt))
+    assert ok, f"y: worst err/rms {worst:.3g} > {tol_for(wdt)}"
+    out_o = oracle.combine(y_o, lay["slot_of_pair"], w_o)
+    ok, worst = rowwise_ok(b.out.cpu(), out_o, tol_for(workloads.TORCH_DTYPE[wl.act]))
+    assert ok, f"out: worst err/rms {worst:.3g}"
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name", list(FULL))
+def test_full_size_layer_sampled_parity(name, cuda_device):
+    wl = workload(name)
+    g = GpuLayer(wl, cuda_device)
+    assert g.run() == 0
+    idx_o, w_o, lay = _check_route_layout(wl, g)
+    b = g.buf
+    toks, mask = sample_rows(lay, wl.T, wl.k, FULL[name])
+    # permute: the oracle writes only the sampled slots
+    pos = lay["pair_of_slot"].clone()
+    pos[~mask] = -1
+    xp_o, sc_o = oracle.permute(g.inputs["x"], wl.k, pos, wl.payload)
+    xp_g = b.xp.cpu()
+    assert torch.equal(bits(xp_g[mask]), bits(xp_o[mask])), "xp differs on sampled slots"
+    if sc_o is not None:
+        assert torch.equal(bits(b.xp_scales.cpu()[mask]), bits(sc_o[mask])), "scales differ"
+    slots, h_o, y_o = oracle_gemm_rows(wl, xp_o, sc_o, lay["expert_offsets"], mask)
+    ok, worst = h_ok(b.h.cpu()[slots], h_o, torch.bfloat16)
+    assert ok, f"h: worst excess {worst:.3g}"
+    ok, worst = rowwise_ok(b.y.cpu()[slots], y_o, BF16_TOL)
+    assert ok, f"y: worst err/rms {worst:.3g}"
+    # combine for the sampled tokens, from the oracle's own (exact) y rows
+    sop = lay["slot_of_pair"].view(wl.T, wl.k)[toks].reshape(-1)
+    compact = torch.searchsorted(slots, sop.long()).to(torch.int32)
+    assert torch.equal(slots[compact.long()], sop.long())
+    out_o = oracle.combine(y_o, compact, w_o[toks].contiguous())
+    ok, worst = rowwise_ok(b.out.cpu()[toks], out_o, BF16_TOL)
+    assert ok, f"out: worst err/rms {worst:.3g}"
+    # full size, identity experts: combine(xp) returns x exactly (bf16 payloads)
+    if wl.payload == "bf16":
+        moe.moe_combine(b.xp, b.slot_of_pair, b.topk_w, b.out)
+        torch.cuda.synchronize()
+        assert torch.equal(bits(b.out), bits(g.inputs["x"])), "identity combine != x"
