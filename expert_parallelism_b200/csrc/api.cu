@@ -26,7 +26,7 @@ cudaError_t launch_grouped_gemm_simt_f32(const float*, const int32_t*, int, int,
                                          cudaStream_t);
 cudaError_t launch_grouped_gemm_tc(const __nv_bfloat16*, const int32_t*, int, int, int64_t, int,
                                    int, const __nv_bfloat16*, const __nv_bfloat16*,
-                                   __nv_bfloat16*, __nv_bfloat16*, int32_t*, cudaStream_t);
+                                   __nv_bfloat16*, void*, bool, int32_t*, cudaStream_t);
 }  // namespace moe
 
 namespace moe {
@@ -113,14 +113,15 @@ moe_status moe_grouped_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_
                             const int32_t* expert_offsets, int32_t expert_begin,
                             int32_t n_experts, int64_t n_rows, int32_t H, int32_t I,
                             const void* w13, const void* w2, moe_dtype w_dtype, void* h, void* y,
-                            void* workspace, size_t workspace_bytes, int32_t* dev_status,
-                            void* stream) {
+                            moe_dtype y_dtype, void* workspace, size_t workspace_bytes,
+                            int32_t* dev_status, void* stream) {
     if (n_rows < 0 || H < 1 || I < 1 || (H % 8) != 0 || (I % 8) != 0) return MOE_ERR_INVALID_ARG;
     if (expert_begin < 0 || n_experts < 1) return MOE_ERR_INVALID_ARG;
     if (n_experts > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
     const bool f32 = (w_dtype == MOE_F32 && xp_dtype == MOE_F32);
     const bool bf16 = (w_dtype == MOE_BF16 && (xp_dtype == MOE_BF16 || xp_dtype == MOE_E4M3));
     if (!f32 && !bf16) return MOE_ERR_INVALID_ARG;
+    if (y_dtype != MOE_F32 && !(bf16 && y_dtype == MOE_BF16)) return MOE_ERR_INVALID_ARG;
     if (xp_dtype == MOE_E4M3 && ((H % 128) != 0 || !xp_scales)) return MOE_ERR_INVALID_ARG;
     if (!expert_offsets || !w13 || !w2 || !dev_status) return MOE_ERR_INVALID_ARG;
     if (n_rows == 0) return MOE_OK;
@@ -145,7 +146,7 @@ moe_status moe_grouped_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_
     }
     return cuda_status(launch_grouped_gemm_tc(
         a, expert_offsets, expert_begin, n_experts, n_rows, H, I, (const __nv_bfloat16*)w13,
-        (const __nv_bfloat16*)w2, (__nv_bfloat16*)h, (__nv_bfloat16*)y, dev_status, s));
+        (const __nv_bfloat16*)w2, (__nv_bfloat16*)h, y, y_dtype == MOE_F32, dev_status, s));
 }
 
 moe_status moe_combine(const void* y, moe_dtype y_dtype, const int32_t* slot_of_pair,

@@ -232,11 +232,36 @@ struct Params {
     int n_out;                // output columns (I in phase 1, H in phase 2)
     int n_ntiles;             // N tiles per M tile
     int n_rows;               // rows of A and out: stores never go past it
-    __nv_bfloat16* out;       // h (phase 1) or y (phase 2), row stride n_out
+    void* out;                // h (phase 1, bf16) or y (phase 2, OutT), row stride n_out
     int32_t* dev_status;
 };
 
-template <bool GLU>
+// 32 consecutive fp32 results of one row: 4 x 16-byte bf16 stores or
+// 8 x 16-byte fp32 stores, skipping pieces past n_out (n_out % 8 == 0).
+__device__ __forceinline__ void store_row32(__nv_bfloat16* orow, int col0, int n_out,
+                                            const float (&v)[32]) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int col = col0 + q * 8;
+        if (col < n_out)
+            st_v4(orow + col, make_uint4(pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]),
+                                         pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]),
+                                         pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]),
+                                         pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7])));
+    }
+}
+__device__ __forceinline__ void store_row32(float* orow, int col0, int n_out,
+                                            const float (&v)[32]) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const int col = col0 + q * 4;
+        if (col < n_out)
+            st_v4(orow + col, make_uint4(__float_as_uint(v[q * 4 + 0]), __float_as_uint(v[q * 4 + 1]),
+                                         __float_as_uint(v[q * 4 + 2]), __float_as_uint(v[q * 4 + 3])));
+    }
+}
+
+template <bool GLU, typename OutT>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a,
                            const __grid_constant__ CUtensorMap tmap_b, const Params p) {
@@ -394,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const int row = row0 + quarter * 32 + lane;
             const bool row_ok = row < row_end;
-            __nv_bfloat16* orow = p.out + (int64_t)row * p.n_out;
+            OutT* orow = reinterpret_cast<OutT*>(p.out) + (int64_t)row * p.n_out;
             const uint32_t tacc = tmem_base + lane_off + (uint32_t)(acc * BN);
             constexpr int kOutCols = GLU ? BN / 2 : BN;
 #pragma unroll 1
@@ -410,19 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 } else {
                     tmem_ld_wait();
                 }
-                if (row_ok) {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int col = n0 + c + q * 8;
-                        if (col < p.n_out) {
-                            st_v4(orow + col,
-                                  make_uint4(pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]),
-                                             pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]),
-                                             pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]),
-                                             pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7])));
-                        }
-                    }
-                }
+                if (row_ok) store_row32(orow, n0 + c, p.n_out, v);
             }
             tc_fence_before();
             mbar_arrive(tempty_bar(acc));
@@ -477,10 +490,10 @@ static int num_sms() {
     return sms;
 }
 
-template <bool GLU>
+template <bool GLU, typename OutT>
 static cudaError_t launch_phase(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p,
                                 cudaStream_t s) {
-    auto kern = grouped_gemm_tc_kernel<GLU>;
+    auto kern = grouped_gemm_tc_kernel<GLU, OutT>;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -491,11 +504,11 @@ static cudaError_t launch_phase(const CUtensorMap& ma, const CUtensorMap& mb, co
 }  // namespace tc
 
 // A [n_rows, H] bf16 (the payload, or its dequantised copy); W13 [n_exp, 2I,
-// H]; W2 [n_exp, H, I]; h [n_rows, I]; y [n_rows, H].
+// H]; W2 [n_exp, H, I]; h [n_rows, I] bf16; y [n_rows, H] in y_f32 ? fp32 : bf16.
 cudaError_t launch_grouped_gemm_tc(const __nv_bfloat16* a, const int32_t* offsets,
                                    int expert_begin, int n_experts, int64_t n_rows, int H, int I,
                                    const __nv_bfloat16* w13, const __nv_bfloat16* w2,
-                                   __nv_bfloat16* h, __nv_bfloat16* y, int32_t* dev_status,
+                                   __nv_bfloat16* h, void* y, bool y_f32, int32_t* dev_status,
                                    cudaStream_t s) {
     using namespace tc;
     CUtensorMap ma1, mb1, ma2, mb2;
@@ -526,11 +539,12 @@ cudaError_t launch_grouped_gemm_tc(const __nv_bfloat16* a, const int32_t* offset
     }
     Params p1{offsets, expert_begin, n_experts, H, I, (I + BN / 2 - 1) / (BN / 2), (int)n_rows,
               h, dev_status};
-    cudaError_t e = launch_phase<true>(ma1, mb1, p1, s);
+    cudaError_t e = launch_phase<true, __nv_bfloat16>(ma1, mb1, p1, s);
     if (e != cudaSuccess) return e;
     Params p2{offsets, expert_begin, n_experts, I, H, (H + BN - 1) / BN, (int)n_rows, y,
               dev_status};
-    e = launch_phase<false>(ma2, mb2, p2, s);
+    e = y_f32 ? launch_phase<false, float>(ma2, mb2, p2, s)
+              : launch_phase<false, __nv_bfloat16>(ma2, mb2, p2, s);
     note_launches(2);
     return e;
 }

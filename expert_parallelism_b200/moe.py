@@ -30,10 +30,12 @@ SIGNATURES = {
     "moe_route_topk": ([_P, _I64, _I32, _I32, _P, _P, _P], _I),
     "moe_dispatch_layout_workspace_bytes": ([_I64, _I32, _I32], _SZ),
     "moe_dispatch_layout": ([_P, _I64, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _SZ, _P, _P], _I),
+    "moe_dispatch_layout_noalloc_max_scratch_bytes": ([], _SZ),
+    "moe_dispatch_layout_noalloc": ([_P, _I64, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _P], _I),
     "moe_permute": ([_P, _I, _I64, _I32, _I32, _P, _P, _I, _P, _P], _I),
     "moe_grouped_gemm_workspace_bytes": ([_I64, _I32, _I32, _I, _I], _SZ),
-    "moe_grouped_gemm": ([_P, _I, _P, _P, _I32, _I32, _I64, _I32, _I32, _P, _P, _I, _P, _P, _P,
-                          _SZ, _P, _P], _I),
+    "moe_grouped_gemm": ([_P, _I, _P, _P, _I32, _I32, _I64, _I32, _I32, _P, _P, _I, _P, _P, _I,
+                          _P, _SZ, _P, _P], _I),
     "moe_combine": ([_P, _I, _P, _P, _I64, _I32, _I32, _P, _I, _P], _I),
     "moe_check_status": ([_P, _P], _I),
     "moe_status_str": ([_I], ctypes.c_char_p),
@@ -107,6 +109,16 @@ def moe_dispatch_layout(topk_idx, E, W, expert_counts, expert_offsets, rank_offs
         workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
 
 
+def moe_dispatch_layout_noalloc(topk_idx, E, W, expert_counts, expert_offsets, rank_offsets,
+                                slot_of_pair, pair_of_slot, dev_status, stream=None):
+    """moe_dispatch_layout without a workspace (scratch inside the library)."""
+    T, k = topk_idx.shape
+    _check("moe_dispatch_layout_noalloc", load_library().moe_dispatch_layout_noalloc(
+        _ptr(topk_idx), T, k, E, W, _ptr(expert_counts), _ptr(expert_offsets),
+        _ptr(rank_offsets), _ptr(slot_of_pair), _ptr(pair_of_slot), _ptr(dev_status),
+        _stream(stream)))
+
+
 def moe_permute(x, k, slot_of_pair, xp, xp_scales=None, stream=None):
     T, H = x.shape
     _check("moe_permute", load_library().moe_permute(
@@ -127,7 +139,7 @@ def moe_grouped_gemm(xp, xp_scales, expert_offsets, expert_begin, n_experts, w13
     _check("moe_grouped_gemm", load_library().moe_grouped_gemm(
         _ptr(xp), dtype_code(xp), _ptr(xp_scales), _ptr(expert_offsets), expert_begin,
         n_experts, n_rows, H, I, _ptr(w13), _ptr(w2), dtype_code(w13), _ptr(h), _ptr(y),
-        _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream)))
+        dtype_code(y), _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream)))
 
 
 def moe_combine(y, slot_of_pair, topk_w, out, stream=None):
@@ -176,7 +188,7 @@ class LayerBuffers:
                           if wl.payload == "e4m3" else None)
         wdt = TORCH_DTYPE[wl.wdt]
         self.h = torch.empty(N, I, dtype=wdt, device=dev)
-        self.y = torch.empty(N, H, dtype=wdt, device=dev)
+        self.y = torch.empty(N, H, dtype=TORCH_DTYPE[wl.ydt], device=dev)
         gb = moe_grouped_gemm_workspace_bytes(N, H, I, pdt, wdt)
         self.gemm_ws = torch.empty(gb, dtype=torch.uint8, device=dev) if gb else None
         self.out = torch.empty(T, H, dtype=TORCH_DTYPE[wl.act], device=dev)

@@ -26,13 +26,13 @@ def kernel_bytes(wl: Workload) -> dict:
     """Algorithmic HBM bytes per launch of each step (each input read once,
     each output written once)."""
     N, T, H, E, k, I = wl.N, wl.T, wl.H, wl.E, wl.k, wl.I
-    xb, pb, wb = ELEM_BYTES[wl.act], ELEM_BYTES[wl.payload], ELEM_BYTES[wl.wdt]
+    xb, pb, yb = ELEM_BYTES[wl.act], ELEM_BYTES[wl.payload], ELEM_BYTES[wl.ydt]
     scales = N * (H // 128) * 4 if wl.payload == "e4m3" else 0
     return {
         "route_topk": T * E * 4 + T * k * 8,
         "dispatch_layout": N * 4 + N * 8 + (2 * E + 1) * 4 + (wl.W + 1) * 4,
         "permute": T * H * xb + N * H * pb + scales,
-        "combine": N * H * wb + T * k * 8 + T * H * xb,
+        "combine": N * H * yb + T * k * 8 + T * H * xb,
     }
 
 

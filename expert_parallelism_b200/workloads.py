@@ -17,6 +17,10 @@ parallelism" (Transformers docs), section "How the sizes combine"):
   skew    16384  2880  128  4  2880  8  bf16 / bf16 / bf16, Zipf(1.2) router bias
   decode  64     7168  256  8  2048  8  bf16 / bf16 / bf16
 
+Expert outputs y are stored in fp32 for every workload (the combine then
+rounds only once, into out); h, the down projection's operand, has the
+GEMM's dtype.
+
 Distributions: router logits ~ N(0, 1) in fp32 (plus, for ``skew``, a
 per-expert bias log p_{pi(e)} with p_r proportional to r^-1.2 over a seeded
 permutation pi); x ~ N(0, 1) cast to the activation dtype; W13[e] ~
@@ -54,6 +58,7 @@ class Workload:
     router: str = "normal"   # "normal" | "zipf"
     zipf_s: float = 1.2
     seed: int = 0
+    ydt: str = "f32"         # storage of the experts' outputs y (combine's input)
 
     @property
     def N(self) -> int:

@@ -135,6 +135,38 @@ moe_status moe_dispatch_layout(const int32_t* topk_idx, int64_t T, int32_t k, in
                                size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /*
+ * moe_dispatch_layout_noalloc -- moe_dispatch_layout for callers that cannot
+ * allocate device memory.  The pages have no counterpart: this is a
+ * convenience of this library, not a step of the method.
+ *
+ * Some callers cannot hand the library a workspace: cudaMalloc may
+ * synchronise the device and is not allowed while a stream is being
+ * captured, and some host frameworks keep all device memory in their own
+ * allocator and give extensions no way to ask for scratch.  This variant
+ * takes the same inputs and outputs as moe_dispatch_layout, minus the
+ * workspace, and computes exactly the same results.
+ *
+ *   - Its scratch is one fixed array inside the library, of
+ *     moe_dispatch_layout_noalloc_max_scratch_bytes() bytes (2 MiB), which
+ *     every GPU that loads the library holds until the process exits.
+ *   - Sizes whose scratch would not fit (E * ceil(T*k / 2048) above about
+ *     262,000, e.g. more than ~2 million pairs at E = 256) return
+ *     MOE_ERR_UNSUPPORTED; moe_dispatch_layout handles those.
+ *   - It allocates nothing.  The first call on each device looks up the
+ *     array's device address (cudaGetSymbolAddress, with that device
+ *     current); make that first call before any stream capture.
+ *   - Every call shares the one array, so calls that overlap on the GPU
+ *     (on different streams, or from different threads) race: serialise
+ *     them, e.g. on one stream.  Nothing needs clearing between calls.
+ */
+size_t moe_dispatch_layout_noalloc_max_scratch_bytes(void);
+moe_status moe_dispatch_layout_noalloc(const int32_t* topk_idx, int64_t T, int32_t k, int32_t E,
+                                       int32_t W, int32_t* expert_counts,
+                                       int32_t* expert_offsets, int32_t* rank_offsets,
+                                       int32_t* slot_of_pair, int32_t* pair_of_slot,
+                                       int32_t* dev_status, void* stream);
+
+/*
  * moe_permute -- write every token's hidden vector into the slots of its
  * k pairs: xp[slot_of_pair[t*k + j]] = x[t] (the "sent = x[order]" of the
  * aiwiki sketch, done as a scatter so each x row is read once).
@@ -178,8 +210,14 @@ moe_status moe_permute(const void* x, moe_dtype x_dtype, int64_t T, int32_t H, i
  *                  read by the kernels, never by the host.
  *   w13            [n_experts, 2I, H] in w_dtype (gate rows, then up rows).
  *   w2             [n_experts, H, I] in w_dtype.
- *   h              [n_rows, I] in w_dtype, written for the experts' rows.
- *   y              [n_rows, H] in w_dtype, written for the experts' rows.
+ *   h              [n_rows, I] in w_dtype, written for the experts' rows (the
+ *                  down projection's operand, so it has the GEMM's dtype).
+ *   y              [n_rows, H] in y_dtype, written for the experts' rows:
+ *                  MOE_F32 (either path) or MOE_BF16 (bf16 path only).  fp32
+ *                  keeps the combine within 2e-2 of a row's RMS of the exact
+ *                  layer output; a bf16 y adds a second bf16 rounding before
+ *                  the weighted sum, which alone can take the largest
+ *                  elements of a row past that bound.
  *   workspace      device scratch of moe_grouped_gemm_workspace_bytes(...)
  *                  bytes (may be 0 / NULL when that is 0), 128-byte aligned.
  *   dev_status     int32 device word (MOE_DEV_TIMEOUT on a bounded wait
@@ -196,8 +234,8 @@ moe_status moe_grouped_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_
                             const int32_t* expert_offsets, int32_t expert_begin,
                             int32_t n_experts, int64_t n_rows, int32_t H, int32_t I,
                             const void* w13, const void* w2, moe_dtype w_dtype, void* h,
-                            void* y, void* workspace, size_t workspace_bytes,
-                            int32_t* dev_status, void* stream);
+                            void* y, moe_dtype y_dtype, void* workspace,
+                            size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /*
  * moe_combine -- un-permute plus the router-weighted sum of each token's k

@@ -4,8 +4,8 @@ C ABI and compare with the CPU oracle on the same seeded inputs.
 The oracle's floating-point results are exact (fp64, unrounded); the only
 narrow type inside its chain is h, the bf16 (or fp32) operand of the down
 projection.  Tolerances:
-  y, out (bf16):  per row, max |gpu - oracle| <= 2e-2 * RMS(oracle row)
-  y, out, h (fp32): per row, max |gpu - oracle| <= 1e-5 * RMS(oracle row)
+  y, out of a bf16 GEMM: per row, max |gpu - oracle| <= 2e-2 * RMS(oracle row)
+  y, out, h of the fp32 GEMM: per row, max |gpu - oracle| <= 1e-5 * RMS(oracle row)
   h (bf16, the GEMM's internal activation): per element,
                   |gpu - oracle| <= 2^-8 * |oracle| + 1e-3 * RMS(oracle row),
                   i.e. the bf16 rounding of that element (at most half an
@@ -42,8 +42,10 @@ def workload(name):
     return workloads.WORKLOADS.get(name) or EXTRA[name]
 
 
-def tol_for(dtype: torch.dtype) -> float:
-    return F32_TOL if dtype == torch.float32 else BF16_TOL
+def tol_for(gemm_dtype: torch.dtype) -> float:
+    """Row tolerance for y and out: by the dtype the GEMM computes in (a bf16
+    GEMM's fp32-stored y is still a bf16-GEMM result)."""
+    return F32_TOL if gemm_dtype == torch.float32 else BF16_TOL
 
 
 def rowwise_ok(got: torch.Tensor, ref: torch.Tensor, tol: float):

@@ -100,15 +100,19 @@ def test_permute_combine_gemm_reject_before_launch(lib):
     assert c(FAKE, moe.MOE_BF16, FAKE, FAKE, 10, 17, 128, FAKE, moe.MOE_BF16, None) == 2
     g = lib.moe_grouped_gemm
     base = [FAKE, moe.MOE_BF16, None, FAKE, 0, 8, 100, 256, 64, FAKE, FAKE, moe.MOE_BF16, FAKE,
-            FAKE, None, 0, FAKE, None]
+            FAKE, moe.MOE_F32, None, 0, FAKE, None]
     bad = list(base); bad[8] = 60                      # I % 8
     assert g(*bad) == 1
     bad = list(base); bad[1] = moe.MOE_F32             # f32 payload with bf16 weights
     assert g(*bad) == 1
     bad = list(base); bad[1] = moe.MOE_E4M3            # FP8 payload needs scales
     assert g(*bad) == 1
-    bad = list(base); bad[16] = None                   # status word
+    bad = list(base); bad[17] = None                   # status word
     assert g(*bad) == 1
+    bad = list(base); bad[14] = moe.MOE_E4M3           # y storage must be fp32 or bf16
+    assert g(*bad) == 1
+    bad = list(base); bad[1] = moe.MOE_F32; bad[11] = moe.MOE_F32; bad[14] = moe.MOE_BF16
+    assert g(*bad) == 1                                # fp32 GEMM stores y in fp32
     bad = list(base); bad[5] = 0                       # no experts
     assert g(*bad) == 1
 

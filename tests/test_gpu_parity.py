@@ -58,7 +58,7 @@ def test_small_layer_full_parity(name, cuda_device):
     ok, worst = rowwise_ok(b.y.cpu(), y_o, tol_for(wdt))
     assert ok, f"y: worst err/rms {worst:.3g} > {tol_for(wdt)}"
     out_o = oracle.combine(y_o, lay["slot_of_pair"], w_o)
-    ok, worst = rowwise_ok(b.out.cpu(), out_o, tol_for(workloads.TORCH_DTYPE[wl.act]))
+    ok, worst = rowwise_ok(b.out.cpu(), out_o, tol_for(wdt))
     assert ok, f"out: worst err/rms {worst:.3g}"
 
 
