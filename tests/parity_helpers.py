@@ -35,6 +35,9 @@ EXTRA = {
     "ragged_bf16": workloads.Workload("ragged_bf16", 777, 200, 6, 3, 136, 3, "bf16", "bf16",
                                       "bf16"),
     "small_f32": workloads.Workload("small_f32", 130, 72, 5, 3, 40, 5, "f32", "f32", "f32"),
+    # >= 512 rows per expert: the GEMM runs 256-row tiles on CTA pairs
+    "pair_bf16": workloads.Workload("pair_bf16", 2100, 256, 4, 2, 192, 2, "bf16", "bf16", "bf16"),
+    "pair_fp8": workloads.Workload("pair_fp8", 1500, 384, 4, 3, 320, 4, "bf16", "e4m3", "bf16"),
 }
 
 
