@@ -6,8 +6,10 @@
 
 One step = one pass of the whole hot path (router top-k -> dispatch layout
 -> permute -> grouped SwiGLU GEMM -> combine) over one batch of the
-workload, inputs resident in HBM.  L2 is flushed (a 512 MiB write) before
-every step, outside the step's CUDA events.  With N > 1 (torchrun), every
+workload, inputs resident in HBM.  When a step streams more than 4x the L2
+(126 MB) in expert weights, that alone evicts L2 between steps ("inputs
+larger than L2"); smaller workloads get an explicit 512 MiB write-flush
+before every step, outside the step's CUDA events.  With N > 1 (torchrun), every
 rank runs an independent replica of the layer on its own GPU (no
 collective on the data path: weak scaling); the per-step time is the max
 over ranks.  Rank 0 prints one JSON line.
@@ -35,6 +37,7 @@ from expert_parallelism_b200 import moe, traffic, workloads  # noqa: E402
 
 METRIC = "MoE-layer tokens/s (dispatch+grouped GEMM+combine); permute/combine HBM GB/s"
 L2_FLUSH_BYTES = 512 << 20
+L2_BYTES = 126 << 20
 
 
 def _peaks():
@@ -190,11 +193,21 @@ def run_reference(args, wl):
     print(json.dumps(line), flush=True)
 
 
+def _weight_bytes(wl):
+    return wl.E * 3 * wl.I * wl.H * workloads.ELEM_BYTES[wl.wdt]
+
+
+def _needs_flush(wl):
+    return _weight_bytes(wl) < 4 * L2_BYTES
+
+
 def _config(wl):
+    l2 = (f"flushed ({L2_FLUSH_BYTES >> 20} MiB write) before every step" if _needs_flush(wl)
+          else f"inputs larger than L2: {_weight_bytes(wl) / 1e9:.1f} GB of expert weights "
+               f"streamed per step")
     return {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "I": wl.I,
             "logical_ranks": wl.W, "activations": wl.act, "payload": wl.payload,
-            "gemm": wl.wdt, "router": wl.router, "seed": wl.seed,
-            "l2": f"flushed ({L2_FLUSH_BYTES >> 20} MiB write) before every step",
+            "gemm": wl.wdt, "y": wl.ydt, "router": wl.router, "seed": wl.seed, "l2": l2,
             "parallelism": "replicas (one independent layer per GPU)"}
 
 
@@ -216,28 +229,19 @@ def run_ours(args, wl):
     w2 = torch.empty(wl.E, wl.H, wl.I, dtype=wdt, device=dev)
     workloads.fill_expert_weights(wl, w13, w2)
     buf = moe.LayerBuffers(wl, dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES if _needs_flush(wl) else 16, dtype=torch.uint8,
+                        device=dev)
     stream = torch.cuda.current_stream()
 
-    names = ["route_topk", "dispatch_layout", "permute", "grouped_gemm", "combine"]
+    # spans between the 8 events moe_layer_forward records
+    names = ["route_topk", "dispatch_layout", "permute", "dequant_e4m3", "gemm_gate_up",
+             "gemm_down", "combine"]
 
     def step(evs):
-        evs[0].record(stream)
-        moe.moe_route_topk(logits, buf.topk_idx, buf.topk_w)
-        evs[1].record(stream)
-        moe.moe_dispatch_layout(buf.topk_idx, wl.E, wl.W, buf.expert_counts, buf.expert_offsets,
-                                buf.rank_offsets, buf.slot_of_pair, buf.pair_of_slot,
-                                buf.layout_ws, buf.dev_status)
-        evs[2].record(stream)
-        moe.moe_permute(x, wl.k, buf.slot_of_pair, buf.xp, buf.xp_scales)
-        evs[3].record(stream)
-        moe.moe_grouped_gemm(buf.xp, buf.xp_scales, buf.expert_offsets, 0, wl.E, w13, w2, buf.h,
-                             buf.y, buf.gemm_ws, buf.dev_status)
-        evs[4].record(stream)
-        moe.moe_combine(buf.y, buf.slot_of_pair, buf.topk_w, buf.out)
-        evs[5].record(stream)
+        # one C call: the five steps, with an event before, between and after them
+        moe.moe_layer_forward(wl, logits, x, w13, w2, buf, step_events=evs)
 
-    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(8)]
     for _ in range(args.warmup):
         flush.fill_(1)
         step(mk())
@@ -264,7 +268,7 @@ def run_ours(args, wl):
     for evs in all_evs:
         for j, n in enumerate(names):
             per[n].append(evs[j].elapsed_time(evs[j + 1]))
-        step_ms.append(evs[0].elapsed_time(evs[5]))
+        step_ms.append(evs[0].elapsed_time(evs[7]))
     ms = statistics.mean(step_ms)
     layer_ms = ms - statistics.mean(per["route_topk"])      # dispatch + GEMM + combine
     if ws > 1:
@@ -272,7 +276,8 @@ def run_ours(args, wl):
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms, layer_ms = float(t[0]), float(t[1])
 
-    # end to end through the C ABI from pinned host buffers
+    # end to end through the C ABI with HOST buffers: the call copies logits
+    # and x from pinned host memory, runs the layer and copies out back
     h_logits = inp["logits"].pin_memory()
     h_x = inp["x"].pin_memory()
     h_out = torch.empty(buf.out.shape, dtype=buf.out.dtype).pin_memory()
@@ -281,10 +286,7 @@ def run_ours(args, wl):
         flush.fill_(1)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        logits.copy_(h_logits, non_blocking=True)
-        x.copy_(h_x, non_blocking=True)
-        moe.layer_forward(wl, logits, x, w13, w2, buf)
-        h_out.copy_(buf.out, non_blocking=True)
+        moe.moe_layer_forward_host(wl, h_logits, h_x, h_out, logits, x, w13, w2, buf)
         e1.record(stream)
         torch.cuda.synchronize()
         if i >= args.warmup:
@@ -303,30 +305,39 @@ def run_ours(args, wl):
         kb = traffic.kernel_bytes(wl)
         fl = traffic.gemm_flops(wl)
         avg = {n: statistics.mean(v) for n, v in per.items()}
-        gemm_tflops = fl["total"] / (avg["grouped_gemm"] * 1e-3) / 1e12
+        gemm_ms = avg["dequant_e4m3"] + avg["gemm_gate_up"] + avg["gemm_down"]
         counts = buf.expert_counts.cpu()
         touched = int((counts > 0).sum())
+        tf = lambda flops, ms: flops / (ms * 1e-3) / 1e12
+        gbs = lambda b, ms: b / (ms * 1e-3) / 1e9
         kernels = {
             "route_topk": {"us": avg["route_topk"] * 1e3,
-                           "gbs": kb["route_topk"] / (avg["route_topk"] * 1e-3) / 1e9},
+                           "gbs": gbs(kb["route_topk"], avg["route_topk"])},
             "dispatch_layout": {"us": avg["dispatch_layout"] * 1e3},
             "permute": {"us": avg["permute"] * 1e3, "bytes": kb["permute"],
-                        "gbs": kb["permute"] / (avg["permute"] * 1e-3) / 1e9},
-            "grouped_gemm": {"us": avg["grouped_gemm"] * 1e3, "flops": fl["total"],
-                             "tflops": gemm_tflops,
-                             "weight_gbs": traffic.touched_weight_bytes(wl, touched)
-                             / (avg["grouped_gemm"] * 1e-3) / 1e9,
+                        "gbs": gbs(kb["permute"], avg["permute"])},
+            "grouped_gemm": {"us": gemm_ms * 1e3, "flops": fl["total"],
+                             "tflops": tf(fl["total"], gemm_ms),
+                             "dequant_e4m3_us": avg["dequant_e4m3"] * 1e3,
+                             "gate_up_us": avg["gemm_gate_up"] * 1e3,
+                             "gate_up_tflops": tf(fl["gate_up"], avg["gemm_gate_up"]),
+                             "down_us": avg["gemm_down"] * 1e3,
+                             "down_tflops": tf(fl["down"], avg["gemm_down"]),
+                             "weight_gbs": gbs(traffic.touched_weight_bytes(wl, touched), gemm_ms),
                              "experts_touched": touched},
             "combine": {"us": avg["combine"] * 1e3, "bytes": kb["combine"],
-                        "gbs": kb["combine"] / (avg["combine"] * 1e-3) / 1e9},
+                        "gbs": gbs(kb["combine"], avg["combine"])},
         }
         for n in ["permute", "combine", "route_topk"]:
             kernels[n]["hbm_frac"] = kernels[n]["gbs"] / peaks["hbm_gbs"]
-        prof = _profile_traffic()
-        roof = {"kernel": "grouped_gemm (gate/up + SwiGLU, then down)", "bound": "tensor",
-                "achieved": gemm_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": gemm_tflops / peaks["bf16_tflops"], "traffic": prof,
-                "peak_source": peaks["source"] + " burst bf16 (timed per call)"}
+        # the dominant kernel: the gate/up grouped GEMM (SwiGLU fused)
+        achieved = tf(fl["gate_up"], avg["gemm_gate_up"])
+        roof = {"kernel": "grouped_gemm_tc_kernel, gate/up + SwiGLU phase", "bound": "tensor",
+                "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"],
+                "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
+                "traffic": _profile_traffic(wl), "algorithmic_flops_per_launch": fl["gate_up"],
+                "peak_source": peaks["source"] + " bf16 burst (sustained also given)"}
         line = {
             "metric": METRIC, "value": ws * wl.T / (ms * 1e-3), "unit": "tokens/s",
             "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -349,13 +360,20 @@ def run_ours(args, wl):
         torch.distributed.destroy_process_group()
 
 
-def _profile_traffic():
-    """DRAM bytes per launch of the GEMM from the committed ncu summary, if
-    one matching the current kernel is recorded there."""
+def _profile_traffic(wl):
+    """DRAM bytes per launch of the gate/up GEMM kernel on this workload, from
+    the committed ncu summary -- None unless that summary was taken on the
+    same kernel source (checked by hash) and for this workload."""
+    import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
-            return json.load(f).get("grouped_gemm_bytes_per_launch")
+            rec = json.load(f)
+        src = os.path.join(ROOT, "expert_parallelism_b200", "csrc", "grouped_gemm_tc.cu")
+        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        if rec.get("source_sha256") != digest:
+            return None
+        return rec.get("gate_up_dram_bytes_per_launch", {}).get(wl.name)
     except Exception:
         return None
 
@@ -369,8 +387,15 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=12.0)
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override T (smaller cases of the same kernels, for profiling)")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="override E (must stay a multiple of the logical ranks)")
     args = ap.parse_args()
     wl = workloads.WORKLOADS[args.workload]
+    if args.tokens is not None or args.experts is not None:
+        wl = wl.replace(T=args.tokens or wl.T, E=args.experts or wl.E,
+                        name=f"{wl.name}[T={args.tokens or wl.T},E={args.experts or wl.E}]")
     if args.impl == "reference":
         run_reference(args, wl)
     else:

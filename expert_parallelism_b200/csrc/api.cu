@@ -23,10 +23,11 @@ cudaError_t launch_dequant_e4m3(const uint8_t*, const float*, const int32_t*, in
                                 int, __nv_bfloat16*, cudaStream_t);
 cudaError_t launch_grouped_gemm_simt_f32(const float*, const int32_t*, int, int, int64_t, int,
                                          int, const float*, const float*, float*, float*,
-                                         cudaStream_t);
+                                         cudaEvent_t, cudaStream_t);
 cudaError_t launch_grouped_gemm_tc(const __nv_bfloat16*, const int32_t*, int, int, int64_t, int,
                                    int, const __nv_bfloat16*, const __nv_bfloat16*,
-                                   __nv_bfloat16*, void*, bool, int32_t*, cudaStream_t);
+                                   __nv_bfloat16*, void*, bool, int32_t*, cudaEvent_t,
+                                   cudaStream_t);
 }  // namespace moe
 
 namespace moe {
@@ -48,16 +49,133 @@ moe_status cuda_status(cudaError_t e) {
     return MOE_ERR_CUDA;
 }
 
+
+// Host-side validation of each step (no launch).  *noop is set when the
+// arguments are valid and there is nothing to launch (an empty batch).
+moe_status check_route(const float* logits, int64_t T, int32_t E, int32_t k,
+                       const int32_t* topk_idx, const float* topk_w, bool* noop) {
+    *noop = false;
+    if (T < 0 || E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
+    if (E > MOE_MAX_EXPERTS || k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
+    if (T == 0) return *noop = true, MOE_OK;
+    if (!logits || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+moe_status check_layout(const int32_t* topk_idx, int64_t T, int32_t k, int32_t E, int32_t W,
+                        const int32_t* expert_counts, const int32_t* expert_offsets,
+                        const int32_t* rank_offsets, const int32_t* slot_of_pair,
+                        const int32_t* pair_of_slot, const void* workspace,
+                        size_t workspace_bytes, const int32_t* dev_status) {
+    if (T < 0 || k < 1 || E < 1 || W < 1 || W > E || (E % W) != 0) return MOE_ERR_INVALID_ARG;
+    if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+    if (T * (int64_t)k >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
+    if (!expert_counts || !expert_offsets || !rank_offsets || !workspace || !dev_status)
+        return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!topk_idx || !slot_of_pair || !pair_of_slot)) return MOE_ERR_INVALID_ARG;
+    if (workspace_bytes < layout_workspace_bytes(T, k, E) || !aligned16(workspace))
+        return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+moe_status check_permute(const void* x, moe_dtype x_dtype, int64_t T, int32_t H, int32_t k,
+                         const int32_t* slot_of_pair, const void* xp, moe_dtype xp_dtype,
+                         const float* xp_scales, bool* noop) {
+    *noop = false;
+    if (T < 0 || H < 1 || k < 1 || (H % 8) != 0) return MOE_ERR_INVALID_ARG;
+    if (!is_act_dtype(x_dtype)) return MOE_ERR_INVALID_ARG;
+    if (xp_dtype != x_dtype && xp_dtype != MOE_E4M3) return MOE_ERR_INVALID_ARG;
+    if (xp_dtype == MOE_E4M3 && ((H % 128) != 0 || !xp_scales)) return MOE_ERR_INVALID_ARG;
+    if (k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
+    if (T == 0) return *noop = true, MOE_OK;
+    if (!x || !slot_of_pair || !xp || !aligned16(x) || !aligned16(xp)) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+size_t gemm_workspace_bytes(int64_t n_rows, int32_t H, moe_dtype xp_dtype) {
+    if (n_rows < 0 || H < 1) return 0;
+    // FP8 payload: a bf16 copy of the dequantised rows for the GEMM's A.
+    return xp_dtype == MOE_E4M3 ? (size_t)n_rows * H * 2 : 0;
+}
+
+moe_status check_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_scales,
+                      const int32_t* expert_offsets, int32_t expert_begin, int32_t n_experts,
+                      int64_t n_rows, int32_t H, int32_t I, const void* w13, const void* w2,
+                      moe_dtype w_dtype, const void* h, const void* y, moe_dtype y_dtype,
+                      const void* workspace, size_t workspace_bytes, const int32_t* dev_status,
+                      bool* noop) {
+    *noop = false;
+    if (n_rows < 0 || H < 1 || I < 1 || (H % 8) != 0 || (I % 8) != 0) return MOE_ERR_INVALID_ARG;
+    if (expert_begin < 0 || n_experts < 1) return MOE_ERR_INVALID_ARG;
+    if (n_experts > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+    const bool f32 = (w_dtype == MOE_F32 && xp_dtype == MOE_F32);
+    const bool bf16 = (w_dtype == MOE_BF16 && (xp_dtype == MOE_BF16 || xp_dtype == MOE_E4M3));
+    if (!f32 && !bf16) return MOE_ERR_INVALID_ARG;
+    if (y_dtype != MOE_F32 && !(bf16 && y_dtype == MOE_BF16)) return MOE_ERR_INVALID_ARG;
+    if (xp_dtype == MOE_E4M3 && ((H % 128) != 0 || !xp_scales)) return MOE_ERR_INVALID_ARG;
+    if (!expert_offsets || !w13 || !w2 || !dev_status) return MOE_ERR_INVALID_ARG;
+    if (n_rows == 0) return *noop = true, MOE_OK;
+    if (!xp || !h || !y) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(xp) || !aligned16(w13) || !aligned16(w2) || !aligned16(h) || !aligned16(y))
+        return MOE_ERR_INVALID_ARG;
+    const size_t need = gemm_workspace_bytes(n_rows, H, xp_dtype);
+    if (need > 0 && (workspace_bytes < need || !workspace || ((uintptr_t)workspace & 127u)))
+        return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+moe_status check_combine(const void* y, moe_dtype y_dtype, const int32_t* slot_of_pair,
+                         const float* topk_w, int64_t T, int32_t k, int32_t H, const void* out,
+                         moe_dtype out_dtype, bool* noop) {
+    *noop = false;
+    if (T < 0 || H < 1 || k < 1 || (H % 8) != 0) return MOE_ERR_INVALID_ARG;
+    if (!is_act_dtype(y_dtype) || !is_act_dtype(out_dtype)) return MOE_ERR_INVALID_ARG;
+    if (k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
+    if (T == 0) return *noop = true, MOE_OK;
+    if (!y || !slot_of_pair || !topk_w || !out || !aligned16(y) || !aligned16(out))
+        return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+// ev_a (after the FP8 dequantisation, or at the start) and ev_b (between
+// the two GEMM phases) may be null.
+cudaError_t run_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_scales,
+                     const int32_t* expert_offsets, int32_t expert_begin, int32_t n_experts,
+                     int64_t n_rows, int32_t H, int32_t I, const void* w13, const void* w2,
+                     moe_dtype w_dtype, void* h, void* y, moe_dtype y_dtype, void* workspace,
+                     int32_t* dev_status, cudaStream_t s, cudaEvent_t ev_a = nullptr,
+                     cudaEvent_t ev_b = nullptr) {
+    cudaError_t e = cudaSuccess;
+    if (w_dtype == MOE_F32) {
+        if (ev_a) e = cudaEventRecord(ev_a, s);
+        if (e != cudaSuccess) return e;
+        return launch_grouped_gemm_simt_f32((const float*)xp, expert_offsets, expert_begin,
+                                            n_experts, n_rows, H, I, (const float*)w13,
+                                            (const float*)w2, (float*)h, (float*)y, ev_b, s);
+    }
+    const __nv_bfloat16* a = (const __nv_bfloat16*)xp;
+    if (xp_dtype == MOE_E4M3) {
+        e = launch_dequant_e4m3((const uint8_t*)xp, xp_scales, expert_offsets, expert_begin,
+                                n_experts, n_rows, H, (__nv_bfloat16*)workspace, s);
+        if (e != cudaSuccess) return e;
+        a = (const __nv_bfloat16*)workspace;
+    }
+    if (ev_a) e = cudaEventRecord(ev_a, s);
+    if (e != cudaSuccess) return e;
+    return launch_grouped_gemm_tc(a, expert_offsets, expert_begin, n_experts, n_rows, H, I,
+                                  (const __nv_bfloat16*)w13, (const __nv_bfloat16*)w2,
+                                  (__nv_bfloat16*)h, y, y_dtype == MOE_F32, dev_status, ev_b, s);
+}
+
 }  // namespace
 
 extern "C" {
 
 moe_status moe_route_topk(const float* logits, int64_t T, int32_t E, int32_t k,
                           int32_t* topk_idx, float* topk_w, void* stream) {
-    if (T < 0 || E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
-    if (E > MOE_MAX_EXPERTS || k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
-    if (T == 0) return MOE_OK;
-    if (!logits || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+    bool noop;
+    const moe_status st = check_route(logits, T, E, k, topk_idx, topk_w, &noop);
+    if (st != MOE_OK || noop) return st;
     return cuda_status(
         launch_route_topk(logits, T, E, k, topk_idx, topk_w, (cudaStream_t)stream));
 }
@@ -72,14 +190,10 @@ moe_status moe_dispatch_layout(const int32_t* topk_idx, int64_t T, int32_t k, in
                                int32_t* rank_offsets, int32_t* slot_of_pair,
                                int32_t* pair_of_slot, void* workspace, size_t workspace_bytes,
                                int32_t* dev_status, void* stream) {
-    if (T < 0 || k < 1 || E < 1 || W < 1 || W > E || (E % W) != 0) return MOE_ERR_INVALID_ARG;
-    if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
-    if (T * (int64_t)k >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
-    if (!expert_counts || !expert_offsets || !rank_offsets || !workspace || !dev_status)
-        return MOE_ERR_INVALID_ARG;
-    if (T > 0 && (!topk_idx || !slot_of_pair || !pair_of_slot)) return MOE_ERR_INVALID_ARG;
-    if (workspace_bytes < layout_workspace_bytes(T, k, E) || !aligned16(workspace))
-        return MOE_ERR_INVALID_ARG;
+    const moe_status st = check_layout(topk_idx, T, k, E, W, expert_counts, expert_offsets,
+                                       rank_offsets, slot_of_pair, pair_of_slot, workspace,
+                                       workspace_bytes, dev_status);
+    if (st != MOE_OK) return st;
     return cuda_status(launch_dispatch_layout(topk_idx, T, k, E, W, expert_counts,
                                               expert_offsets, rank_offsets, slot_of_pair,
                                               pair_of_slot, workspace, dev_status,
@@ -89,13 +203,10 @@ moe_status moe_dispatch_layout(const int32_t* topk_idx, int64_t T, int32_t k, in
 moe_status moe_permute(const void* x, moe_dtype x_dtype, int64_t T, int32_t H, int32_t k,
                        const int32_t* slot_of_pair, void* xp, moe_dtype xp_dtype,
                        float* xp_scales, void* stream) {
-    if (T < 0 || H < 1 || k < 1 || (H % 8) != 0) return MOE_ERR_INVALID_ARG;
-    if (!is_act_dtype(x_dtype)) return MOE_ERR_INVALID_ARG;
-    if (xp_dtype != x_dtype && xp_dtype != MOE_E4M3) return MOE_ERR_INVALID_ARG;
-    if (xp_dtype == MOE_E4M3 && ((H % 128) != 0 || !xp_scales)) return MOE_ERR_INVALID_ARG;
-    if (k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
-    if (T == 0) return MOE_OK;
-    if (!x || !slot_of_pair || !xp || !aligned16(x) || !aligned16(xp)) return MOE_ERR_INVALID_ARG;
+    bool noop;
+    const moe_status st =
+        check_permute(x, x_dtype, T, H, k, slot_of_pair, xp, xp_dtype, xp_scales, &noop);
+    if (st != MOE_OK || noop) return st;
     return cuda_status(launch_permute(x, x_dtype, T, H, k, slot_of_pair, xp, xp_dtype, xp_scales,
                                       (cudaStream_t)stream));
 }
@@ -104,9 +215,7 @@ size_t moe_grouped_gemm_workspace_bytes(int64_t n_rows, int32_t H, int32_t I, mo
                                         moe_dtype w_dtype) {
     (void)I;
     (void)w_dtype;
-    if (n_rows < 0 || H < 1) return 0;
-    // FP8 payload: a bf16 copy of the dequantised rows for the GEMM's A.
-    return xp_dtype == MOE_E4M3 ? (size_t)n_rows * H * 2 : 0;
+    return gemm_workspace_bytes(n_rows, H, xp_dtype);
 }
 
 moe_status moe_grouped_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_scales,
@@ -115,51 +224,128 @@ moe_status moe_grouped_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_
                             const void* w13, const void* w2, moe_dtype w_dtype, void* h, void* y,
                             moe_dtype y_dtype, void* workspace, size_t workspace_bytes,
                             int32_t* dev_status, void* stream) {
-    if (n_rows < 0 || H < 1 || I < 1 || (H % 8) != 0 || (I % 8) != 0) return MOE_ERR_INVALID_ARG;
-    if (expert_begin < 0 || n_experts < 1) return MOE_ERR_INVALID_ARG;
-    if (n_experts > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
-    const bool f32 = (w_dtype == MOE_F32 && xp_dtype == MOE_F32);
-    const bool bf16 = (w_dtype == MOE_BF16 && (xp_dtype == MOE_BF16 || xp_dtype == MOE_E4M3));
-    if (!f32 && !bf16) return MOE_ERR_INVALID_ARG;
-    if (y_dtype != MOE_F32 && !(bf16 && y_dtype == MOE_BF16)) return MOE_ERR_INVALID_ARG;
-    if (xp_dtype == MOE_E4M3 && ((H % 128) != 0 || !xp_scales)) return MOE_ERR_INVALID_ARG;
-    if (!expert_offsets || !w13 || !w2 || !dev_status) return MOE_ERR_INVALID_ARG;
-    if (n_rows == 0) return MOE_OK;
-    if (!xp || !h || !y) return MOE_ERR_INVALID_ARG;
-    if (!aligned16(xp) || !aligned16(w13) || !aligned16(w2) || !aligned16(h) || !aligned16(y))
-        return MOE_ERR_INVALID_ARG;
-    const size_t need = moe_grouped_gemm_workspace_bytes(n_rows, H, I, xp_dtype, w_dtype);
-    if (need > 0 && (workspace_bytes < need || !workspace || ((uintptr_t)workspace & 127u)))
-        return MOE_ERR_INVALID_ARG;
-    cudaStream_t s = (cudaStream_t)stream;
-    if (f32)
-        return cuda_status(launch_grouped_gemm_simt_f32(
-            (const float*)xp, expert_offsets, expert_begin, n_experts, n_rows, H, I,
-            (const float*)w13, (const float*)w2, (float*)h, (float*)y, s));
-    const __nv_bfloat16* a = (const __nv_bfloat16*)xp;
-    if (xp_dtype == MOE_E4M3) {
-        cudaError_t e = launch_dequant_e4m3((const uint8_t*)xp, xp_scales, expert_offsets,
-                                            expert_begin, n_experts, n_rows, H,
-                                            (__nv_bfloat16*)workspace, s);
-        if (e != cudaSuccess) return cuda_status(e);
-        a = (const __nv_bfloat16*)workspace;
-    }
-    return cuda_status(launch_grouped_gemm_tc(
-        a, expert_offsets, expert_begin, n_experts, n_rows, H, I, (const __nv_bfloat16*)w13,
-        (const __nv_bfloat16*)w2, (__nv_bfloat16*)h, y, y_dtype == MOE_F32, dev_status, s));
+    bool noop;
+    const moe_status st =
+        check_gemm(xp, xp_dtype, xp_scales, expert_offsets, expert_begin, n_experts, n_rows, H,
+                   I, w13, w2, w_dtype, h, y, y_dtype, workspace, workspace_bytes, dev_status,
+                   &noop);
+    if (st != MOE_OK || noop) return st;
+    return cuda_status(run_gemm(xp, xp_dtype, xp_scales, expert_offsets, expert_begin, n_experts,
+                                n_rows, H, I, w13, w2, w_dtype, h, y, y_dtype, workspace,
+                                dev_status, (cudaStream_t)stream));
 }
 
 moe_status moe_combine(const void* y, moe_dtype y_dtype, const int32_t* slot_of_pair,
                        const float* topk_w, int64_t T, int32_t k, int32_t H, void* out,
                        moe_dtype out_dtype, void* stream) {
-    if (T < 0 || H < 1 || k < 1 || (H % 8) != 0) return MOE_ERR_INVALID_ARG;
-    if (!is_act_dtype(y_dtype) || !is_act_dtype(out_dtype)) return MOE_ERR_INVALID_ARG;
-    if (k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
-    if (T == 0) return MOE_OK;
-    if (!y || !slot_of_pair || !topk_w || !out || !aligned16(y) || !aligned16(out))
-        return MOE_ERR_INVALID_ARG;
+    bool noop;
+    const moe_status st =
+        check_combine(y, y_dtype, slot_of_pair, topk_w, T, k, H, out, out_dtype, &noop);
+    if (st != MOE_OK || noop) return st;
     return cuda_status(launch_combine(y, y_dtype, slot_of_pair, topk_w, T, k, H, out, out_dtype,
                                       (cudaStream_t)stream));
+}
+
+static moe_status check_layer(const float* logits, const void* x, moe_dtype x_dtype, int64_t T,
+                              int32_t H, int32_t E, int32_t k, int32_t W, int32_t I,
+                              const void* w13, const void* w2, moe_dtype w_dtype,
+                              moe_dtype payload_dtype, moe_dtype y_dtype,
+                              const moe_layer_buffers* b, const void* out) {
+    if (!b) return MOE_ERR_INVALID_ARG;
+    bool noop;
+    moe_status st = check_route(logits, T, E, k, b->topk_idx, b->topk_w, &noop);
+    if (st == MOE_OK)
+        st = check_layout(b->topk_idx, T, k, E, W, b->expert_counts, b->expert_offsets,
+                          b->rank_offsets, b->slot_of_pair, b->pair_of_slot,
+                          b->layout_workspace, b->layout_workspace_bytes, b->dev_status);
+    if (st == MOE_OK)
+        st = check_permute(x, x_dtype, T, H, k, b->slot_of_pair, b->xp, payload_dtype,
+                           b->xp_scales, &noop);
+    if (st == MOE_OK)
+        st = check_gemm(b->xp, payload_dtype, b->xp_scales, b->expert_offsets, 0, E, T * k, H, I,
+                        w13, w2, w_dtype, b->h, b->y, y_dtype, b->gemm_workspace,
+                        b->gemm_workspace_bytes, b->dev_status, &noop);
+    if (st == MOE_OK)
+        st = check_combine(b->y, y_dtype, b->slot_of_pair, b->topk_w, T, k, H, out, x_dtype,
+                           &noop);
+    return st;
+}
+
+static cudaError_t launch_layer(const float* logits, const void* x, moe_dtype x_dtype, int64_t T,
+                                int32_t H, int32_t E, int32_t k, int32_t W, int32_t I,
+                                const void* w13, const void* w2, moe_dtype w_dtype,
+                                moe_dtype payload_dtype, moe_dtype y_dtype,
+                                const moe_layer_buffers* b, void* out, void* const* ev,
+                                cudaStream_t s) {
+    auto mark = [&](int i) {
+        return ev ? cudaEventRecord((cudaEvent_t)ev[i], s) : cudaSuccess;
+    };
+    cudaError_t e = mark(0);
+    if (e == cudaSuccess && T > 0) e = launch_route_topk(logits, T, E, k, b->topk_idx, b->topk_w, s);
+    if (e == cudaSuccess) e = mark(1);
+    if (e == cudaSuccess)
+        e = launch_dispatch_layout(b->topk_idx, T, k, E, W, b->expert_counts, b->expert_offsets,
+                                   b->rank_offsets, b->slot_of_pair, b->pair_of_slot,
+                                   b->layout_workspace, b->dev_status, s);
+    if (e == cudaSuccess) e = mark(2);
+    if (e == cudaSuccess && T > 0)
+        e = launch_permute(x, x_dtype, T, H, k, b->slot_of_pair, b->xp, payload_dtype,
+                           b->xp_scales, s);
+    if (e == cudaSuccess) e = mark(3);
+    if (e == cudaSuccess && T > 0) {
+        e = run_gemm(b->xp, payload_dtype, b->xp_scales, b->expert_offsets, 0, E, T * k, H, I,
+                     w13, w2, w_dtype, b->h, b->y, y_dtype, b->gemm_workspace, b->dev_status, s,
+                     ev ? (cudaEvent_t)ev[4] : nullptr, ev ? (cudaEvent_t)ev[5] : nullptr);
+    } else if (e == cudaSuccess) {
+        e = mark(4);
+        if (e == cudaSuccess) e = mark(5);
+    }
+    if (e == cudaSuccess) e = mark(6);
+    if (e == cudaSuccess && T > 0)
+        e = launch_combine(b->y, y_dtype, b->slot_of_pair, b->topk_w, T, k, H, out, x_dtype, s);
+    if (e == cudaSuccess) e = mark(7);
+    return e;
+}
+
+moe_status moe_layer_forward(const float* logits, const void* x, moe_dtype x_dtype, int64_t T,
+                             int32_t H, int32_t E, int32_t k, int32_t W, int32_t I,
+                             const void* w13, const void* w2, moe_dtype w_dtype,
+                             moe_dtype payload_dtype, moe_dtype y_dtype,
+                             const moe_layer_buffers* b, void* out, void* const* step_events,
+                             void* stream) {
+    const moe_status st = check_layer(logits, x, x_dtype, T, H, E, k, W, I, w13, w2, w_dtype,
+                                      payload_dtype, y_dtype, b, out);
+    if (st != MOE_OK) return st;
+    return cuda_status(launch_layer(logits, x, x_dtype, T, H, E, k, W, I, w13, w2, w_dtype,
+                                    payload_dtype, y_dtype, b, out, step_events,
+                                    (cudaStream_t)stream));
+}
+
+moe_status moe_layer_forward_host(const float* logits_host, const void* x_host, void* out_host,
+                                  float* logits_dev, void* x_dev, void* out_dev,
+                                  moe_dtype x_dtype, int64_t T, int32_t H, int32_t E, int32_t k,
+                                  int32_t W, int32_t I, const void* w13, const void* w2,
+                                  moe_dtype w_dtype, moe_dtype payload_dtype, moe_dtype y_dtype,
+                                  const moe_layer_buffers* b, void* const* step_events,
+                                  void* stream) {
+    const moe_status st = check_layer(logits_dev, x_dev, x_dtype, T, H, E, k, W, I, w13, w2,
+                                      w_dtype, payload_dtype, y_dtype, b, out_dev);
+    if (st != MOE_OK) return st;
+    if (T > 0 && (!logits_host || !x_host || !out_host)) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t xb = (x_dtype == MOE_F32 ? 4 : 2) * (size_t)T * H;
+    cudaError_t e = cudaSuccess;
+    if (T > 0) {
+        e = cudaMemcpyAsync(logits_dev, logits_host, sizeof(float) * (size_t)T * E,
+                            cudaMemcpyHostToDevice, s);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(x_dev, x_host, xb, cudaMemcpyHostToDevice, s);
+    }
+    if (e == cudaSuccess)
+        e = launch_layer(logits_dev, x_dev, x_dtype, T, H, E, k, W, I, w13, w2, w_dtype,
+                         payload_dtype, y_dtype, b, out_dev, step_events, s);
+    if (e == cudaSuccess && T > 0)
+        e = cudaMemcpyAsync(out_host, out_dev, xb, cudaMemcpyDeviceToHost, s);
+    return cuda_status(e);
 }
 
 moe_status moe_check_status(int32_t* dev_status, void* stream) {

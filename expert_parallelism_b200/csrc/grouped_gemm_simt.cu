@@ -159,12 +159,14 @@ cudaError_t launch_dequant_e4m3(const uint8_t* q, const float* scales, const int
 template <typename TA, typename TW>
 static cudaError_t simt_two_phase(const TA* xp, const int32_t* offsets, int expert_begin,
                                   int n_experts, int64_t n_rows, int H, int I, const TW* w13,
-                                  const TW* w2, TW* h, TW* y, cudaStream_t s) {
+                                  const TW* w2, TW* h, TW* y, cudaEvent_t ev_mid,
+                                  cudaStream_t s) {
     int64_t gy = (n_rows + kSimtBM - 1) / kSimtBM + n_experts;
     if (gy > 65535) gy = 65535;
     const dim3 g1((I + kSimtBN - 1) / kSimtBN, (unsigned)gy);
     simt_grouped_gemm_kernel<TA, TW, true><<<g1, 256, 0, s>>>(xp, H, w13, I, offsets,
                                                               expert_begin, n_experts, n_rows, h);
+    if (ev_mid) cudaEventRecord(ev_mid, s);
     const dim3 g2((H + kSimtBN - 1) / kSimtBN, (unsigned)gy);
     simt_grouped_gemm_kernel<TW, TW, false><<<g2, 256, 0, s>>>(h, I, w2, H, offsets,
                                                                expert_begin, n_experts, n_rows, y);
@@ -175,9 +177,9 @@ static cudaError_t simt_two_phase(const TA* xp, const int32_t* offsets, int expe
 cudaError_t launch_grouped_gemm_simt_f32(const float* xp, const int32_t* offsets,
                                          int expert_begin, int n_experts, int64_t n_rows, int H,
                                          int I, const float* w13, const float* w2, float* h,
-                                         float* y, cudaStream_t s) {
+                                         float* y, cudaEvent_t ev_mid, cudaStream_t s) {
     return simt_two_phase<float, float>(xp, offsets, expert_begin, n_experts, n_rows, H, I, w13,
-                                        w2, h, y, s);
+                                        w2, h, y, ev_mid, s);
 }
 
 }  // namespace moe

@@ -675,7 +675,7 @@ template <int NCTA>
 static cudaError_t run_gemm(const __nv_bfloat16* a, const int32_t* offsets, int expert_begin,
                             int n_experts, int64_t n_rows, int H, int I, const __nv_bfloat16* w13,
                             const __nv_bfloat16* w2, __nv_bfloat16* h, void* y, bool y_f32,
-                            int32_t* dev_status, cudaStream_t s) {
+                            int32_t* dev_status, cudaEvent_t ev_mid, cudaStream_t s) {
     using G = Geo<NCTA>;
     CUtensorMap ma1, mb1, ma2, mb2;
     {
@@ -706,6 +706,7 @@ static cudaError_t run_gemm(const __nv_bfloat16* a, const int32_t* offsets, int 
     Params p1{offsets, expert_begin, n_experts, H, I, (I + BN / 2 - 1) / (BN / 2), (int)n_rows,
               h, dev_status};
     cudaError_t e = launch_phase<true, __nv_bfloat16, NCTA>(ma1, mb1, p1, s);
+    if (e == cudaSuccess && ev_mid) e = cudaEventRecord(ev_mid, s);
     if (e != cudaSuccess) return e;
     Params p2{offsets, expert_begin, n_experts, I, H, (H + BN - 1) / BN, (int)n_rows, y,
               dev_status};
@@ -729,16 +730,17 @@ static int gemm_ctas_per_tile(int64_t n_rows, int n_experts) {
 
 // A [n_rows, H] bf16 (the payload, or its dequantised copy); W13 [n_exp, 2I,
 // H]; W2 [n_exp, H, I]; h [n_rows, I] bf16; y [n_rows, H] in y_f32 ? fp32 : bf16.
+// ev_mid (may be null) is recorded between the two phases.
 cudaError_t launch_grouped_gemm_tc(const __nv_bfloat16* a, const int32_t* offsets,
                                    int expert_begin, int n_experts, int64_t n_rows, int H, int I,
                                    const __nv_bfloat16* w13, const __nv_bfloat16* w2,
                                    __nv_bfloat16* h, void* y, bool y_f32, int32_t* dev_status,
-                                   cudaStream_t s) {
+                                   cudaEvent_t ev_mid, cudaStream_t s) {
     if (gemm_ctas_per_tile(n_rows, n_experts) == 2)
         return tc::run_gemm<2>(a, offsets, expert_begin, n_experts, n_rows, H, I, w13, w2, h, y,
-                               y_f32, dev_status, s);
+                               y_f32, dev_status, ev_mid, s);
     return tc::run_gemm<1>(a, offsets, expert_begin, n_experts, n_rows, H, I, w13, w2, h, y,
-                           y_f32, dev_status, s);
+                           y_f32, dev_status, ev_mid, s);
 }
 
 }  // namespace moe

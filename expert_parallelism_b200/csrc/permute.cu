@@ -9,7 +9,7 @@
 // The copy runs token-major: a CTA reads x[t] once (16-byte vector loads
 // that do not allocate in L1) and stores it to its k slots, so HBM sees
 // T*H*b bytes of reads and N*H*b' bytes of writes, the algorithmic
-// minimum.  In FP8 mode 16 lanes own one 128-element block: they reduce
+// minimum.  In FP8 mode 8 lanes own one 128-element block: they reduce
 // amax with shuffles, divide by 448 (IEEE), and convert x/scale (IEEE
 // division) with the hardware's round-to-nearest-even, saturating cvt.
 #include "common.cuh"
@@ -55,54 +55,89 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&f)[8]) {
     unpack16(ld_nc_v4(p), f);
 }
 
+// Four e4m3 codes of a / scale (IEEE divisions, RNE, saturating), packed
+// low byte first.
+__device__ __forceinline__ uint32_t quant4(float a, float b, float c, float d, float scale) {
+    const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
+        make_float2(__fdiv_rn(a, scale), __fdiv_rn(b, scale)), __NV_SATFINITE, __NV_E4M3);
+    const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+        make_float2(__fdiv_rn(c, scale), __fdiv_rn(d, scale)), __NV_SATFINITE, __NV_E4M3);
+    return (uint32_t)lo | ((uint32_t)hi << 16);
+}
+
+constexpr int kQuantThreads = 256;
+constexpr int kMaxBlocks = 64;           // scales staged in shared memory: H <= 8192
+
+// FP8 payload: one CTA per token (grid-stride).  8 lanes own a 128-element
+// block (16 elements each): amax by shuffles, scale = amax / 448, and
+// 16-byte stores of codes to each of the token's k slots.  The token's
+// scales are staged in shared memory and written as 16-byte vectors per
+// slot once the row is done.
 template <typename T>
-__global__ void __launch_bounds__(256) permute_e4m3_kernel(const T* __restrict__ x, int64_t T_,
-                                                           int H, int k,
-                                                           const int32_t* __restrict__ slot_of_pair,
-                                                           uint8_t* __restrict__ xp,
-                                                           float* __restrict__ xp_scales) {
+__global__ void __launch_bounds__(kQuantThreads) permute_e4m3_kernel(
+    const T* __restrict__ x, int64_t T_, int H, int k, const int32_t* __restrict__ slot_of_pair,
+    uint8_t* __restrict__ xp, float* __restrict__ xp_scales) {
     __shared__ int32_t s_slot[kMaxTopK];
+    __shared__ __align__(16) float s_scale[kMaxBlocks];
     const int nblk = H / 128;
-    const int half = (threadIdx.x >> 4) & 1;   // which 16-lane half of the warp
-    const int l16 = threadIdx.x & 15;
-    const int warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    const int l8 = threadIdx.x & 7;                 // lane within the block's 8
+    const int grp = threadIdx.x >> 3;               // block handled in this pass
+    const int ngrp = blockDim.x >> 3;
+    const bool vec_scales = (nblk % 4) == 0 && nblk <= kMaxBlocks;
     for (int64_t t = blockIdx.x; t < T_; t += gridDim.x) {
         if (threadIdx.x < k) s_slot[threadIdx.x] = slot_of_pair[t * k + threadIdx.x];
         __syncthreads();
-        // whole warps iterate together so the 16-lane shuffles stay converged
-        for (int g0 = 2 * warp; g0 < nblk; g0 += 2 * nwarps) {
-            const int g = g0 + half;
+        const T* row = x + t * H;
+        // whole warps iterate together so the 8-lane shuffles stay converged
+        for (int g0 = 0; g0 < nblk; g0 += ngrp) {
+            const int g = g0 + grp;
             const bool live = g < nblk;
-            float f[8];
+            float f[16];
             float amax = 0.0f;
             if (live) {
-                load8(x + t * H + g * 128 + l16 * 8, f);
+                float a8[8], b8[8];
+                load8(row + g * 128 + l8 * 16, a8);
+                load8(row + g * 128 + l8 * 16 + 8, b8);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+                for (int i = 0; i < 8; ++i) {
+                    f[i] = a8[i];
+                    f[8 + i] = b8[i];
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
             }
 #pragma unroll
-            for (int off = 8; off > 0; off >>= 1)
+            for (int off = 4; off > 0; off >>= 1)
                 amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
             if (!live) continue;
             float scale = __fdiv_rn(amax, 448.0f);
             if (scale == 0.0f) scale = 1.0f;
-            uint32_t packed[2];
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
-                    make_float2(__fdiv_rn(f[4 * i], scale), __fdiv_rn(f[4 * i + 1], scale)),
-                    __NV_SATFINITE, __NV_E4M3);
-                const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
-                    make_float2(__fdiv_rn(f[4 * i + 2], scale), __fdiv_rn(f[4 * i + 3], scale)),
-                    __NV_SATFINITE, __NV_E4M3);
-                packed[i] = (uint32_t)lo | ((uint32_t)hi << 16);
-            }
-            const uint2 q = make_uint2(packed[0], packed[1]);
+            const uint4 q = make_uint4(quant4(f[0], f[1], f[2], f[3], scale),
+                                       quant4(f[4], f[5], f[6], f[7], scale),
+                                       quant4(f[8], f[9], f[10], f[11], scale),
+                                       quant4(f[12], f[13], f[14], f[15], scale));
             for (int j = 0; j < k; ++j) {
                 const int32_t s = s_slot[j];
-                if (s < 0) continue;
-                *reinterpret_cast<uint2*>(xp + (int64_t)s * H + g * 128 + l16 * 8) = q;
-                if (l16 == 0) xp_scales[(int64_t)s * nblk + g] = scale;
+                if (s >= 0) st_v4(xp + (int64_t)s * H + g * 128 + l8 * 16, q);
+            }
+            if (l8 == 0) {
+                if (vec_scales) {
+                    s_scale[g] = scale;
+                } else {
+                    for (int j = 0; j < k; ++j)
+                        if (s_slot[j] >= 0) xp_scales[(int64_t)s_slot[j] * nblk + g] = scale;
+                }
+            }
+        }
+        if (vec_scales) {
+            __syncthreads();
+            const int nvec = nblk / 4;              // 16-byte pieces of one slot's scales
+            for (int i = threadIdx.x; i < k * nvec; i += blockDim.x) {
+                const int j = i / nvec, v = i - j * nvec;
+                const int32_t s = s_slot[j];
+                if (s >= 0)
+                    st_v4(xp_scales + (int64_t)s * nblk + v * 4,
+                          *reinterpret_cast<const uint4*>(s_scale + v * 4));
             }
         }
         __syncthreads();

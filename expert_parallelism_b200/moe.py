@@ -37,10 +37,24 @@ SIGNATURES = {
     "moe_grouped_gemm": ([_P, _I, _P, _P, _I32, _I32, _I64, _I32, _I32, _P, _P, _I, _P, _P, _I,
                           _P, _SZ, _P, _P], _I),
     "moe_combine": ([_P, _I, _P, _P, _I64, _I32, _I32, _P, _I, _P], _I),
+    "moe_layer_forward": ([_P, _P, _I, _I64, _I32, _I32, _I32, _I32, _I32, _P, _P, _I, _I, _I,
+                           _P, _P, _P, _P], _I),
+    "moe_layer_forward_host": ([_P, _P, _P, _P, _P, _P, _I, _I64, _I32, _I32, _I32, _I32, _I32,
+                                _P, _P, _I, _I, _I, _P, _P, _P], _I),
     "moe_check_status": ([_P, _P], _I),
     "moe_status_str": ([_I], ctypes.c_char_p),
     "moe_launch_count": ([], ctypes.c_uint64),
 }
+
+
+class LayerBuffersC(ctypes.Structure):
+    """moe_layer_buffers (include/moe.h)."""
+    _fields_ = [("topk_idx", _P), ("topk_w", _P), ("expert_counts", _P),
+                ("expert_offsets", _P), ("rank_offsets", _P), ("slot_of_pair", _P),
+                ("pair_of_slot", _P), ("layout_workspace", _P),
+                ("layout_workspace_bytes", _SZ), ("xp", _P), ("xp_scales", _P), ("h", _P),
+                ("y", _P), ("gemm_workspace", _P), ("gemm_workspace_bytes", _SZ),
+                ("dev_status", _P)]
 
 
 class MoEError(RuntimeError):
@@ -194,14 +208,56 @@ class LayerBuffers:
         self.out = torch.empty(T, H, dtype=TORCH_DTYPE[wl.act], device=dev)
 
 
-def layer_forward(wl, logits, x, w13, w2, buf: LayerBuffers, stream=None):
-    """The whole hot path: route -> layout -> permute -> grouped GEMM -> combine."""
-    moe_route_topk(logits, buf.topk_idx, buf.topk_w, stream)
-    moe_dispatch_layout(buf.topk_idx, wl.E, wl.W, buf.expert_counts, buf.expert_offsets,
-                        buf.rank_offsets, buf.slot_of_pair, buf.pair_of_slot, buf.layout_ws,
-                        buf.dev_status, stream)
-    moe_permute(x, wl.k, buf.slot_of_pair, buf.xp, buf.xp_scales, stream)
-    moe_grouped_gemm(buf.xp, buf.xp_scales, buf.expert_offsets, 0, wl.E, w13, w2, buf.h, buf.y,
-                     buf.gemm_ws, buf.dev_status, stream)
-    moe_combine(buf.y, buf.slot_of_pair, buf.topk_w, buf.out, stream)
+def _nbytes(t):
+    return 0 if t is None else t.numel() * t.element_size()
+
+
+def layer_buffers_c(buf: "LayerBuffers") -> LayerBuffersC:
+    return LayerBuffersC(
+        _ptr(buf.topk_idx), _ptr(buf.topk_w), _ptr(buf.expert_counts), _ptr(buf.expert_offsets),
+        _ptr(buf.rank_offsets), _ptr(buf.slot_of_pair), _ptr(buf.pair_of_slot),
+        _ptr(buf.layout_ws), _nbytes(buf.layout_ws), _ptr(buf.xp), _ptr(buf.xp_scales),
+        _ptr(buf.h), _ptr(buf.y), _ptr(buf.gemm_ws), _nbytes(buf.gemm_ws), _ptr(buf.dev_status))
+
+
+def _events(step_events, stream=None):
+    if step_events is None:
+        return None
+    s = torch.cuda.current_stream() if stream is None else stream
+    for e in step_events:
+        if not e.cuda_event:      # torch creates the CUDA event on its first record
+            e.record(s)
+    assert len(step_events) == 8, "8 events: see moe_layer_forward in include/moe.h"
+    arr = (ctypes.c_void_p * 8)(*[ctypes.c_void_p(e.cuda_event) for e in step_events])
+    return ctypes.cast(arr, ctypes.c_void_p), arr
+
+
+def moe_layer_forward(wl, logits, x, w13, w2, buf: "LayerBuffers", step_events=None,
+                      stream=None):
+    """The whole hot path in one C call (route, layout, permute, grouped
+    GEMM, combine); optionally records 8 torch.cuda.Events between the
+    kernels (see include/moe.h for their positions)."""
+    cb = layer_buffers_c(buf)
+    ev = _events(step_events, stream)
+    _check("moe_layer_forward", load_library().moe_layer_forward(
+        _ptr(logits), _ptr(x), dtype_code(x), wl.T, wl.H, wl.E, wl.k, wl.W, wl.I, _ptr(w13),
+        _ptr(w2), dtype_code(w13), dtype_code(buf.xp), dtype_code(buf.y), ctypes.byref(cb),
+        _ptr(buf.out), ev[0] if ev else None, _stream(stream)))
     return buf.out
+
+
+def moe_layer_forward_host(wl, logits_host, x_host, out_host, logits_dev, x_dev, w13, w2,
+                           buf: "LayerBuffers", step_events=None, stream=None):
+    """moe_layer_forward with host inputs/output (copies inside the call)."""
+    cb = layer_buffers_c(buf)
+    ev = _events(step_events, stream)
+    _check("moe_layer_forward_host", load_library().moe_layer_forward_host(
+        _ptr(logits_host), _ptr(x_host), _ptr(out_host), _ptr(logits_dev), _ptr(x_dev),
+        _ptr(buf.out), dtype_code(x_dev), wl.T, wl.H, wl.E, wl.k, wl.W, wl.I, _ptr(w13), _ptr(w2),
+        dtype_code(w13), dtype_code(buf.xp), dtype_code(buf.y), ctypes.byref(cb),
+        ev[0] if ev else None, _stream(stream)))
+
+
+def layer_forward(wl, logits, x, w13, w2, buf: "LayerBuffers", stream=None):
+    """The whole hot path: route -> layout -> permute -> grouped GEMM -> combine."""
+    return moe_layer_forward(wl, logits, x, w13, w2, buf, stream=stream)

@@ -259,6 +259,68 @@ moe_status moe_combine(const void* y, moe_dtype y_dtype, const int32_t* slot_of_
                        moe_dtype out_dtype, void* stream);
 
 /*
+ * moe_layer_forward -- the whole hot path in one call: moe_route_topk,
+ * moe_dispatch_layout, moe_permute, moe_grouped_gemm (every expert, local
+ * expert j = global expert j) and moe_combine, in that order on `stream`,
+ * with exactly the semantics of the five calls ("Expert parallelism and
+ * all-to-all", "Walking through one MoE layer", steps 1-4).  All five
+ * calls' arguments are validated before the first launch.
+ *
+ *   logits [T, E] fp32 and x [T, H] (x_dtype) are the layer's inputs;
+ *   w13 / w2 the stacked expert weights (w_dtype); out [T, H] in x_dtype.
+ *   b holds every intermediate buffer and workspace (device, caller
+ *   owned); b->xp is in payload_dtype (x_dtype or MOE_E4M3), b->y in
+ *   y_dtype.
+ *   step_events: NULL, or 8 cudaEvent_t handles recorded on `stream` at:
+ *   0 before routing, 1 after routing, 2 after the layout, 3 after the
+ *   permute, 4 after the FP8 dequantisation inside the GEMM (the same point
+ *   as 3 without an FP8 payload), 5 after the gate/up GEMM, 6 after the down
+ *   GEMM, 7 after combine -- so that a caller can time each kernel on the
+ *   stream it runs on, without launch gaps between them.
+ */
+typedef struct moe_layer_buffers {
+    int32_t* topk_idx;       /* [T, k] */
+    float* topk_w;           /* [T, k] */
+    int32_t* expert_counts;  /* [E] */
+    int32_t* expert_offsets; /* [E + 1] */
+    int32_t* rank_offsets;   /* [W + 1] */
+    int32_t* slot_of_pair;   /* [T*k] */
+    int32_t* pair_of_slot;   /* [T*k] */
+    void* layout_workspace;  /* moe_dispatch_layout_workspace_bytes(T, k, E) */
+    size_t layout_workspace_bytes;
+    void* xp;                /* [T*k, H] payload */
+    float* xp_scales;        /* [T*k, H/128] (FP8 payload only) */
+    void* h;                 /* [T*k, I] in w_dtype */
+    void* y;                 /* [T*k, H] in y_dtype */
+    void* gemm_workspace;    /* moe_grouped_gemm_workspace_bytes(...) */
+    size_t gemm_workspace_bytes;
+    int32_t* dev_status;     /* int32, zero-initialised */
+} moe_layer_buffers;
+
+moe_status moe_layer_forward(const float* logits, const void* x, moe_dtype x_dtype, int64_t T,
+                             int32_t H, int32_t E, int32_t k, int32_t W, int32_t I,
+                             const void* w13, const void* w2, moe_dtype w_dtype,
+                             moe_dtype payload_dtype, moe_dtype y_dtype,
+                             const moe_layer_buffers* b, void* out, void* const* step_events,
+                             void* stream);
+
+/*
+ * moe_layer_forward_host -- moe_layer_forward with the inputs and the
+ * output in HOST memory: copies logits and x from the host (cudaMemcpyAsync
+ * on `stream`; pinned host memory makes the copies asynchronous), runs the
+ * layer, and copies out back to the host.  logits_dev, x_dev and out_dev
+ * are device staging buffers of the same shapes.  Returns once everything
+ * is enqueued; synchronise the stream before reading out_host.
+ */
+moe_status moe_layer_forward_host(const float* logits_host, const void* x_host, void* out_host,
+                                  float* logits_dev, void* x_dev, void* out_dev,
+                                  moe_dtype x_dtype, int64_t T, int32_t H, int32_t E, int32_t k,
+                                  int32_t W, int32_t I, const void* w13, const void* w2,
+                                  moe_dtype w_dtype, moe_dtype payload_dtype, moe_dtype y_dtype,
+                                  const moe_layer_buffers* b, void* const* step_events,
+                                  void* stream);
+
+/*
  * moe_check_status -- synchronise `stream`, read the device status word,
  * clear it, and map it to a status: MOE_ERR_TIMEOUT if a wait ran out,
  * else MOE_ERR_BAD_INDEX if an id was skipped, else MOE_OK (MOE_ERR_CUDA if

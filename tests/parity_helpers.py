@@ -32,6 +32,8 @@ EXTRA = {
     # and ragged tails of the GEMM (partial M, N and K tiles)
     "small_bf16": workloads.Workload("small_bf16", 300, 256, 8, 2, 192, 2, "bf16", "bf16", "bf16"),
     "small_fp8": workloads.Workload("small_fp8", 200, 384, 16, 4, 320, 4, "bf16", "e4m3", "bf16"),
+    # H/128 a multiple of 4: block scales leave the permute as 16-byte vectors
+    "small_fp8v": workloads.Workload("small_fp8v", 120, 512, 8, 4, 64, 2, "bf16", "e4m3", "bf16"),
     "ragged_bf16": workloads.Workload("ragged_bf16", 777, 200, 6, 3, 136, 3, "bf16", "bf16",
                                       "bf16"),
     "small_f32": workloads.Workload("small_f32", 130, 72, 5, 3, 40, 5, "f32", "f32", "f32"),

@@ -125,3 +125,14 @@ def test_missing_library_fails_loudly(tmp_path):
             moe.load_library(str(tmp_path / "nope.so"))
     finally:
         moe._lib = saved
+
+
+def test_layer_call_rejects_before_launch(lib):
+    f = lib.moe_layer_forward
+    # no buffer struct
+    assert f(FAKE, FAKE, moe.MOE_BF16, 10, 128, 8, 2, 2, 64, FAKE, FAKE, moe.MOE_BF16,
+             moe.MOE_BF16, moe.MOE_F32, None, FAKE, None, None) == 1
+    cb = moe.LayerBuffersC(*([FAKE] * 8 + [0] + [FAKE] * 5 + [0] + [FAKE]))
+    # E % W != 0 is caught before anything runs (workspace size 0 too)
+    assert f(FAKE, FAKE, moe.MOE_BF16, 10, 128, 8, 2, 3, 64, FAKE, FAKE, moe.MOE_BF16,
+             moe.MOE_BF16, moe.MOE_F32, ctypes.byref(cb), FAKE, None, None) == 1

@@ -188,3 +188,38 @@ def test_layer_captures_in_a_cuda_graph(name, cuda_device):
     assert torch.equal(bits(g.buf.out), bits(eager))
     assert moe.moe_check_status(g.buf.dev_status) == 0
     del graph
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name", ["small_fp8", "ragged_bf16"])
+def test_layer_call_equals_the_five_calls(name, cuda_device):
+    """moe_layer_forward (one call, events between steps) and
+    moe_layer_forward_host (host inputs/output) give the five-call chain's
+    results bit for bit."""
+    from parity_helpers import workload
+    wl = workload(name)
+    g = GpuLayer(wl, cuda_device)
+    b = g.buf
+    moe.moe_route_topk(g.logits, b.topk_idx, b.topk_w)
+    moe.moe_dispatch_layout(b.topk_idx, wl.E, wl.W, b.expert_counts, b.expert_offsets,
+                            b.rank_offsets, b.slot_of_pair, b.pair_of_slot, b.layout_ws,
+                            b.dev_status)
+    moe.moe_permute(g.x, wl.k, b.slot_of_pair, b.xp, b.xp_scales)
+    moe.moe_grouped_gemm(b.xp, b.xp_scales, b.expert_offsets, 0, wl.E, g.w13, g.w2, b.h, b.y,
+                         b.gemm_ws, b.dev_status)
+    moe.moe_combine(b.y, b.slot_of_pair, b.topk_w, b.out)
+    torch.cuda.synchronize()
+    five = b.out.clone()
+    b.out.zero_()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(8)]
+    moe.moe_layer_forward(wl, g.logits, g.x, g.w13, g.w2, b, step_events=evs)
+    torch.cuda.synchronize()
+    assert torch.equal(bits(b.out), bits(five))
+    assert all(evs[i].elapsed_time(evs[i + 1]) >= 0 for i in range(7))
+    h_out = torch.zeros(b.out.shape, dtype=b.out.dtype).pin_memory()
+    moe.moe_layer_forward_host(wl, g.inputs["logits"].pin_memory(), g.inputs["x"].pin_memory(),
+                               h_out, torch.empty_like(g.logits), torch.empty_like(g.x), g.w13,
+                               g.w2, b)
+    torch.cuda.synchronize()
+    assert torch.equal(bits(h_out), bits(five))
+    assert moe.moe_check_status(b.dev_status) == 0

@@ -19,7 +19,8 @@ from expert_parallelism_b200 import moe, workloads
 from parity_helpers import (BF16_TOL, F32_TOL, GpuLayer, bits, h_ok, oracle_gemm_rows,
                             rowwise_ok, sample_rows, tol_for, workload)
 
-SMALL = ["tiny", "small_f32", "small_bf16", "small_fp8", "ragged_bf16", "pair_bf16", "pair_fp8"]
+SMALL = ["tiny", "small_f32", "small_bf16", "small_fp8", "small_fp8v", "ragged_bf16", "pair_bf16",
+         "pair_fp8"]
 FULL = {"decode": 64, "mid": 192, "skew": 128, "dsv3": 96}   # name -> sampled tokens
 
 
