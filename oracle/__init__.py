@@ -48,6 +48,9 @@ def _load():
         lib.oracle_route_topk.restype = I
         lib.oracle_dispatch_layout.argtypes = [P, I64, I32, I32, I32, P, P, P, P, P]
         lib.oracle_dispatch_layout.restype = I64
+        lib.oracle_dispatch_layout_capacity.argtypes = [P, I64, I32, I32, I32, I32, P, P, P, P,
+                                                         P, P]
+        lib.oracle_dispatch_layout_capacity.restype = I64
         lib.oracle_permute.argtypes = [P, I, I64, I32, I32, P, I64, P, I, P]
         lib.oracle_permute.restype = I
         lib.oracle_grouped_gemm.argtypes = [P, I, P, P, I32, I32, I32, I32, P, P, I, P, P, P, I]
@@ -123,6 +126,34 @@ def dispatch_layout(topk_idx: torch.Tensor, E: int, W: int):
                                          _p(rank_offsets), _p(slot_of_pair), _p(pair_of_slot))
     return dict(expert_counts=counts, expert_offsets=offsets, rank_offsets=rank_offsets,
                 slot_of_pair=slot_of_pair, pair_of_slot=pair_of_slot, skipped=int(bad))
+
+
+def dispatch_layout_capacity(topk_idx: torch.Tensor, E: int, W: int, C: int):
+    """Fixed-capacity layout: expert e's slab is rows [e*C, (e+1)*C), filled
+    by its earliest pairs; later pairs are dropped (slot -1).  Returns the
+    dropless layout's keys plus ``dropped``; ``expert_counts`` holds the
+    kept rows per expert and ``pair_of_slot`` has E*C entries."""
+    topk_idx = topk_idx.to(torch.int32).contiguous()
+    T, k = topk_idx.shape
+    counts = torch.empty(E, dtype=torch.int32)
+    offsets = torch.empty(E + 1, dtype=torch.int32)
+    rank_offsets = torch.empty(W + 1, dtype=torch.int32)
+    slot_of_pair = torch.empty(T * k, dtype=torch.int32)
+    pair_of_slot = torch.empty(max(E * C, 1), dtype=torch.int32)
+    skipped = ctypes.c_int64(0)
+    dropped = _load().oracle_dispatch_layout_capacity(
+        _p(topk_idx), T, k, E, W, C, _p(counts), _p(offsets), _p(rank_offsets),
+        _p(slot_of_pair), _p(pair_of_slot), ctypes.byref(skipped))
+    return dict(expert_counts=counts, expert_offsets=offsets, rank_offsets=rank_offsets,
+                slot_of_pair=slot_of_pair, pair_of_slot=pair_of_slot[:E * C],
+                dropped=int(dropped), skipped=int(skipped.value))
+
+
+def capacity_rows(T: int, k: int, E: int, capacity_factor: float) -> int:
+    """Rows per expert slab: ceil(capacity_factor * T * k / E) (the plainest
+    reading; the pages give no formula)."""
+    import math
+    return int(math.ceil(capacity_factor * T * k / E))
 
 
 def permute(x: torch.Tensor, k: int, pair_of_slot: torch.Tensor, payload: str,

@@ -227,6 +227,44 @@ int64_t oracle_dispatch_layout(const int32_t* idx, int64_t T, int32_t k, int32_t
 }
 
 /* ------------------------------------------------------------------ */
+/* S2' fixed-capacity dispatch layout (token dropping)                  */
+/* ------------------------------------------------------------------ */
+/* "Expert Parallelism" (aiwiki), "Implementation", the closing note on
+ * fixed capacity: with buffers of a fixed size every destination's size is
+ * known in advance, and the tokens that do not fit are dropped.  Reading
+ * (the page gives neither the size nor the drop rule): every expert e owns
+ * a fixed slab of C rows, [e*C, (e+1)*C); its pairs, taken in pair order
+ * (the stable order of the dropless layout), fill the slab from the top,
+ * and the pairs past the C-th are dropped (slot_of_pair = -1), so the
+ * earliest pairs keep their place.  counts[e] = min(#pairs of e, C) (the
+ * rows the experts compute), offsets[e] = e*C, rank_offsets[r] =
+ * offsets[r*E/W]; slab rows nobody fills hold pair_of_slot = -1.  Pairs
+ * with an expert id outside [0, E) are skipped as in the dropless layout.
+ * pair_of_slot has E*C entries.  Returns the number of dropped pairs;
+ * *skipped receives the number of out-of-range ids. */
+int64_t oracle_dispatch_layout_capacity(const int32_t* idx, int64_t T, int32_t k, int32_t E,
+                                        int32_t W, int32_t C, int32_t* counts,
+                                        int32_t* offsets, int32_t* rank_offsets,
+                                        int32_t* slot_of_pair, int32_t* pair_of_slot,
+                                        int64_t* skipped) {
+    int64_t N = T * k, dropped = 0, bad = 0;
+    for (int32_t e = 0; e < E; ++e) counts[e] = 0;
+    for (int32_t e = 0; e <= E; ++e) offsets[e] = e * C;
+    for (int32_t r = 0; r <= W; ++r) rank_offsets[r] = offsets[(int64_t)r * E / W];
+    for (int64_t s = 0; s < (int64_t)E * C; ++s) pair_of_slot[s] = -1;
+    for (int64_t p = 0; p < N; ++p) {
+        int32_t e = idx[p];
+        if (e < 0 || e >= E) { slot_of_pair[p] = -1; ++bad; continue; }
+        if (counts[e] >= C) { slot_of_pair[p] = -1; ++dropped; continue; }
+        int32_t s = offsets[e] + counts[e]++;
+        slot_of_pair[p] = s;
+        pair_of_slot[s] = (int32_t)p;
+    }
+    if (skipped) *skipped = bad;
+    return dropped;
+}
+
+/* ------------------------------------------------------------------ */
 /* S3 permute: xp[s] = x[pair_of_slot[s] / k], optional FP8 payload     */
 /* ------------------------------------------------------------------ */
 /* Same-dtype payload: a bitwise row copy.  FP8 payload: for every
