@@ -52,58 +52,114 @@ def _peaks():
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    """SM clock and clock-event (throttle) reasons sampled every 10 ms while
+    the timed region runs.  Reads NVML (the library nvidia-smi reports from),
+    for the device whose UUID the CUDA runtime gives; falls back to polling
+    nvidia-smi when NVML cannot be loaded.  Read-only: changes no setting."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
+    SMI_FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+                  "clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, device: torch.device, period_s: float = 0.01):
+        self.device = device
+        self.period = period_s
+        self.sm, self.max_mhz, self.reasons = [], None, set()
+        self.stop = threading.Event()
+        self.t = None
         self.proc = None
-        self.lines = []
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        uuid = str(torch.cuda.get_device_properties(self.device).uuid)
+        if not uuid.startswith("GPU-"):
+            uuid = "GPU-" + uuid
+        return pynvml, pynvml.nvmlDeviceGetHandleByUUID(uuid)
+
+    def _poll_nvml(self, nv, h):
+        self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        while not self.stop.is_set():
+            self.sm.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
+            bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+            for n, b in self.REASONS.items():
+                if bits & b:
+                    self.reasons.add(n)
+            self.stop.wait(self.period)
+
+    def _read_smi(self):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.proc.stdout:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 6:
+                continue
+            try:
+                self.sm.append(float(parts[0]))
+                self.max_mhz = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[2:6]):
+                if v.lower() == "active":
+                    self.reasons.add(n)
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
+            nv, h = self._nvml_handle()
+            self.t = threading.Thread(target=self._poll_nvml, args=(nv, h), daemon=True)
+            self.source = "nvml, 10 ms"
         except Exception:
-            self.proc = None
+            try:
+                idx = str(torch.cuda.get_device_properties(self.device).uuid)
+                idx = idx if idx.startswith("GPU-") else "GPU-" + idx
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", "-i", idx, f"--query-gpu={self.SMI_FIELDS}",
+                     "--format=csv,noheader,nounits", "-lms", "100"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.t = threading.Thread(target=self._read_smi, daemon=True)
+                self.source = "nvidia-smi, 100 ms"
+            except Exception:
+                self.t = None
+        if self.t is not None:
+            self.t.start()
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def __exit__(self, *a):
+        self.stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
+        if self.t is not None:
+            self.t.join(timeout=5)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        sm = sorted(self.sm)
+        pct = lambda q: sm[min(len(sm) - 1, int(q * len(sm)))] if sm else None
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                "sm_mhz_p10": pct(0.1), "sm_mhz_min": sm[0] if sm else None,
+                "reasons": sorted(self.reasons), "samples": len(sm), "source": self.source}
+
+
+def max_over_ranks(values, device):
+    """Element-wise max of per-rank times over the process group (identity
+    without one).  Every rank must call it, in the same order."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def whole_job_rate(units_per_rank: int, world_size: int, ms_max: float) -> float:
+    """Units all ranks processed divided by the slowest rank's time (weak
+    scaling: every rank runs the same per-GPU work)."""
+    return world_size * units_per_rank / (ms_max * 1e-3)
 
 
 def _dist():
@@ -129,19 +185,24 @@ def oracle_sample(wl, target_s: float = 12.0, max_tokens: int | None = None):
         lg, x = logits_all[:S].contiguous(), x_all[:S].contiguous()
         t0 = time.perf_counter()
         idx, w = oracle.route_topk(lg, wl.k)
-        lay = oracle.dispatch_layout(idx, wl.E, wl.W)
+        if wl.capacity_factor is None:
+            lay = oracle.dispatch_layout(idx, wl.E, wl.W)
+        else:
+            lay = oracle.dispatch_layout_capacity(
+                idx, wl.E, wl.W, oracle.capacity_rows(S, wl.k, wl.E, wl.capacity_factor))
         xp, sc = oracle.permute(x, wl.k, lay["pair_of_slot"], wl.payload)
         el = time.perf_counter() - t0
         off = lay["expert_offsets"].tolist()
-        touched = [e for e in range(wl.E) if off[e + 1] > off[e]]
+        cnt = lay["expert_counts"].tolist()         # rows each expert computes
+        touched = [e for e in range(wl.E) if cnt[e] > 0]
         for e in touched:
             if e not in cache:
                 cache[e] = (workloads.expert_w13(wl, e), workloads.expert_w2(wl, e))
-        y = torch.empty(sub.N, wl.H, dtype=torch.float64)
+        y = torch.zeros(xp.shape[0], wl.H, dtype=torch.float64)
         for i in range(0, len(touched), 32):
             grp = touched[i:i + 32]
-            rows = torch.cat([torch.arange(off[e], off[e + 1]) for e in grp])
-            oe = torch.tensor([0] + list(torch.tensor([off[e + 1] - off[e] for e in grp])
+            rows = torch.cat([torch.arange(off[e], off[e] + cnt[e]) for e in grp])
+            oe = torch.tensor([0] + list(torch.tensor([cnt[e] for e in grp])
                                          .cumsum(0).tolist()), dtype=torch.int32)
             a13 = torch.stack([cache[e][0] for e in grp])
             a2 = torch.stack([cache[e][1] for e in grp])
@@ -201,6 +262,12 @@ def _needs_flush(wl):
     return _weight_bytes(wl) < 4 * L2_BYTES
 
 
+def _capacity_info(buf, dropped):
+    if buf.capacity < 0:
+        return {}
+    return {"capacity_rows_per_expert": buf.capacity, "pairs_dropped": dropped}
+
+
 def _config(wl):
     l2 = (f"flushed ({L2_FLUSH_BYTES >> 20} MiB write) before every step" if _needs_flush(wl)
           else f"inputs larger than L2: {_weight_bytes(wl) / 1e9:.1f} GB of expert weights "
@@ -208,6 +275,7 @@ def _config(wl):
     return {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "I": wl.I,
             "logical_ranks": wl.W, "activations": wl.act, "payload": wl.payload,
             "gemm": wl.wdt, "y": wl.ydt, "router": wl.router, "seed": wl.seed, "l2": l2,
+            **({"capacity_factor": wl.capacity_factor} if wl.capacity_factor is not None else {}),
             "parallelism": "replicas (one independent layer per GPU)"}
 
 
@@ -255,14 +323,14 @@ def run_ours(args, wl):
     if ws > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    with ClockSampler(dev) as clk:
         for i in range(args.steps):
             flush.fill_(1)
             step(all_evs[i])
         torch.cuda.synchronize()
     if ws > 1:
         torch.distributed.barrier()
-    launches = (lib.moe_launch_count() - launches0) // max(args.steps, 1)
+    launches = lib.moe_launch_count() - launches0      # over the whole timed region
     per = {n: [] for n in names}
     step_ms = []
     for evs in all_evs:
@@ -271,10 +339,7 @@ def run_ours(args, wl):
         step_ms.append(evs[0].elapsed_time(evs[7]))
     ms = statistics.mean(step_ms)
     layer_ms = ms - statistics.mean(per["route_topk"])      # dispatch + GEMM + combine
-    if ws > 1:
-        t = torch.tensor([ms, layer_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms, layer_ms = float(t[0]), float(t[1])
+    ms, layer_ms = max_over_ranks([ms, layer_ms], dev)
 
     # end to end through the C ABI with HOST buffers: the call copies logits
     # and x from pinned host memory, runs the layer and copies out back
@@ -292,18 +357,22 @@ def run_ours(args, wl):
         if i >= args.warmup:
             e2e_ms.append(e0.elapsed_time(e1))
     e2e = statistics.mean(e2e_ms)
-    if ws > 1:
-        t = torch.tensor([e2e], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e = float(t[0])
+    (e2e,) = max_over_ranks([e2e], dev)
+    # the whole layer captured once in a CUDA graph and replayed: median
+    # device time per replay (launch overhead of the separate calls removed)
+    graph_us, replays = _graph_replay_us(wl, logits, x, w13, w2, buf, 100 if wl.T <= 1024 else 20)
+    (graph_us,) = max_over_ranks([graph_us], dev)
     st = moe.moe_check_status(buf.dev_status)
     if st != 0:
         raise RuntimeError(f"device status after timing: {moe.STATUS.get(st, st)}")
 
     if rank == 0:
         peaks = _peaks()
-        kb = traffic.kernel_bytes(wl)
-        fl = traffic.gemm_flops(wl)
+        # rows the experts computed: all T*k, or the kept ones under a capacity
+        dropped = int(buf.n_dropped.cpu()[0]) if buf.capacity >= 0 else 0
+        rows = wl.N - dropped
+        kb = traffic.kernel_bytes(wl, rows)
+        fl = traffic.gemm_flops(wl, rows)
         avg = {n: statistics.mean(v) for n, v in per.items()}
         gemm_ms = avg["dequant_e4m3"] + avg["gemm_gate_up"] + avg["gemm_down"]
         counts = buf.expert_counts.cpu()
@@ -332,25 +401,31 @@ def run_ours(args, wl):
             kernels[n]["hbm_frac"] = kernels[n]["gbs"] / peaks["hbm_gbs"]
         # the dominant kernel: the gate/up grouped GEMM (SwiGLU fused)
         achieved = tf(fl["gate_up"], avg["gemm_gate_up"])
-        roof = {"kernel": "grouped_gemm_tc_kernel, gate/up + SwiGLU phase", "bound": "tensor",
-                "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops"],
-                "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
+        # timed inside a long run of back-to-back steps under the 1000 W cap:
+        # the sustained bf16 peak is the denominator (burst fraction also given)
+        roof = {"kernel": "grouped GEMM, gate/up + SwiGLU phase", "bound": "tensor",
+                "achieved": achieved, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops_sustained"],
+                "frac_of_burst": achieved / peaks["bf16_tflops"],
                 "traffic": _profile_traffic(wl), "algorithmic_flops_per_launch": fl["gate_up"],
-                "peak_source": peaks["source"] + " bf16 burst (sustained also given)"}
+                "peak_source": peaks["source"] + " bf16 sustained (burst fraction also given)"}
         line = {
-            "metric": METRIC, "value": ws * wl.T / (ms * 1e-3), "unit": "tokens/s",
+            "metric": METRIC, "value": whole_job_rate(wl.T, ws, ms), "unit": "tokens/s",
             "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic", "config": _config(wl),
-            "layer_tokens_per_s": ws * wl.T / (layer_ms * 1e-3),
+            "data": "synthetic", "config": dict(_config(wl), **_capacity_info(buf, dropped)),
+            "layer_tokens_per_s": whole_job_rate(wl.T, ws, layer_ms),
             "layer_ms_excl_route": layer_ms,
             "kernels": kernels, "roofline": roof,
-            "e2e": {"value": ws * wl.T / (e2e * 1e-3), "unit": "tokens/s",
+            "e2e": {"value": whole_job_rate(wl.T, ws, e2e), "unit": "tokens/s",
                     "h2d_bytes_per_step": h_logits.numel() * 4 + h_x.numel() * h_x.element_size(),
                     "d2h_bytes_per_step": h_out.numel() * h_out.element_size(),
                     "ms_per_step": e2e},
-            "gpu_launches": int(launches), "clocks": clk.summary(),
+            "graph": {"us_median_per_layer": graph_us, "replays": replays,
+                      "tokens_per_s": whole_job_rate(wl.T, ws, graph_us * 1e-3)},
+            "gpu_launches": int(launches),
+            "gpu_launches_per_step": int(launches) // max(args.steps, 1),
+            "clocks": clk.summary(),
         }
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = oracle_sample(wl)
@@ -358,6 +433,31 @@ def run_ours(args, wl):
     if ws > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
+
+
+def _graph_replay_us(wl, logits, x, w13, w2, buf, replays):
+    """Capture moe_layer_forward in one CUDA graph on a side stream, replay
+    it ``replays`` times with events around each replay; median in us."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        moe.moe_layer_forward(wl, logits, x, w13, w2, buf, stream=s)
+        s.synchronize()
+        with torch.cuda.graph(graph, stream=s):
+            moe.moe_layer_forward(wl, logits, x, w13, w2, buf, stream=s)
+        for _ in range(3):
+            graph.replay()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(replays)]
+        for a, b in evs:
+            a.record(s)
+            graph.replay()
+            b.record(s)
+        s.synchronize()
+    times = [a.elapsed_time(b) * 1e3 for a, b in evs]
+    del graph
+    return statistics.median(times), replays
 
 
 def _profile_traffic(wl):
@@ -381,7 +481,7 @@ def _profile_traffic(wl):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="dsv3", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

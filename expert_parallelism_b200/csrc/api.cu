@@ -13,19 +13,20 @@
 namespace moe {
 cudaError_t launch_route_topk(const float*, int64_t, int, int, int32_t*, float*, cudaStream_t);
 size_t layout_workspace_bytes(int64_t T, int k, int E);
-cudaError_t launch_dispatch_layout(const int32_t*, int64_t, int, int, int, int32_t*, int32_t*,
-                                   int32_t*, int32_t*, int32_t*, void*, int32_t*, cudaStream_t);
+cudaError_t launch_dispatch_layout(const int32_t*, int64_t, int, int, int, int, int32_t*,
+                                   int32_t*, int32_t*, int32_t*, int32_t*, int32_t*, void*,
+                                   int32_t*, cudaStream_t);
 cudaError_t launch_permute(const void*, moe_dtype, int64_t, int, int, const int32_t*, void*,
                            moe_dtype, float*, cudaStream_t);
 cudaError_t launch_combine(const void*, moe_dtype, const int32_t*, const float*, int64_t, int,
                            int, void*, moe_dtype, cudaStream_t);
 cudaError_t launch_dequant_e4m3(const uint8_t*, const float*, const int32_t*, int, int, int64_t,
                                 int, __nv_bfloat16*, cudaStream_t);
-cudaError_t launch_grouped_gemm_simt_f32(const float*, const int32_t*, int, int, int64_t, int,
-                                         int, const float*, const float*, float*, float*,
-                                         cudaEvent_t, cudaStream_t);
-cudaError_t launch_grouped_gemm_tc(const __nv_bfloat16*, const int32_t*, int, int, int64_t, int,
-                                   int, const __nv_bfloat16*, const __nv_bfloat16*,
+cudaError_t launch_grouped_gemm_simt_f32(const float*, const int32_t*, const int32_t*, int, int,
+                                         int64_t, int, int, const float*, const float*, float*,
+                                         float*, cudaEvent_t, cudaStream_t);
+cudaError_t launch_grouped_gemm_tc(const __nv_bfloat16*, const int32_t*, const int32_t*, int, int,
+                                   int64_t, int, int, const __nv_bfloat16*, const __nv_bfloat16*,
                                    __nv_bfloat16*, void*, bool, int32_t*, cudaEvent_t,
                                    cudaStream_t);
 }  // namespace moe
@@ -140,7 +141,8 @@ moe_status check_combine(const void* y, moe_dtype y_dtype, const int32_t* slot_o
 // ev_a (after the FP8 dequantisation, or at the start) and ev_b (between
 // the two GEMM phases) may be null.
 cudaError_t run_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_scales,
-                     const int32_t* expert_offsets, int32_t expert_begin, int32_t n_experts,
+                     const int32_t* expert_offsets, const int32_t* expert_counts,
+                     int32_t expert_begin, int32_t n_experts,
                      int64_t n_rows, int32_t H, int32_t I, const void* w13, const void* w2,
                      moe_dtype w_dtype, void* h, void* y, moe_dtype y_dtype, void* workspace,
                      int32_t* dev_status, cudaStream_t s, cudaEvent_t ev_a = nullptr,
@@ -149,9 +151,10 @@ cudaError_t run_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_scales,
     if (w_dtype == MOE_F32) {
         if (ev_a) e = cudaEventRecord(ev_a, s);
         if (e != cudaSuccess) return e;
-        return launch_grouped_gemm_simt_f32((const float*)xp, expert_offsets, expert_begin,
-                                            n_experts, n_rows, H, I, (const float*)w13,
-                                            (const float*)w2, (float*)h, (float*)y, ev_b, s);
+        return launch_grouped_gemm_simt_f32((const float*)xp, expert_offsets, expert_counts,
+                                            expert_begin, n_experts, n_rows, H, I,
+                                            (const float*)w13, (const float*)w2, (float*)h,
+                                            (float*)y, ev_b, s);
     }
     const __nv_bfloat16* a = (const __nv_bfloat16*)xp;
     if (xp_dtype == MOE_E4M3) {
@@ -162,7 +165,8 @@ cudaError_t run_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_scales,
     }
     if (ev_a) e = cudaEventRecord(ev_a, s);
     if (e != cudaSuccess) return e;
-    return launch_grouped_gemm_tc(a, expert_offsets, expert_begin, n_experts, n_rows, H, I,
+    return launch_grouped_gemm_tc(a, expert_offsets, expert_counts, expert_begin, n_experts,
+                                  n_rows, H, I,
                                   (const __nv_bfloat16*)w13, (const __nv_bfloat16*)w2,
                                   (__nv_bfloat16*)h, y, y_dtype == MOE_F32, dev_status, ev_b, s);
 }
@@ -194,9 +198,29 @@ moe_status moe_dispatch_layout(const int32_t* topk_idx, int64_t T, int32_t k, in
                                        rank_offsets, slot_of_pair, pair_of_slot, workspace,
                                        workspace_bytes, dev_status);
     if (st != MOE_OK) return st;
-    return cuda_status(launch_dispatch_layout(topk_idx, T, k, E, W, expert_counts,
+    return cuda_status(launch_dispatch_layout(topk_idx, T, k, E, W, -1, expert_counts,
                                               expert_offsets, rank_offsets, slot_of_pair,
-                                              pair_of_slot, workspace, dev_status,
+                                              pair_of_slot, nullptr, workspace, dev_status,
+                                              (cudaStream_t)stream));
+}
+
+moe_status moe_dispatch_layout_capacity(const int32_t* topk_idx, int64_t T, int32_t k, int32_t E,
+                                        int32_t W, int32_t capacity, int32_t* expert_counts,
+                                        int32_t* expert_offsets, int32_t* rank_offsets,
+                                        int32_t* slot_of_pair, int32_t* pair_of_slot,
+                                        int32_t* n_dropped, void* workspace,
+                                        size_t workspace_bytes, int32_t* dev_status,
+                                        void* stream) {
+    if (capacity < 0) return MOE_ERR_INVALID_ARG;
+    if ((int64_t)E * capacity >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
+    moe_status st = check_layout(topk_idx, T, k, E, W, expert_counts, expert_offsets,
+                                 rank_offsets, slot_of_pair, pair_of_slot, workspace,
+                                 workspace_bytes, dev_status);
+    if (st != MOE_OK) return st;
+    if ((int64_t)E * capacity > 0 && !pair_of_slot) return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_dispatch_layout(topk_idx, T, k, E, W, capacity, expert_counts,
+                                              expert_offsets, rank_offsets, slot_of_pair,
+                                              pair_of_slot, n_dropped, workspace, dev_status,
                                               (cudaStream_t)stream));
 }
 
@@ -219,7 +243,8 @@ size_t moe_grouped_gemm_workspace_bytes(int64_t n_rows, int32_t H, int32_t I, mo
 }
 
 moe_status moe_grouped_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_scales,
-                            const int32_t* expert_offsets, int32_t expert_begin,
+                            const int32_t* expert_offsets, const int32_t* expert_counts,
+                            int32_t expert_begin,
                             int32_t n_experts, int64_t n_rows, int32_t H, int32_t I,
                             const void* w13, const void* w2, moe_dtype w_dtype, void* h, void* y,
                             moe_dtype y_dtype, void* workspace, size_t workspace_bytes,
@@ -230,9 +255,9 @@ moe_status moe_grouped_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_
                    I, w13, w2, w_dtype, h, y, y_dtype, workspace, workspace_bytes, dev_status,
                    &noop);
     if (st != MOE_OK || noop) return st;
-    return cuda_status(run_gemm(xp, xp_dtype, xp_scales, expert_offsets, expert_begin, n_experts,
-                                n_rows, H, I, w13, w2, w_dtype, h, y, y_dtype, workspace,
-                                dev_status, (cudaStream_t)stream));
+    return cuda_status(run_gemm(xp, xp_dtype, xp_scales, expert_offsets, expert_counts,
+                                expert_begin, n_experts, n_rows, H, I, w13, w2, w_dtype, h, y,
+                                y_dtype, workspace, dev_status, (cudaStream_t)stream));
 }
 
 moe_status moe_combine(const void* y, moe_dtype y_dtype, const int32_t* slot_of_pair,
@@ -246,12 +271,18 @@ moe_status moe_combine(const void* y, moe_dtype y_dtype, const int32_t* slot_of_
                                       (cudaStream_t)stream));
 }
 
+// Rows of the permuted buffers: T*k (dropless) or E*capacity (fixed slabs).
+static int64_t layer_slots(int64_t T, int32_t k, int32_t E, int32_t capacity) {
+    return capacity < 0 ? T * k : (int64_t)E * capacity;
+}
+
 static moe_status check_layer(const float* logits, const void* x, moe_dtype x_dtype, int64_t T,
                               int32_t H, int32_t E, int32_t k, int32_t W, int32_t I,
                               const void* w13, const void* w2, moe_dtype w_dtype,
-                              moe_dtype payload_dtype, moe_dtype y_dtype,
+                              moe_dtype payload_dtype, moe_dtype y_dtype, int32_t capacity,
                               const moe_layer_buffers* b, const void* out) {
     if (!b) return MOE_ERR_INVALID_ARG;
+    if (capacity >= 0 && (int64_t)E * capacity >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
     bool noop;
     moe_status st = check_route(logits, T, E, k, b->topk_idx, b->topk_w, &noop);
     if (st == MOE_OK)
@@ -262,9 +293,10 @@ static moe_status check_layer(const float* logits, const void* x, moe_dtype x_dt
         st = check_permute(x, x_dtype, T, H, k, b->slot_of_pair, b->xp, payload_dtype,
                            b->xp_scales, &noop);
     if (st == MOE_OK)
-        st = check_gemm(b->xp, payload_dtype, b->xp_scales, b->expert_offsets, 0, E, T * k, H, I,
-                        w13, w2, w_dtype, b->h, b->y, y_dtype, b->gemm_workspace,
-                        b->gemm_workspace_bytes, b->dev_status, &noop);
+        st = check_gemm(b->xp, payload_dtype, b->xp_scales, b->expert_offsets, 0, E,
+                        layer_slots(T, k, E, capacity), H, I, w13, w2, w_dtype, b->h, b->y,
+                        y_dtype, b->gemm_workspace, b->gemm_workspace_bytes, b->dev_status,
+                        &noop);
     if (st == MOE_OK)
         st = check_combine(b->y, y_dtype, b->slot_of_pair, b->topk_w, T, k, H, out, x_dtype,
                            &noop);
@@ -274,9 +306,10 @@ static moe_status check_layer(const float* logits, const void* x, moe_dtype x_dt
 static cudaError_t launch_layer(const float* logits, const void* x, moe_dtype x_dtype, int64_t T,
                                 int32_t H, int32_t E, int32_t k, int32_t W, int32_t I,
                                 const void* w13, const void* w2, moe_dtype w_dtype,
-                                moe_dtype payload_dtype, moe_dtype y_dtype,
+                                moe_dtype payload_dtype, moe_dtype y_dtype, int32_t capacity,
                                 const moe_layer_buffers* b, void* out, void* const* ev,
                                 cudaStream_t s) {
+    const int64_t n_slots = layer_slots(T, k, E, capacity);
     auto mark = [&](int i) {
         return ev ? cudaEventRecord((cudaEvent_t)ev[i], s) : cudaSuccess;
     };
@@ -284,17 +317,20 @@ static cudaError_t launch_layer(const float* logits, const void* x, moe_dtype x_
     if (e == cudaSuccess && T > 0) e = launch_route_topk(logits, T, E, k, b->topk_idx, b->topk_w, s);
     if (e == cudaSuccess) e = mark(1);
     if (e == cudaSuccess)
-        e = launch_dispatch_layout(b->topk_idx, T, k, E, W, b->expert_counts, b->expert_offsets,
-                                   b->rank_offsets, b->slot_of_pair, b->pair_of_slot,
-                                   b->layout_workspace, b->dev_status, s);
+        e = launch_dispatch_layout(b->topk_idx, T, k, E, W, capacity < 0 ? -1 : capacity,
+                                   b->expert_counts, b->expert_offsets, b->rank_offsets,
+                                   b->slot_of_pair, b->pair_of_slot,
+                                   capacity < 0 ? nullptr : b->n_dropped, b->layout_workspace,
+                                   b->dev_status, s);
     if (e == cudaSuccess) e = mark(2);
     if (e == cudaSuccess && T > 0)
         e = launch_permute(x, x_dtype, T, H, k, b->slot_of_pair, b->xp, payload_dtype,
                            b->xp_scales, s);
     if (e == cudaSuccess) e = mark(3);
-    if (e == cudaSuccess && T > 0) {
-        e = run_gemm(b->xp, payload_dtype, b->xp_scales, b->expert_offsets, 0, E, T * k, H, I,
-                     w13, w2, w_dtype, b->h, b->y, y_dtype, b->gemm_workspace, b->dev_status, s,
+    if (e == cudaSuccess && T > 0 && n_slots > 0) {
+        e = run_gemm(b->xp, payload_dtype, b->xp_scales, b->expert_offsets,
+                     capacity < 0 ? nullptr : b->expert_counts, 0, E, n_slots, H, I, w13, w2,
+                     w_dtype, b->h, b->y, y_dtype, b->gemm_workspace, b->dev_status, s,
                      ev ? (cudaEvent_t)ev[4] : nullptr, ev ? (cudaEvent_t)ev[5] : nullptr);
     } else if (e == cudaSuccess) {
         e = mark(4);
@@ -310,14 +346,14 @@ static cudaError_t launch_layer(const float* logits, const void* x, moe_dtype x_
 moe_status moe_layer_forward(const float* logits, const void* x, moe_dtype x_dtype, int64_t T,
                              int32_t H, int32_t E, int32_t k, int32_t W, int32_t I,
                              const void* w13, const void* w2, moe_dtype w_dtype,
-                             moe_dtype payload_dtype, moe_dtype y_dtype,
+                             moe_dtype payload_dtype, moe_dtype y_dtype, int32_t capacity,
                              const moe_layer_buffers* b, void* out, void* const* step_events,
                              void* stream) {
     const moe_status st = check_layer(logits, x, x_dtype, T, H, E, k, W, I, w13, w2, w_dtype,
-                                      payload_dtype, y_dtype, b, out);
+                                      payload_dtype, y_dtype, capacity, b, out);
     if (st != MOE_OK) return st;
     return cuda_status(launch_layer(logits, x, x_dtype, T, H, E, k, W, I, w13, w2, w_dtype,
-                                    payload_dtype, y_dtype, b, out, step_events,
+                                    payload_dtype, y_dtype, capacity, b, out, step_events,
                                     (cudaStream_t)stream));
 }
 
@@ -326,10 +362,10 @@ moe_status moe_layer_forward_host(const float* logits_host, const void* x_host, 
                                   moe_dtype x_dtype, int64_t T, int32_t H, int32_t E, int32_t k,
                                   int32_t W, int32_t I, const void* w13, const void* w2,
                                   moe_dtype w_dtype, moe_dtype payload_dtype, moe_dtype y_dtype,
-                                  const moe_layer_buffers* b, void* const* step_events,
-                                  void* stream) {
+                                  int32_t capacity, const moe_layer_buffers* b,
+                                  void* const* step_events, void* stream) {
     const moe_status st = check_layer(logits_dev, x_dev, x_dtype, T, H, E, k, W, I, w13, w2,
-                                      w_dtype, payload_dtype, y_dtype, b, out_dev);
+                                      w_dtype, payload_dtype, y_dtype, capacity, b, out_dev);
     if (st != MOE_OK) return st;
     if (T > 0 && (!logits_host || !x_host || !out_host)) return MOE_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
@@ -342,7 +378,7 @@ moe_status moe_layer_forward_host(const float* logits_host, const void* x_host, 
     }
     if (e == cudaSuccess)
         e = launch_layer(logits_dev, x_dev, x_dtype, T, H, E, k, W, I, w13, w2, w_dtype,
-                         payload_dtype, y_dtype, b, out_dev, step_events, s);
+                         payload_dtype, y_dtype, capacity, b, out_dev, step_events, s);
     if (e == cudaSuccess && T > 0)
         e = cudaMemcpyAsync(out_host, out_dev, xb, cudaMemcpyDeviceToHost, s);
     return cuda_status(e);

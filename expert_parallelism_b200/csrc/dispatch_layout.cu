@@ -20,6 +20,14 @@
 //                      counts are scanned across warps), slot = base +
 //                      rank; writes slot_of_pair / pair_of_slot, and CTA 0
 //                      writes the counts, offsets and rank offsets.
+//
+// Fixed-capacity mode (C >= 0; "Expert Parallelism" (aiwiki),
+// "Implementation", closing note: fixed buffers make every size known in
+// advance at the price of the tokens that do not fit): expert e owns the
+// slab [e*C, (e+1)*C).  A pair's rank among its expert's pairs is its
+// dropless slot minus the expert's dropless start; ranks below C keep that
+// place in the slab, later pairs are dropped (slot -1).  The same three
+// launches, the scatter doing the remap.
 #include "common.cuh"
 
 namespace moe {
@@ -160,21 +168,28 @@ __global__ void __launch_bounds__(kScanThreads) layout_scan_kernel(
     }
 }
 
+// C < 0: dropless.  C >= 0: fixed slabs of C rows (pair_of_slot has E*C
+// entries); n_dropped (may be null) receives the number of dropped pairs.
 __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(
     const int32_t* __restrict__ idx, int64_t N, int E, int W, int64_t nt,
-    const int32_t* __restrict__ counts, const int32_t* __restrict__ base, int64_t L,
+    const int32_t* __restrict__ counts, const int32_t* __restrict__ base, int64_t L, int C,
     int32_t* __restrict__ expert_counts, int32_t* __restrict__ expert_offsets,
     int32_t* __restrict__ rank_offsets, int32_t* __restrict__ slot_of_pair,
-    int32_t* __restrict__ pair_of_slot) {
+    int32_t* __restrict__ pair_of_slot, int32_t* __restrict__ n_dropped) {
     extern __shared__ int32_t sm[];
     int32_t* wcount = sm;                      // [warps][E]: counts, then warp prefixes
     int32_t* s_base = sm + kLayoutWarps * E;   // [E]: base of this tile per expert
+    int32_t* s_start = s_base + E;             // [E + 1]: dropless start of each expert
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t b = blockIdx.x;
     const int32_t total = base[L - 1] + counts[L - 1];
+    const bool capped = C >= 0;
 
     for (int i = tid; i < kLayoutWarps * E; i += blockDim.x) wcount[i] = 0;
     for (int e = tid; e < E; e += blockDim.x) s_base[e] = base[(int64_t)e * nt + b];
+    if (capped)
+        for (int e = tid; e <= E; e += blockDim.x)
+            s_start[e] = (e < E) ? base[(int64_t)e * nt] : total;
     __syncthreads();
 
     // pass 1: each warp walks its pairs in order; equal experts inside a
@@ -217,9 +232,43 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(
             slot_of_pair[p] = -1;
             continue;
         }
-        const int32_t s = s_base[e] + wcount[warp * E + e] + rank[g];
+        int32_t s = s_base[e] + wcount[warp * E + e] + rank[g];
+        if (capped) {
+            const int32_t pos = s - s_start[e];      // rank among the expert's pairs
+            s = pos < C ? e * C + pos : -1;
+        }
         slot_of_pair[p] = s;
-        pair_of_slot[s] = (int32_t)p;
+        if (s >= 0) pair_of_slot[s] = (int32_t)p;
+    }
+    if (capped) {
+        // slab rows past each expert's kept pairs
+        const int64_t rows = (int64_t)E * C;
+        for (int64_t s = b * blockDim.x + tid; s < rows; s += nt * blockDim.x) {
+            const int e = (int)(s / C);
+            const int32_t kept = min(s_start[e + 1] - s_start[e], C);
+            if (s - (int64_t)e * C >= kept) pair_of_slot[s] = -1;
+        }
+        if (b == 0) {
+            int32_t drop = 0;
+            for (int e = tid; e < E; e += blockDim.x) {
+                const int32_t cnt = s_start[e + 1] - s_start[e];
+                expert_counts[e] = min(cnt, C);
+                drop += max(cnt - C, 0);
+            }
+            for (int e = tid; e <= E; e += blockDim.x) expert_offsets[e] = e * C;
+            for (int r = tid; r <= W; r += blockDim.x)
+                rank_offsets[r] = (int32_t)((int64_t)r * E / W) * C;
+            drop = __reduce_add_sync(0xffffffffu, drop);
+            __syncthreads();                         // wcount is free again
+            if (lane == 0) wcount[warp] = drop;
+            __syncthreads();
+            if (tid == 0 && n_dropped) {
+                int32_t sum = 0;
+                for (int w = 0; w < kLayoutWarps; ++w) sum += wcount[w];
+                *n_dropped = sum;
+            }
+        }
+        return;
     }
     // slots past the last routed row (only when ids were skipped)
     for (int64_t s = (int64_t)total + b * blockDim.x + tid; s < N; s += nt * blockDim.x)
@@ -240,15 +289,15 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(
     }
 }
 
-cudaError_t launch_dispatch_layout(const int32_t* idx, int64_t T, int k, int E, int W,
+cudaError_t launch_dispatch_layout(const int32_t* idx, int64_t T, int k, int E, int W, int C,
                                    int32_t* expert_counts, int32_t* expert_offsets,
                                    int32_t* rank_offsets, int32_t* slot_of_pair,
-                                   int32_t* pair_of_slot, void* workspace,
+                                   int32_t* pair_of_slot, int32_t* n_dropped, void* workspace,
                                    int32_t* dev_status, cudaStream_t s) {
     const int64_t N = T * k;
     LayoutWorkspace w = carve(workspace, T, k, E);
     const size_t hist_smem = (size_t)E * 4;
-    const size_t scatter_smem = (size_t)(kLayoutWarps + 1) * E * 4;
+    const size_t scatter_smem = ((size_t)(kLayoutWarps + 2) * E + 1) * 4;
     if (scatter_smem > 48 * 1024) {
         cudaError_t err = cudaFuncSetAttribute(
             layout_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scatter_smem);
@@ -260,8 +309,8 @@ cudaError_t launch_dispatch_layout(const int32_t* idx, int64_t T, int k, int E, 
                                                                     w.status, w.ticket,
                                                                     dev_status);
     layout_scatter_kernel<<<(unsigned)w.nt, kLayoutThreads, scatter_smem, s>>>(
-        idx, N, E, W, w.nt, w.counts, w.base, w.L, expert_counts, expert_offsets, rank_offsets,
-        slot_of_pair, pair_of_slot);
+        idx, N, E, W, w.nt, w.counts, w.base, w.L, C, expert_counts, expert_offsets,
+        rank_offsets, slot_of_pair, pair_of_slot, n_dropped);
     note_launches(3);
     return cudaGetLastError();
 }

@@ -18,8 +18,9 @@
 
 namespace moe {
 size_t layout_workspace_bytes(int64_t T, int k, int E);
-cudaError_t launch_dispatch_layout(const int32_t*, int64_t, int, int, int, int32_t*, int32_t*,
-                                   int32_t*, int32_t*, int32_t*, void*, int32_t*, cudaStream_t);
+cudaError_t launch_dispatch_layout(const int32_t*, int64_t, int, int, int, int, int32_t*,
+                                   int32_t*, int32_t*, int32_t*, int32_t*, int32_t*, void*,
+                                   int32_t*, cudaStream_t);
 }  // namespace moe
 
 // 2 MiB: enough for E * ceil(T*k / 2048) <= ~262,000, e.g. 256 experts and
@@ -70,8 +71,8 @@ moe_status moe_dispatch_layout_noalloc(const int32_t* topk_idx, int64_t T, int32
     // the layout clears the look-back flags and the ticket itself, and the
     // rest is fully overwritten before it is read.
     const cudaError_t e = moe::launch_dispatch_layout(
-        topk_idx, T, k, E, W, expert_counts, expert_offsets, rank_offsets, slot_of_pair,
-        pair_of_slot, scratch, dev_status, (cudaStream_t)stream);
+        topk_idx, T, k, E, W, -1, expert_counts, expert_offsets, rank_offsets, slot_of_pair,
+        pair_of_slot, nullptr, scratch, dev_status, (cudaStream_t)stream);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -26,15 +26,15 @@ __device__ __forceinline__ float silu_f32(float g) { return __fdiv_rn(g, 1.0f + 
 template <typename TA, typename TW, bool GLU>
 __global__ void __launch_bounds__(256) simt_grouped_gemm_kernel(
     const TA* __restrict__ A, int K, const TW* __restrict__ B, int Nout,
-    const int32_t* __restrict__ offsets, int expert_begin, int n_experts, int64_t n_rows,
-    TW* __restrict__ C) {
+    const int32_t* __restrict__ offsets, const int32_t* __restrict__ counts, int expert_begin,
+    int n_experts, int64_t n_rows, TW* __restrict__ C) {
     __shared__ int32_t s_prefix[MOE_MAX_EXPERTS + 1];
     __shared__ int32_t s_ws[8];
     __shared__ float As[kSimtBK][kSimtBM + 4];
     __shared__ float Bg[kSimtBK][kSimtBN + 4];
     __shared__ float Bu[GLU ? kSimtBK : 1][kSimtBN + 4];
 
-    build_tile_prefix(offsets, expert_begin, n_experts, kSimtBM, s_prefix, s_ws);
+    build_tile_prefix(offsets, counts, expert_begin, n_experts, kSimtBM, s_prefix, s_ws);
     const int total_tiles = s_prefix[n_experts];
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
     const int n0 = blockIdx.x * kSimtBN;
@@ -43,7 +43,9 @@ __global__ void __launch_bounds__(256) simt_grouped_gemm_kernel(
     for (int mt = blockIdx.y; mt < total_tiles; mt += gridDim.y) {
         const int j = find_tile_expert(s_prefix, n_experts, mt);
         const int64_t row0 = offsets[expert_begin + j] + (int64_t)(mt - s_prefix[j]) * kSimtBM;
-        const int64_t row_end = min((int64_t)offsets[expert_begin + j + 1], n_rows);
+        const int64_t row_end =
+            min((int64_t)offsets[expert_begin + j] + segment_rows(offsets, counts, expert_begin, j),
+                n_rows);
         const TW* Bj = B + (int64_t)j * brows * K;
         float acc_g[4][4], acc_u[4][4];
 #pragma unroll
@@ -157,29 +159,30 @@ cudaError_t launch_dequant_e4m3(const uint8_t* q, const float* scales, const int
 }
 
 template <typename TA, typename TW>
-static cudaError_t simt_two_phase(const TA* xp, const int32_t* offsets, int expert_begin,
-                                  int n_experts, int64_t n_rows, int H, int I, const TW* w13,
-                                  const TW* w2, TW* h, TW* y, cudaEvent_t ev_mid,
+static cudaError_t simt_two_phase(const TA* xp, const int32_t* offsets, const int32_t* counts,
+                                  int expert_begin, int n_experts, int64_t n_rows, int H, int I,
+                                  const TW* w13, const TW* w2, TW* h, TW* y, cudaEvent_t ev_mid,
                                   cudaStream_t s) {
     int64_t gy = (n_rows + kSimtBM - 1) / kSimtBM + n_experts;
     if (gy > 65535) gy = 65535;
     const dim3 g1((I + kSimtBN - 1) / kSimtBN, (unsigned)gy);
-    simt_grouped_gemm_kernel<TA, TW, true><<<g1, 256, 0, s>>>(xp, H, w13, I, offsets,
-                                                              expert_begin, n_experts, n_rows, h);
+    simt_grouped_gemm_kernel<TA, TW, true><<<g1, 256, 0, s>>>(
+        xp, H, w13, I, offsets, counts, expert_begin, n_experts, n_rows, h);
     if (ev_mid) cudaEventRecord(ev_mid, s);
     const dim3 g2((H + kSimtBN - 1) / kSimtBN, (unsigned)gy);
-    simt_grouped_gemm_kernel<TW, TW, false><<<g2, 256, 0, s>>>(h, I, w2, H, offsets,
-                                                               expert_begin, n_experts, n_rows, y);
+    simt_grouped_gemm_kernel<TW, TW, false><<<g2, 256, 0, s>>>(
+        h, I, w2, H, offsets, counts, expert_begin, n_experts, n_rows, y);
     note_launches(2);
     return cudaGetLastError();
 }
 
 cudaError_t launch_grouped_gemm_simt_f32(const float* xp, const int32_t* offsets,
-                                         int expert_begin, int n_experts, int64_t n_rows, int H,
-                                         int I, const float* w13, const float* w2, float* h,
-                                         float* y, cudaEvent_t ev_mid, cudaStream_t s) {
-    return simt_two_phase<float, float>(xp, offsets, expert_begin, n_experts, n_rows, H, I, w13,
-                                        w2, h, y, ev_mid, s);
+                                         const int32_t* counts, int expert_begin, int n_experts,
+                                         int64_t n_rows, int H, int I, const float* w13,
+                                         const float* w2, float* h, float* y, cudaEvent_t ev_mid,
+                                         cudaStream_t s) {
+    return simt_two_phase<float, float>(xp, offsets, counts, expert_begin, n_experts, n_rows, H,
+                                        I, w13, w2, h, y, ev_mid, s);
 }
 
 }  // namespace moe

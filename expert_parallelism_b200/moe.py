@@ -10,6 +10,7 @@ loading fails loudly when ``libmoe.so`` has not been built.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 
 import torch
@@ -30,17 +31,19 @@ SIGNATURES = {
     "moe_route_topk": ([_P, _I64, _I32, _I32, _P, _P, _P], _I),
     "moe_dispatch_layout_workspace_bytes": ([_I64, _I32, _I32], _SZ),
     "moe_dispatch_layout": ([_P, _I64, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _SZ, _P, _P], _I),
+    "moe_dispatch_layout_capacity": ([_P, _I64, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P,
+                                      _P, _SZ, _P, _P], _I),
     "moe_dispatch_layout_noalloc_max_scratch_bytes": ([], _SZ),
     "moe_dispatch_layout_noalloc": ([_P, _I64, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _P], _I),
     "moe_permute": ([_P, _I, _I64, _I32, _I32, _P, _P, _I, _P, _P], _I),
     "moe_grouped_gemm_workspace_bytes": ([_I64, _I32, _I32, _I, _I], _SZ),
-    "moe_grouped_gemm": ([_P, _I, _P, _P, _I32, _I32, _I64, _I32, _I32, _P, _P, _I, _P, _P, _I,
-                          _P, _SZ, _P, _P], _I),
+    "moe_grouped_gemm": ([_P, _I, _P, _P, _P, _I32, _I32, _I64, _I32, _I32, _P, _P, _I, _P, _P,
+                          _I, _P, _SZ, _P, _P], _I),
     "moe_combine": ([_P, _I, _P, _P, _I64, _I32, _I32, _P, _I, _P], _I),
     "moe_layer_forward": ([_P, _P, _I, _I64, _I32, _I32, _I32, _I32, _I32, _P, _P, _I, _I, _I,
-                           _P, _P, _P, _P], _I),
+                           _I32, _P, _P, _P, _P], _I),
     "moe_layer_forward_host": ([_P, _P, _P, _P, _P, _P, _I, _I64, _I32, _I32, _I32, _I32, _I32,
-                                _P, _P, _I, _I, _I, _P, _P, _P], _I),
+                                _P, _P, _I, _I, _I, _I32, _P, _P, _P], _I),
     "moe_check_status": ([_P, _P], _I),
     "moe_status_str": ([_I], ctypes.c_char_p),
     "moe_launch_count": ([], ctypes.c_uint64),
@@ -54,7 +57,7 @@ class LayerBuffersC(ctypes.Structure):
                 ("pair_of_slot", _P), ("layout_workspace", _P),
                 ("layout_workspace_bytes", _SZ), ("xp", _P), ("xp_scales", _P), ("h", _P),
                 ("y", _P), ("gemm_workspace", _P), ("gemm_workspace_bytes", _SZ),
-                ("dev_status", _P)]
+                ("dev_status", _P), ("n_dropped", _P)]
 
 
 class MoEError(RuntimeError):
@@ -123,6 +126,17 @@ def moe_dispatch_layout(topk_idx, E, W, expert_counts, expert_offsets, rank_offs
         workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
 
 
+def moe_dispatch_layout_capacity(topk_idx, E, W, capacity, expert_counts, expert_offsets,
+                                 rank_offsets, slot_of_pair, pair_of_slot, workspace, dev_status,
+                                 n_dropped=None, stream=None):
+    T, k = topk_idx.shape
+    _check("moe_dispatch_layout_capacity", load_library().moe_dispatch_layout_capacity(
+        _ptr(topk_idx), T, k, E, W, capacity, _ptr(expert_counts), _ptr(expert_offsets),
+        _ptr(rank_offsets), _ptr(slot_of_pair), _ptr(pair_of_slot), _ptr(n_dropped),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_status),
+        _stream(stream)))
+
+
 def moe_dispatch_layout_noalloc(topk_idx, E, W, expert_counts, expert_offsets, rank_offsets,
                                 slot_of_pair, pair_of_slot, dev_status, stream=None):
     """moe_dispatch_layout without a workspace (scratch inside the library)."""
@@ -146,12 +160,13 @@ def moe_grouped_gemm_workspace_bytes(n_rows, H, I, xp_dtype, w_dtype) -> int:
 
 
 def moe_grouped_gemm(xp, xp_scales, expert_offsets, expert_begin, n_experts, w13, w2, h, y,
-                     workspace, dev_status, stream=None):
+                     workspace, dev_status, stream=None, expert_counts=None):
     n_rows, H = xp.shape
     I = w2.shape[2]
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("moe_grouped_gemm", load_library().moe_grouped_gemm(
-        _ptr(xp), dtype_code(xp), _ptr(xp_scales), _ptr(expert_offsets), expert_begin,
+        _ptr(xp), dtype_code(xp), _ptr(xp_scales), _ptr(expert_offsets), _ptr(expert_counts),
+        expert_begin,
         n_experts, n_rows, H, I, _ptr(w13), _ptr(w2), dtype_code(w13), _ptr(h), _ptr(y),
         dtype_code(y), _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream)))
 
@@ -174,6 +189,20 @@ def moe_status_str(code: int) -> str:
 
 
 # ----------------------------------------------------------------- buffers
+def capacity_rows(wl) -> int:
+    """Rows per expert slab for a fixed-capacity workload, ceil(factor * T*k
+    / E); -1 for a dropless one."""
+    if wl.capacity_factor is None:
+        return -1
+    return int(math.ceil(wl.capacity_factor * wl.T * wl.k / wl.E))
+
+
+def slot_rows(wl) -> int:
+    """Rows of the permuted buffers: T*k, or E * capacity."""
+    c = capacity_rows(wl)
+    return wl.T * wl.k if c < 0 else wl.E * c
+
+
 class LayerBuffers:
     """Device buffers for one layer of a workload (outputs and workspaces).
 
@@ -182,7 +211,9 @@ class LayerBuffers:
 
     def __init__(self, wl, device="cuda"):
         from .workloads import TORCH_DTYPE
-        T, H, E, k, I, W, N = wl.T, wl.H, wl.E, wl.k, wl.I, wl.W, wl.N
+        T, H, E, k, I, W = wl.T, wl.H, wl.E, wl.k, wl.I, wl.W
+        self.capacity = capacity_rows(wl)
+        N = slot_rows(wl)                      # rows of the permuted buffers
         dev = torch.device(device)
         i32 = dict(dtype=torch.int32, device=dev)
         self.wl = wl
@@ -191,8 +222,9 @@ class LayerBuffers:
         self.expert_counts = torch.empty(E, **i32)
         self.expert_offsets = torch.empty(E + 1, **i32)
         self.rank_offsets = torch.empty(W + 1, **i32)
-        self.slot_of_pair = torch.empty(max(N, 1), **i32)
+        self.slot_of_pair = torch.empty(max(T * k, 1), **i32)
         self.pair_of_slot = torch.empty(max(N, 1), **i32)
+        self.n_dropped = torch.zeros(1, **i32)
         self.layout_ws = torch.empty(max(moe_dispatch_layout_workspace_bytes(T, k, E), 16),
                                      dtype=torch.uint8, device=dev)
         self.dev_status = torch.zeros(1, **i32)
@@ -217,7 +249,8 @@ def layer_buffers_c(buf: "LayerBuffers") -> LayerBuffersC:
         _ptr(buf.topk_idx), _ptr(buf.topk_w), _ptr(buf.expert_counts), _ptr(buf.expert_offsets),
         _ptr(buf.rank_offsets), _ptr(buf.slot_of_pair), _ptr(buf.pair_of_slot),
         _ptr(buf.layout_ws), _nbytes(buf.layout_ws), _ptr(buf.xp), _ptr(buf.xp_scales),
-        _ptr(buf.h), _ptr(buf.y), _ptr(buf.gemm_ws), _nbytes(buf.gemm_ws), _ptr(buf.dev_status))
+        _ptr(buf.h), _ptr(buf.y), _ptr(buf.gemm_ws), _nbytes(buf.gemm_ws), _ptr(buf.dev_status),
+        _ptr(buf.n_dropped))
 
 
 def _events(step_events, stream=None):
@@ -241,8 +274,8 @@ def moe_layer_forward(wl, logits, x, w13, w2, buf: "LayerBuffers", step_events=N
     ev = _events(step_events, stream)
     _check("moe_layer_forward", load_library().moe_layer_forward(
         _ptr(logits), _ptr(x), dtype_code(x), wl.T, wl.H, wl.E, wl.k, wl.W, wl.I, _ptr(w13),
-        _ptr(w2), dtype_code(w13), dtype_code(buf.xp), dtype_code(buf.y), ctypes.byref(cb),
-        _ptr(buf.out), ev[0] if ev else None, _stream(stream)))
+        _ptr(w2), dtype_code(w13), dtype_code(buf.xp), dtype_code(buf.y), buf.capacity,
+        ctypes.byref(cb), _ptr(buf.out), ev[0] if ev else None, _stream(stream)))
     return buf.out
 
 
@@ -254,7 +287,7 @@ def moe_layer_forward_host(wl, logits_host, x_host, out_host, logits_dev, x_dev,
     _check("moe_layer_forward_host", load_library().moe_layer_forward_host(
         _ptr(logits_host), _ptr(x_host), _ptr(out_host), _ptr(logits_dev), _ptr(x_dev),
         _ptr(buf.out), dtype_code(x_dev), wl.T, wl.H, wl.E, wl.k, wl.W, wl.I, _ptr(w13), _ptr(w2),
-        dtype_code(w13), dtype_code(buf.xp), dtype_code(buf.y), ctypes.byref(cb),
+        dtype_code(w13), dtype_code(buf.xp), dtype_code(buf.y), buf.capacity, ctypes.byref(cb),
         ev[0] if ev else None, _stream(stream)))
 
 

@@ -22,10 +22,12 @@ def dispatch_bytes_from_layout(rank_offsets_last: int, H: int, bytes_per_elem: i
     return rank_offsets_last * H * bytes_per_elem
 
 
-def kernel_bytes(wl: Workload) -> dict:
+def kernel_bytes(wl: Workload, rows: int | None = None) -> dict:
     """Algorithmic HBM bytes per launch of each step (each input read once,
-    each output written once)."""
-    N, T, H, E, k, I = wl.N, wl.T, wl.H, wl.E, wl.k, wl.I
+    each output written once) for ``rows`` routed rows kept (all T*k by
+    default; fewer when a fixed capacity drops pairs)."""
+    T, H, E, k, I = wl.T, wl.H, wl.E, wl.k, wl.I
+    N = wl.N if rows is None else rows
     xb, pb, yb = ELEM_BYTES[wl.act], ELEM_BYTES[wl.payload], ELEM_BYTES[wl.ydt]
     scales = N * (H // 128) * 4 if wl.payload == "e4m3" else 0
     return {

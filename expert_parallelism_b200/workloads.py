@@ -59,6 +59,7 @@ class Workload:
     zipf_s: float = 1.2
     seed: int = 0
     ydt: str = "f32"         # storage of the experts' outputs y (combine's input)
+    capacity_factor: float | None = None   # None: dropless; else fixed slabs per expert
 
     @property
     def N(self) -> int:
@@ -80,6 +81,11 @@ WORKLOADS = {
     "skew": Workload("skew", 16384, 2880, 128, 4, 2880, 8, "bf16", "bf16", "bf16",
                      router="zipf"),
     "decode": Workload("decode", 64, 7168, 256, 8, 2048, 8, "bf16", "bf16", "bf16"),
+    # fixed-capacity variants: slabs of ceil(factor * T*k / E) rows per expert
+    "dsv3_cap": Workload("dsv3_cap", 8192, 7168, 256, 8, 2048, 8, "bf16", "e4m3", "bf16",
+                         capacity_factor=1.0),
+    "skew_cap": Workload("skew_cap", 16384, 2880, 128, 4, 2880, 8, "bf16", "bf16", "bf16",
+                         router="zipf", capacity_factor=1.25),
 }
 
 TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16,

@@ -135,6 +135,41 @@ moe_status moe_dispatch_layout(const int32_t* topk_idx, int64_t T, int32_t k, in
                                size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /*
+ * moe_dispatch_layout_capacity -- the dispatch layout with a fixed capacity
+ * of C rows per expert; the pairs that do not fit are dropped.
+ *
+ * Source: "Expert Parallelism" (aiwiki), "Implementation", closing note:
+ * with fixed buffers every destination's size is known in advance (no
+ * count exchange before the payload), and the tokens that do not fit are
+ * the price.  The page gives neither the size nor the drop rule; this
+ * library reads it as: expert e owns the fixed slab [e*C, (e+1)*C) of the
+ * permuted buffer; its pairs, in pair order (the stable order of
+ * moe_dispatch_layout), fill the slab from the top, and the pairs past the
+ * C-th are dropped.  A dropped pair contributes nothing to the combine.
+ *
+ *   capacity       C >= 0 rows per expert (e.g. ceil(factor * T*k / E)).
+ *   expert_counts  [E] int32, written: rows kept per expert, min(count, C).
+ *   expert_offsets [E+1] int32, written: e*C (fixed).
+ *   rank_offsets   [W+1] int32, written: (r*E/W)*C (fixed).
+ *   slot_of_pair   [T*k] int32, written: e*C + the pair's rank among
+ *                  expert e's pairs; -1 for a dropped pair or a bad id.
+ *   pair_of_slot   [E*C] int32, written: inverse map; slab rows past an
+ *                  expert's kept pairs hold -1.
+ *   n_dropped      int32 device word or NULL: written with the number of
+ *                  dropped pairs (bad ids not included).
+ *   workspace, workspace_bytes, dev_status, stream: as moe_dispatch_layout.
+ * Requirements as moe_dispatch_layout, plus E*C < 2^31.  C < 0 returns
+ * MOE_ERR_INVALID_ARG.  The segments handed to moe_grouped_gemm are then
+ * expert_offsets with expert_counts (the rows each expert computes).
+ */
+moe_status moe_dispatch_layout_capacity(const int32_t* topk_idx, int64_t T, int32_t k, int32_t E,
+                                        int32_t W, int32_t capacity, int32_t* expert_counts,
+                                        int32_t* expert_offsets, int32_t* rank_offsets,
+                                        int32_t* slot_of_pair, int32_t* pair_of_slot,
+                                        int32_t* n_dropped, void* workspace,
+                                        size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
  * moe_dispatch_layout_noalloc -- moe_dispatch_layout for callers that cannot
  * allocate device memory.  The pages have no counterpart: this is a
  * convenience of this library, not a step of the method.
@@ -197,7 +232,10 @@ moe_status moe_permute(const void* x, moe_dtype x_dtype, int64_t T, int32_t H, i
  * weights stacked along the expert dimension, "GroupedGemmParallel").
  *
  * For local expert j (global expert e = expert_begin + j) and every slot s
- * in [expert_offsets[e], expert_offsets[e+1]):
+ * in [expert_offsets[e], expert_offsets[e] + rows_e), rows_e =
+ * expert_offsets[e+1] - expert_offsets[e] (or min(that, expert_counts[e])
+ * when expert_counts is given: the fixed slabs of
+ * moe_dispatch_layout_capacity, whose tail rows hold no pair):
  *     g = A_s W13[j, 0:I, :]^T,  u = A_s W13[j, I:2I, :]^T,
  *     h_s = silu(g) * u  (silu(g) = g / (1 + exp(-g))),
  *     y_s = h_s W2[j]^T,
@@ -208,6 +246,8 @@ moe_status moe_permute(const void* x, moe_dtype x_dtype, int64_t T, int32_t H, i
  *   xp_scales      [n_rows, H/128] fp32 when xp_dtype == MOE_E4M3, else NULL.
  *   expert_offsets [>= expert_begin + n_experts + 1] int32, DEVICE memory:
  *                  read by the kernels, never by the host.
+ *   expert_counts  NULL, or [>= expert_begin + n_experts] int32 in DEVICE
+ *                  memory: rows computed per expert (see above).
  *   w13            [n_experts, 2I, H] in w_dtype (gate rows, then up rows).
  *   w2             [n_experts, H, I] in w_dtype.
  *   h              [n_rows, I] in w_dtype, written for the experts' rows (the
@@ -231,7 +271,8 @@ moe_status moe_permute(const void* x, moe_dtype x_dtype, int64_t T, int32_t H, i
 size_t moe_grouped_gemm_workspace_bytes(int64_t n_rows, int32_t H, int32_t I,
                                         moe_dtype xp_dtype, moe_dtype w_dtype);
 moe_status moe_grouped_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_scales,
-                            const int32_t* expert_offsets, int32_t expert_begin,
+                            const int32_t* expert_offsets, const int32_t* expert_counts,
+                            int32_t expert_begin,
                             int32_t n_experts, int64_t n_rows, int32_t H, int32_t I,
                             const void* w13, const void* w2, moe_dtype w_dtype, void* h,
                             void* y, moe_dtype y_dtype, void* workspace,
@@ -271,6 +312,10 @@ moe_status moe_combine(const void* y, moe_dtype y_dtype, const int32_t* slot_of_
  *   b holds every intermediate buffer and workspace (device, caller
  *   owned); b->xp is in payload_dtype (x_dtype or MOE_E4M3), b->y in
  *   y_dtype.
+ *   capacity: -1 for the dropless layout (moe_dispatch_layout; the
+ *   permuted buffers have T*k rows), or C >= 0 for fixed slabs of C rows
+ *   per expert (moe_dispatch_layout_capacity; E*C rows, dropped pairs add
+ *   nothing, b->n_dropped receives their number when not NULL).
  *   step_events: NULL, or 8 cudaEvent_t handles recorded on `stream` at:
  *   0 before routing, 1 after routing, 2 after the layout, 3 after the
  *   permute, 4 after the FP8 dequantisation inside the GEMM (the same point
@@ -285,22 +330,23 @@ typedef struct moe_layer_buffers {
     int32_t* expert_offsets; /* [E + 1] */
     int32_t* rank_offsets;   /* [W + 1] */
     int32_t* slot_of_pair;   /* [T*k] */
-    int32_t* pair_of_slot;   /* [T*k] */
+    int32_t* pair_of_slot;   /* [S] slots: S = T*k, or E*capacity */
     void* layout_workspace;  /* moe_dispatch_layout_workspace_bytes(T, k, E) */
     size_t layout_workspace_bytes;
-    void* xp;                /* [T*k, H] payload */
-    float* xp_scales;        /* [T*k, H/128] (FP8 payload only) */
-    void* h;                 /* [T*k, I] in w_dtype */
-    void* y;                 /* [T*k, H] in y_dtype */
-    void* gemm_workspace;    /* moe_grouped_gemm_workspace_bytes(...) */
+    void* xp;                /* [S, H] payload */
+    float* xp_scales;        /* [S, H/128] (FP8 payload only) */
+    void* h;                 /* [S, I] in w_dtype */
+    void* y;                 /* [S, H] in y_dtype */
+    void* gemm_workspace;    /* moe_grouped_gemm_workspace_bytes(S, ...) */
     size_t gemm_workspace_bytes;
     int32_t* dev_status;     /* int32, zero-initialised */
+    int32_t* n_dropped;      /* int32 or NULL: dropped pairs (capacity >= 0) */
 } moe_layer_buffers;
 
 moe_status moe_layer_forward(const float* logits, const void* x, moe_dtype x_dtype, int64_t T,
                              int32_t H, int32_t E, int32_t k, int32_t W, int32_t I,
                              const void* w13, const void* w2, moe_dtype w_dtype,
-                             moe_dtype payload_dtype, moe_dtype y_dtype,
+                             moe_dtype payload_dtype, moe_dtype y_dtype, int32_t capacity,
                              const moe_layer_buffers* b, void* out, void* const* step_events,
                              void* stream);
 
@@ -317,8 +363,8 @@ moe_status moe_layer_forward_host(const float* logits_host, const void* x_host, 
                                   moe_dtype x_dtype, int64_t T, int32_t H, int32_t E, int32_t k,
                                   int32_t W, int32_t I, const void* w13, const void* w2,
                                   moe_dtype w_dtype, moe_dtype payload_dtype, moe_dtype y_dtype,
-                                  const moe_layer_buffers* b, void* const* step_events,
-                                  void* stream);
+                                  int32_t capacity, const moe_layer_buffers* b,
+                                  void* const* step_events, void* stream);
 
 /*
  * moe_check_status -- synchronise `stream`, read the device status word,

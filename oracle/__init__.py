@@ -231,9 +231,16 @@ def layer(wl, inputs, row_mask=None):
     intermediate (dict).  h, y and out are unrounded (fp64): out is the
     weighted sum of the exact y.  ``row_mask`` (per slot) samples the GEMM
     rows; combine is then only meaningful for tokens whose pairs were all
-    computed."""
+    computed.  A workload with a capacity_factor uses the fixed-capacity
+    layout (dropped pairs add nothing to out)."""
     idx, w = route_topk(inputs["logits"], wl.k)
-    lay = dispatch_layout(idx, wl.E, wl.W)
+    if getattr(wl, "capacity_factor", None) is None:
+        lay = dispatch_layout(idx, wl.E, wl.W)
+    else:   # fixed slabs: only the slab rows holding a pair are computed
+        C = capacity_rows(wl.T, wl.k, wl.E, wl.capacity_factor)
+        lay = dispatch_layout_capacity(idx, wl.E, wl.W, C)
+        kept = lay["pair_of_slot"] >= 0
+        row_mask = kept if row_mask is None else (row_mask & kept)
     xp, sc = permute(inputs["x"], wl.k, lay["pair_of_slot"], wl.payload)
     h, y, _ = grouped_gemm(xp, sc, lay["expert_offsets"], 0, wl.E, inputs["w13"], inputs["w2"],
                            row_mask)

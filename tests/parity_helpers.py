@@ -100,18 +100,21 @@ class GpuLayer:
 
 
 def sample_rows(lay: dict, T: int, k: int, n_tokens: int, seed: int = 0):
-    """Slots of a seeded token sample (all k pairs of each), plus the first
-    and last slot of every non-empty expert (the ragged M tails)."""
+    """Slots of a seeded token sample (all kept pairs of each), plus the
+    first and last computed slot of every non-empty expert (the ragged
+    tails).  Works for the dropless and the fixed-capacity layouts."""
     rng = np.random.default_rng(seed)
     toks = np.sort(rng.choice(T, size=min(n_tokens, T), replace=False))
     sop = lay["slot_of_pair"].numpy().reshape(T, k)
-    mask = np.zeros(T * k, dtype=bool)
-    mask[sop[toks].reshape(-1)] = True
+    mask = np.zeros(lay["pair_of_slot"].numel(), dtype=bool)
+    picked = sop[toks].reshape(-1)
+    mask[picked[picked >= 0]] = True
     off = lay["expert_offsets"].numpy()
+    cnt = lay["expert_counts"].numpy()
     for e in range(len(off) - 1):
-        if off[e + 1] > off[e]:
+        if cnt[e] > 0:
             mask[off[e]] = True
-            mask[off[e + 1] - 1] = True
+            mask[off[e] + cnt[e] - 1] = True
     return torch.from_numpy(toks), torch.from_numpy(mask)
 
 

@@ -85,6 +85,17 @@ def test_layout_rejects_before_launch(lib):
     assert f(*args(E=2048, W=2)) == 2
 
 
+def test_capacity_layout_rejects_before_launch(lib):
+    f = lib.moe_dispatch_layout_capacity
+    ws = lib.moe_dispatch_layout_workspace_bytes(10, 2, 8)
+    args = lambda **kw: [FAKE, 10, 2, kw.get("E", 8), kw.get("W", 2), kw.get("C", 4), FAKE, FAKE,
+                         FAKE, FAKE, kw.get("pos", FAKE), None, FAKE, ws, FAKE, None]
+    assert f(*args(C=-1)) == 1                # negative capacity
+    assert f(*args(W=3)) == 1                 # same checks as the dropless layout
+    assert f(*args(pos=None)) == 1            # slab map missing
+    assert f(*args(E=1024, W=1, C=1 << 21)) == 2   # E * C rows do not fit int32
+
+
 def test_permute_combine_gemm_reject_before_launch(lib):
     p = lib.moe_permute
     assert p(FAKE, moe.MOE_BF16, 10, 100, 2, FAKE, FAKE, moe.MOE_BF16, None, None) == 1   # H % 8
@@ -99,21 +110,21 @@ def test_permute_combine_gemm_reject_before_launch(lib):
     assert c(FAKE, moe.MOE_BF16, FAKE, FAKE, 10, 0, 128, FAKE, moe.MOE_BF16, None) == 1
     assert c(FAKE, moe.MOE_BF16, FAKE, FAKE, 10, 17, 128, FAKE, moe.MOE_BF16, None) == 2
     g = lib.moe_grouped_gemm
-    base = [FAKE, moe.MOE_BF16, None, FAKE, 0, 8, 100, 256, 64, FAKE, FAKE, moe.MOE_BF16, FAKE,
-            FAKE, moe.MOE_F32, None, 0, FAKE, None]
-    bad = list(base); bad[8] = 60                      # I % 8
+    base = [FAKE, moe.MOE_BF16, None, FAKE, None, 0, 8, 100, 256, 64, FAKE, FAKE, moe.MOE_BF16,
+            FAKE, FAKE, moe.MOE_F32, None, 0, FAKE, None]
+    bad = list(base); bad[9] = 60                      # I % 8
     assert g(*bad) == 1
     bad = list(base); bad[1] = moe.MOE_F32             # f32 payload with bf16 weights
     assert g(*bad) == 1
     bad = list(base); bad[1] = moe.MOE_E4M3            # FP8 payload needs scales
     assert g(*bad) == 1
-    bad = list(base); bad[17] = None                   # status word
+    bad = list(base); bad[18] = None                   # status word
     assert g(*bad) == 1
-    bad = list(base); bad[14] = moe.MOE_E4M3           # y storage must be fp32 or bf16
+    bad = list(base); bad[15] = moe.MOE_E4M3           # y storage must be fp32 or bf16
     assert g(*bad) == 1
-    bad = list(base); bad[1] = moe.MOE_F32; bad[11] = moe.MOE_F32; bad[14] = moe.MOE_BF16
+    bad = list(base); bad[1] = moe.MOE_F32; bad[12] = moe.MOE_F32; bad[15] = moe.MOE_BF16
     assert g(*bad) == 1                                # fp32 GEMM stores y in fp32
-    bad = list(base); bad[5] = 0                       # no experts
+    bad = list(base); bad[6] = 0                       # no experts
     assert g(*bad) == 1
 
 
@@ -131,8 +142,11 @@ def test_layer_call_rejects_before_launch(lib):
     f = lib.moe_layer_forward
     # no buffer struct
     assert f(FAKE, FAKE, moe.MOE_BF16, 10, 128, 8, 2, 2, 64, FAKE, FAKE, moe.MOE_BF16,
-             moe.MOE_BF16, moe.MOE_F32, None, FAKE, None, None) == 1
-    cb = moe.LayerBuffersC(*([FAKE] * 8 + [0] + [FAKE] * 5 + [0] + [FAKE]))
+             moe.MOE_BF16, moe.MOE_F32, -1, None, FAKE, None, None) == 1
+    cb = moe.LayerBuffersC(*([FAKE] * 8 + [0] + [FAKE] * 5 + [0] + [FAKE, None]))
     # E % W != 0 is caught before anything runs (workspace size 0 too)
     assert f(FAKE, FAKE, moe.MOE_BF16, 10, 128, 8, 2, 3, 64, FAKE, FAKE, moe.MOE_BF16,
-             moe.MOE_BF16, moe.MOE_F32, ctypes.byref(cb), FAKE, None, None) == 1
+             moe.MOE_BF16, moe.MOE_F32, -1, ctypes.byref(cb), FAKE, None, None) == 1
+    # a capacity whose E * C rows do not fit int32
+    assert f(FAKE, FAKE, moe.MOE_BF16, 10, 128, 8, 2, 2, 64, FAKE, FAKE, moe.MOE_BF16,
+             moe.MOE_BF16, moe.MOE_F32, 1 << 28, ctypes.byref(cb), FAKE, None, None) == 2

@@ -2,13 +2,14 @@
 kernels' maximum sizes, multi-chunk scans, one logical rank's slab run on
 its own, invalid calls that must not touch outputs, and CUDA-graph capture
 of the whole layer."""
+import numpy as np
 import pytest
 import torch
 
 import oracle
 from expert_parallelism_b200 import moe, workloads
 
-from parity_helpers import BF16_TOL, GpuLayer, bits, rowwise_ok
+from parity_helpers import BF16_TOL, GpuLayer, bits, h_ok, rowwise_ok
 
 SENT = -7
 
@@ -223,3 +224,33 @@ def test_layer_call_equals_the_five_calls(name, cuda_device):
     torch.cuda.synchronize()
     assert torch.equal(bits(h_out), bits(five))
     assert moe.moe_check_status(b.dev_status) == 0
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("ydt", ["f32", "bf16"])
+def test_gemm_rows_on_chunk_boundaries(ydt, cuda_device):
+    """Expert row counts on and around every padding boundary of the grouped
+    GEMM (multiples of 16 and of 256, empty experts), H and I not multiples
+    of the weight tile: every row of h and y against the oracle."""
+    counts = [0, 1, 15, 16, 17, 31, 32, 33, 0, 255, 256, 257, 511, 512, 513]
+    E, H, I = len(counts), 320, 200
+    wl = workloads.Workload("chunks", 1, H, E, 1, I, 1, "bf16", "bf16", "bf16", ydt=ydt)
+    off = torch.tensor([0] + list(np.cumsum(counts)), dtype=torch.int32)
+    n = int(off[-1])
+    g = torch.Generator().manual_seed(7)
+    xp = torch.randn(n, H, generator=g).to(torch.bfloat16)
+    w13 = torch.stack([workloads.expert_w13(wl, e) for e in range(E)])
+    w2 = torch.stack([workloads.expert_w2(wl, e) for e in range(E)])
+    h_ref, y_ref, done = oracle.grouped_gemm(xp, None, off, 0, E, w13, w2)
+    assert done == n
+    dev = cuda_device
+    h = torch.full((n, I), float("nan"), dtype=torch.bfloat16, device=dev)
+    y = torch.full((n, H), float("nan"), dtype=workloads.TORCH_DTYPE[ydt], device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    moe.moe_grouped_gemm(xp.to(dev), None, off.to(dev), 0, E, w13.to(dev), w2.to(dev), h, y,
+                         None, st)
+    assert moe.moe_check_status(st) == 0
+    ok, worst = h_ok(h.cpu(), h_ref, torch.bfloat16)
+    assert ok, worst
+    ok, worst = rowwise_ok(y.cpu(), y_ref, BF16_TOL)
+    assert ok, worst

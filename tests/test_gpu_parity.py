@@ -21,7 +21,8 @@ from parity_helpers import (BF16_TOL, F32_TOL, GpuLayer, bits, h_ok, oracle_gemm
 
 SMALL = ["tiny", "small_f32", "small_bf16", "small_fp8", "small_fp8v", "ragged_bf16", "pair_bf16",
          "pair_fp8"]
-FULL = {"decode": 64, "mid": 192, "skew": 128, "dsv3": 96}   # name -> sampled tokens
+FULL = {"decode": 64, "mid": 192, "skew": 128, "dsv3": 96,    # name -> sampled tokens
+        "dsv3_cap": 96, "skew_cap": 128}
 
 
 def _check_route_layout(wl, g: GpuLayer):
@@ -30,7 +31,12 @@ def _check_route_layout(wl, g: GpuLayer):
     assert torch.equal(b.topk_idx.cpu(), idx_o), "topk_idx differs"
     wg = b.topk_w.cpu().double()
     assert bool(((wg - w_o.double()).abs() <= 1e-5 * w_o.double().abs()).all()), "topk_w"
-    lay = oracle.dispatch_layout(idx_o, wl.E, wl.W)
+    if wl.capacity_factor is None:
+        lay = oracle.dispatch_layout(idx_o, wl.E, wl.W)
+    else:
+        C = oracle.capacity_rows(wl.T, wl.k, wl.E, wl.capacity_factor)
+        lay = oracle.dispatch_layout_capacity(idx_o, wl.E, wl.W, C)
+        assert int(b.n_dropped.cpu()[0]) == lay["dropped"]
     for key in ["expert_counts", "expert_offsets", "rank_offsets", "slot_of_pair",
                 "pair_of_slot"]:
         got = getattr(b, key).cpu()[:lay[key].numel()]
@@ -86,14 +92,17 @@ def test_full_size_layer_sampled_parity(name, cuda_device):
     ok, worst = rowwise_ok(b.y.cpu()[slots], y_o, BF16_TOL)
     assert ok, f"y: worst err/rms {worst:.3g}"
     # combine for the sampled tokens, from the oracle's own (exact) y rows
+    # (a dropped pair, slot -1, stays -1 and adds nothing)
     sop = lay["slot_of_pair"].view(wl.T, wl.k)[toks].reshape(-1)
-    compact = torch.searchsorted(slots, sop.long()).to(torch.int32)
-    assert torch.equal(slots[compact.long()], sop.long())
+    kept = sop >= 0
+    compact = torch.full_like(sop, -1)
+    compact[kept] = torch.searchsorted(slots, sop[kept].long()).to(torch.int32)
+    assert torch.equal(slots[compact[kept].long()], sop[kept].long())
     out_o = oracle.combine(y_o, compact, w_o[toks].contiguous())
     ok, worst = rowwise_ok(b.out.cpu()[toks], out_o, BF16_TOL)
     assert ok, f"out: worst err/rms {worst:.3g}"
     # full size, identity experts: combine(xp) returns x exactly (bf16 payloads)
-    if wl.payload == "bf16":
+    if wl.payload == "bf16" and wl.capacity_factor is None:
         moe.moe_combine(b.xp, b.slot_of_pair, b.topk_w, b.out)
         torch.cuda.synchronize()
         assert torch.equal(bits(b.out), bits(g.inputs["x"])), "identity combine != x"

@@ -116,3 +116,31 @@ def test_capacity_rows_formula():
     assert oracle.capacity_rows(8192, 8, 256, 1.0) == 256
     assert oracle.capacity_rows(8192, 8, 256, 1.25) == 320
     assert oracle.capacity_rows(10, 3, 7, 1.0) == 5          # ceil(30 / 7)
+
+
+def test_capacity_layer_is_the_dropless_layer_minus_the_dropped_pairs():
+    """The whole oracle layer with fixed slabs: every kept pair's expert
+    output equals the dropless layer's for that pair, and each token's
+    output is the weighted sum over its kept pairs only (same fp64 values,
+    same j order: bit-exact)."""
+    from expert_parallelism_b200 import workloads
+    wl = workloads.Workload("cap", 96, 64, 8, 3, 48, 2, "bf16", "bf16", "bf16", seed=4)
+    inputs = workloads.layer_inputs(wl)
+    free = oracle.layer(wl, inputs)
+    for factor in (0.5, 1.0, 5.0):
+        cap = oracle.layer(wl.replace(capacity_factor=factor), inputs)
+        sop_c, sop_f = cap["slot_of_pair"].long(), free["slot_of_pair"].long()
+        kept = sop_c >= 0
+        assert torch.equal(cap["y"][sop_c[kept]], free["y"][sop_f[kept]])
+        w = cap["topk_w"].double()
+        want = torch.zeros(wl.T, wl.H, dtype=torch.float64)
+        for t in range(wl.T):
+            for j in range(wl.k):
+                p = t * wl.k + j
+                if kept[p]:
+                    want[t] += w[t, j] * free["y"][sop_f[p]]
+        assert torch.equal(cap["out"], want)
+        if factor == 5.0:
+            assert bool(kept.all()) and torch.equal(cap["out"], free["out"])
+        else:
+            assert not bool(kept.all())
