@@ -62,6 +62,7 @@ constexpr int kTailN = 64;           // second chunk of a one-pass expert: at mo
 constexpr int BK = 64;               // K per stage: one 128-byte swizzle row of bf16
 constexpr int UMMA_K = 16;
 constexpr int kEpiWarps = 8;
+constexpr int kEpiGroups = kEpiWarps / 4;   // groups of 4 warps cover the 128 lanes
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kThreads = 64 + kEpiThreads;
 constexpr int kRowBytes = BK * 2;                               // one staged row: 128 bytes
@@ -70,7 +71,6 @@ constexpr int kTRows = (kMainN + kTailN) / 2;                   // routed rows p
 constexpr int kTailOff = (kMainN / 2) * kRowBytes;              // second chunk's rows: 16 KB in
 constexpr int kTBytes = kTRows * kRowBytes;                     // 20 KB
 constexpr int kStages = 5;
-constexpr int kPrefetch = 12;        // k-steps of weights brought into L2 ahead of the ring
 constexpr int kSlotCols = 256;
 constexpr int kTmemCols = 2 * kSlotCols;
 
@@ -81,8 +81,9 @@ constexpr int kGluPitch = 33;
 constexpr int kGluGroupBytes = 128 * kGluPitch * 4;              // 16896 B
 constexpr int kOutPitch = 36;
 constexpr int kOutWarpBytes = 32 * kOutPitch * 4;                // 4608 B
-constexpr int kEpiBytes = 2 * kGluGroupBytes > kEpiWarps * kOutWarpBytes ? 2 * kGluGroupBytes
-                                                                          : kEpiWarps * kOutWarpBytes;
+constexpr int kEpiBytes = kEpiGroups * kGluGroupBytes > kEpiWarps * kOutWarpBytes
+                              ? kEpiGroups * kGluGroupBytes
+                              : kEpiWarps * kOutWarpBytes;
 
 struct Smem {
     static constexpr int w = 0;
@@ -174,21 +175,19 @@ __device__ __forceinline__ bool group_all(int group, bool ok) {
 // ulp of fp32; the result is rounded to bf16).  e^-g = inf gives 0.
 __device__ __forceinline__ float silu_fast(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
-// Loads `rows` (a multiple of 8) routed rows starting at row r0, K columns
-// k0..k0+63, into shared memory at dst: one 128-row box for a full half
-// chunk, else 32-row boxes, then 8-row boxes.
+// Rows one TMA box stages for `rows` routed rows: the smallest of 8, 32
+// and 128 that covers them.  One box per chunk: each TMA instruction has a
+// large fixed cost, so a few extra rows (multiplied by nothing: the MMA reads
+// only `rows` of them) are cheaper than several smaller boxes.
+__device__ __forceinline__ int box_rows(int rows) { return rows <= 8 ? 8 : rows <= 32 ? 32 : 128; }
+
+// Loads the box covering `rows` routed rows from row r0, K columns
+// k0..k0+63, into shared memory at dst.
 __device__ __forceinline__ void load_rows(uint32_t dst, const CUtensorMap* m128,
                                           const CUtensorMap* m32, const CUtensorMap* m8,
                                           uint32_t bar, int k0, int r0, int rows) {
-    if (rows == 128) {
-        tma_load_2d<2>(dst, m128, bar, k0, r0);
-        return;
-    }
-    const int n_big = rows >> 5, n_small = (rows & 31) >> 3;
-    for (int b = 0; b < n_big; ++b)
-        tma_load_2d<2>(dst + b * 32 * kRowBytes, m32, bar, k0, r0 + 32 * b);
-    for (int b = 0; b < n_small; ++b)
-        tma_load_2d<2>(dst + (n_big * 32 + b * 8) * kRowBytes, m8, bar, k0, r0 + 32 * n_big + 8 * b);
+    const int b = box_rows(rows);
+    tma_load_2d<2>(dst, b == 128 ? m128 : b == 32 ? m32 : m8, bar, k0, r0);
 }
 
 template <bool GLU, typename OutT>
@@ -256,28 +255,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             return GLU ? ti.wt * kWRows + (int)rank * (kWRows / 2)
                        : ti.wt * 2 * kWRows + (int)rank * kWRows;
         };
-        // L2 prefetch cursor: walks the same (tile, k-step) sequence as the
-        // loads, kPrefetch steps ahead of them
-        int pt = unit, pk = 0;
-        TileInfo pti = {};
-        if (pt < n_tiles) pti = tile_info(p, s_prefix, pt);
-        auto prefetch_next = [&]() {
-            if (pt >= n_tiles) return;
-            if (GLU) tma_prefetch_l2_4d(&tmap_w, pk * BK, w_row(pti), 0, pti.j);
-            else tma_prefetch_l2_3d(&tmap_w, pk * BK, w_row(pti), pti.j);
-            if (++pk == nk) {
-                pk = 0;
-                pt += n_units;
-                if (pt < n_tiles) pti = tile_info(p, s_prefix, pt);
-            }
-        };
-        for (int i = 0; i < kPrefetch; ++i) prefetch_next();
         int stage = 0;
         uint32_t phase = 0;
         for (int t = unit; t < n_tiles; t += n_units) {
             const TileInfo ti = tile_info(p, s_prefix, t);
-            const int h0 = ti.n0 >> 1, h1 = ti.n1 >> 1;       // rows this CTA stages per chunk
-            const uint32_t tx = 2u * (uint32_t)(kWBytes + (h0 + h1) * kRowBytes);
+            const int h0 = ti.n0 >> 1, h1 = ti.n1 >> 1;       // rows this CTA multiplies per chunk
+            const uint32_t tx =
+                2u * (uint32_t)(kWBytes + (box_rows(h0) + (h1 ? box_rows(h1) : 0)) * kRowBytes);
             for (int kb = 0; kb < nk; ++kb) {
                 if (!mbar_wait(empty_bar(stage), phase ^ 1u, s_abort, p.dev_status)) {
                     aborted = true;
@@ -298,7 +282,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (h1)
                     load_rows(st + kTailOff, &tmap_t128, &tmap_t32, &tmap_t8, cfb, k0,
                               ti.row0 + kMainN + (int)rank * h1, h1);
-                prefetch_next();
                 if (++stage == kStages) {
                     stage = 0;
                     phase ^= 1u;
@@ -358,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp >= 2) {
         // ------------------------------------------------ epilogue (both CTAs)
         const int ew = warp - 2;                 // 0..7
-        const int group = ew >> 2;               // takes 32-column pieces group, group + 2, ..
+        const int group = ew >> 2;               // takes every kEpiGroups-th 32-column piece
         const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
         const int lrow = quarter * 32 + lane;    // this thread's weight row in the CTA
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
@@ -383,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const uint32_t tacc = tmem_base + lane_off + (nslot & 1) * kSlotCols;
 #pragma unroll 1
-                for (int col = 32 * group; col < ncols; col += 64) {
+                for (int col = 32 * group; col < ncols; col += 32 * kEpiGroups) {
                     float v[32];
                     tmem_ld32(tacc + (uint32_t)col, v);
                     tmem_ld_wait();

@@ -143,22 +143,6 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
 
-// Bring one TMA box into L2 without staging it anywhere (no barrier, no
-// completion to wait for): used to start DRAM reads further ahead than the
-// shared-memory ring allows.
-__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c0, int c1,
-                                                   int c2) {
-    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(map),
-                 "r"(c0), "r"(c1), "r"(c2)
-                 : "memory");
-}
-__device__ __forceinline__ void tma_prefetch_l2_4d(const CUtensorMap* map, int c0, int c1, int c2,
-                                                   int c3) {
-    asm volatile(
-        "cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(map),
-        "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-        : "memory");
-}
 
 // Shared-memory matrix descriptor for a K-major, 128-byte-swizzled bf16
 // tile whose rows are 128 bytes apart and whose 8-row groups are 1024 bytes
