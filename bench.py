@@ -463,13 +463,14 @@ def _graph_replay_us(wl, logits, x, w13, w2, buf, replays):
 def _profile_traffic(wl):
     """DRAM bytes per launch of the gate/up GEMM kernel on this workload, from
     the committed ncu summary -- None unless that summary was taken on the
-    same kernel source (checked by hash) and for this workload."""
+    same kernel source file (named in it, checked by hash) and for this
+    workload."""
     import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
             rec = json.load(f)
-        src = os.path.join(ROOT, "expert_parallelism_b200", "csrc", "grouped_gemm_tc.cu")
+        src = os.path.join(ROOT, "expert_parallelism_b200", "csrc", rec.get("source", "?"))
         digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
         if rec.get("source_sha256") != digest:
             return None
