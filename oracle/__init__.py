@@ -48,6 +48,8 @@ def _load():
         lib.oracle_route_topk.restype = I
         lib.oracle_dispatch_layout.argtypes = [P, I64, I32, I32, I32, P, P, P, P, P]
         lib.oracle_dispatch_layout.restype = I64
+        lib.oracle_route_topk_grouped.argtypes = [P, I64, I32, I32, I32, I32, P, P]
+        lib.oracle_route_topk_grouped.restype = I
         lib.oracle_dispatch_layout_capacity.argtypes = [P, I64, I32, I32, I32, I32, P, P, P, P,
                                                          P, P]
         lib.oracle_dispatch_layout_capacity.restype = I64
@@ -110,6 +112,20 @@ def route_topk(logits: torch.Tensor, k: int):
     idx = torch.empty(T, k, dtype=torch.int32)
     w = torch.empty(T, k, dtype=torch.float32)
     _load().oracle_route_topk(_p(logits), T, E, k, _p(idx), _p(w))
+    return idx, w
+
+
+def route_topk_grouped(logits: torch.Tensor, k: int, groups: int, max_groups: int):
+    """Top-k restricted to the ``max_groups`` best of ``groups`` equal expert
+    groups (a group's score: its largest logit); softmax over the picks."""
+    logits = logits.to(torch.float32).contiguous()
+    T, E = logits.shape
+    idx = torch.empty(T, k, dtype=torch.int32)
+    w = torch.empty(T, k, dtype=torch.float32)
+    rc = _load().oracle_route_topk_grouped(_p(logits), T, E, k, groups, max_groups, _p(idx),
+                                           _p(w))
+    if rc != 0:
+        raise ValueError("route_topk_grouped: need groups | E and k <= max_groups * E / groups")
     return idx, w
 
 

@@ -191,6 +191,70 @@ int oracle_route_topk(const float* logits, int64_t T, int32_t E, int32_t k,
 }
 
 /* ------------------------------------------------------------------ */
+/* S1' group-limited route: at most M expert groups per token           */
+/* ------------------------------------------------------------------ */
+/* "Expert Parallelism" (aiwiki), "Hiding the latency", topology-aware
+ * routing: DeepSeek-V3's router sends each token to at most 4 nodes, which
+ * bounds the inter-node fan-out.  The page does not say how the nodes are
+ * chosen.  Reading: the E experts form G equal groups of E/G consecutive
+ * experts (a node = a logical rank's block, "How the sizes combine"); a
+ * group's score is its largest logit; each token keeps the M groups with
+ * the largest scores (ties: lower group id) and picks its top k among their
+ * experts with the ordinary rule (logit descending, expert id ascending);
+ * the weights are the softmax over the k picks.  With M = G this is
+ * oracle_route_topk.  Needs G | E and k <= M * E / G.  Returns 0, or -1 on
+ * invalid sizes. */
+int oracle_route_topk_grouped(const float* logits, int64_t T, int32_t E, int32_t k, int32_t G,
+                              int32_t M, int32_t* topk_idx, float* topk_w) {
+    if (G < 1 || E % G != 0 || M < 1 || M > G || k < 1 || k > M * (E / G)) return -1;
+    const int32_t per = E / G;
+    float* score = (float*)malloc(sizeof(float) * (size_t)G);
+    unsigned char* keep = (unsigned char*)calloc((size_t)G, 1);
+    unsigned char* taken = (unsigned char*)calloc((size_t)E > 0 ? (size_t)E : 1u, 1);
+    double* z = (double*)malloc(sizeof(double) * (size_t)k);
+    for (int64_t t = 0; t < T; ++t) {
+        const float* L = logits + t * E;
+        for (int32_t g = 0; g < G; ++g) {
+            float m = L[g * per];
+            for (int32_t e = g * per + 1; e < (g + 1) * per; ++e)
+                if (L[e] > m) m = L[e];
+            score[g] = m;
+            keep[g] = 0;
+        }
+        for (int32_t r = 0; r < M; ++r) {     /* the M best groups */
+            int32_t best = -1;
+            for (int32_t g = 0; g < G; ++g) {
+                if (keep[g]) continue;
+                if (best < 0 || score[g] > score[best]) best = g;   /* ties keep lower id */
+            }
+            keep[best] = 1;
+        }
+        for (int32_t e = 0; e < E; ++e) taken[e] = 0;
+        for (int32_t j = 0; j < k; ++j) {     /* top k inside the kept groups */
+            int32_t best = -1;
+            for (int32_t e = 0; e < E; ++e) {
+                if (taken[e] || !keep[e / per]) continue;
+                if (best < 0 || L[e] > L[best]) best = e;
+            }
+            taken[best] = 1;
+            topk_idx[t * k + j] = best;
+        }
+        double m = (double)L[topk_idx[t * k]];
+        double sum = 0.0;
+        for (int32_t j = 0; j < k; ++j) {
+            z[j] = exp((double)L[topk_idx[t * k + j]] - m);
+            sum += z[j];
+        }
+        for (int32_t j = 0; j < k; ++j) topk_w[t * k + j] = (float)(z[j] / sum);
+    }
+    free(score);
+    free(keep);
+    free(taken);
+    free(z);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
 /* S2 dispatch layout: histogram, exclusive scan, stable counting sort */
 /* ------------------------------------------------------------------ */
 /* Pair p = t*k + j goes to expert idx[p].  Slots are expert-major, ties by
