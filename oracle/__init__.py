@@ -48,6 +48,10 @@ def _load():
         lib.oracle_route_topk.restype = I
         lib.oracle_dispatch_layout.argtypes = [P, I64, I32, I32, I32, P, P, P, P, P]
         lib.oracle_dispatch_layout.restype = I64
+        lib.oracle_quantize_rows_e4m3.argtypes = [P, I64, I32, P, P]
+        lib.oracle_quantize_rows_e4m3.restype = I
+        lib.oracle_combine_e4m3.argtypes = [P, P, P, P, I64, I32, I32, P, I]
+        lib.oracle_combine_e4m3.restype = I
         lib.oracle_route_topk_grouped.argtypes = [P, I64, I32, I32, I32, I32, P, P]
         lib.oracle_route_topk_grouped.restype = I
         lib.oracle_dispatch_layout_capacity.argtypes = [P, I64, I32, I32, I32, I32, P, P, P, P,
@@ -233,6 +237,35 @@ def combine(y: torch.Tensor, slot_of_pair: torch.Tensor, topk_w: torch.Tensor,
     return out
 
 
+def quantize_rows_e4m3(v: torch.Tensor):
+    """Per-128 block FP8 e4m3 quantisation of rows of fp32 values (the
+    dispatch payload's rule): returns (codes as float8_e4m3fn, fp32 scales)."""
+    v = v.to(torch.float32).contiguous()
+    rows, H = v.shape
+    q = torch.empty(rows, H, dtype=torch.uint8)
+    sc = torch.empty(rows, H // 128, dtype=torch.float32)
+    if _load().oracle_quantize_rows_e4m3(_p(v), rows, H, _p(q), _p(sc)) != 0:
+        raise ValueError("quantize_rows_e4m3: H must be a multiple of 128")
+    return q.view(torch.float8_e4m3fn), sc
+
+
+def combine_e4m3(q: torch.Tensor, scales: torch.Tensor, slot_of_pair: torch.Tensor,
+                 topk_w: torch.Tensor, out_dtype: str = "f64"):
+    """Weighted sum of each token's k FP8 rows, each dequantised as the fp32
+    product decode(q) * scale; summed in fp64 ("f64": unrounded)."""
+    q = q.contiguous().view(torch.uint8)
+    T, k = topk_w.shape
+    H = q.shape[1]
+    out = torch.empty(T, H, dtype=_TDT[out_dtype])
+    rc = _load().oracle_combine_e4m3(_p(q), _p(scales.to(torch.float32).contiguous()),
+                                     _p(slot_of_pair.to(torch.int32).contiguous()),
+                                     _p(topk_w.to(torch.float32).contiguous()), T, k, H,
+                                     _p(out), _CODE[out_dtype])
+    if rc != 0:
+        raise ValueError("combine_e4m3: H must be a multiple of 128")
+    return out
+
+
 def round_to(v: torch.Tensor, dtype: str) -> torch.Tensor:
     """fp64 values rounded to a storage type with the oracle's own rounding."""
     if dtype == "bf16":
@@ -249,7 +282,10 @@ def layer(wl, inputs, row_mask=None):
     rows; combine is then only meaningful for tokens whose pairs were all
     computed.  A workload with a capacity_factor uses the fixed-capacity
     layout (dropped pairs add nothing to out)."""
-    idx, w = route_topk(inputs["logits"], wl.k)
+    if getattr(wl, "route_groups", 0):
+        idx, w = route_topk_grouped(inputs["logits"], wl.k, wl.route_groups, wl.route_max_groups)
+    else:
+        idx, w = route_topk(inputs["logits"], wl.k)
     if getattr(wl, "capacity_factor", None) is None:
         lay = dispatch_layout(idx, wl.E, wl.W)
     else:   # fixed slabs: only the slab rows holding a pair are computed
@@ -260,5 +296,11 @@ def layer(wl, inputs, row_mask=None):
     xp, sc = permute(inputs["x"], wl.k, lay["pair_of_slot"], wl.payload)
     h, y, _ = grouped_gemm(xp, sc, lay["expert_offsets"], 0, wl.E, inputs["w13"], inputs["w2"],
                            row_mask)
+    if getattr(wl, "ydt", None) == "e4m3":
+        # FP8 combine payload: the exact y, held in fp32, quantised per 128 block
+        yq, ysc = quantize_rows_e4m3(torch.nan_to_num(y, nan=0.0).float())
+        out = combine_e4m3(yq, ysc, lay["slot_of_pair"], w)
+        return dict(topk_idx=idx, topk_w=w, xp=xp, xp_scales=sc, h=h, y=y, y_q=yq, y_scales=ysc,
+                    out=out, **lay)
     out = combine(y, lay["slot_of_pair"], w)
     return dict(topk_idx=idx, topk_w=w, xp=xp, xp_scales=sc, h=h, y=y, out=out, **lay)

@@ -438,6 +438,63 @@ int64_t oracle_grouped_gemm(const void* xp, int xp_dt, const float* xp_scales,
 }
 
 /* ------------------------------------------------------------------ */
+/* S5' FP8 combine payload: y as e4m3 codes with per-128 block scales   */
+/* ------------------------------------------------------------------ */
+/* "Expert parallelism and all-to-all", "Traffic math": the figure of
+ * 2 * k * H * bytes per token assumes 1-byte activations both ways, i.e.
+ * the experts' outputs also travel back as FP8.  Reading: each y row is
+ * quantised exactly like the dispatch payload (per 128-element block of
+ * the fp32 value: scale = amax / 448 by fp32 IEEE division, 1 when amax is
+ * 0; q = e4m3(y / scale), fp32 IEEE division, round-to-nearest-even,
+ * saturating), and the combine uses decode(q) * scale as an fp32 product.
+ * oracle_quantize_rows_e4m3 quantises rows of fp32 values; the caller
+ * passes fp32(y). */
+int oracle_quantize_rows_e4m3(const float* v, int64_t rows, int32_t H, uint8_t* q,
+                              float* scales) {
+    if ((H % 128) != 0) return -1;
+    const int32_t nb = H / 128;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int32_t b = 0; b < nb; ++b) {
+            const float* blk = v + r * H + b * 128;
+            float amax = 0.0f;
+            for (int32_t i = 0; i < 128; ++i)
+                if (fabsf(blk[i]) > amax) amax = fabsf(blk[i]);
+            float scale = amax / 448.0f;
+            if (scale == 0.0f) scale = 1.0f;
+            scales[r * nb + b] = scale;
+            for (int32_t i = 0; i < 128; ++i) q[r * H + b * 128 + i] = e4m3_from_float(blk[i] / scale);
+        }
+    }
+    return 0;
+}
+
+/* Combine from an FP8 y: out[t] = sum_j w[t,j] * (float)(decode(q) * scale)
+ * for each kept pick, summed in fp64 in j order (out_dt fp64: unrounded). */
+int oracle_combine_e4m3(const uint8_t* q, const float* scales, const int32_t* slot_of_pair,
+                        const float* topk_w, int64_t T, int32_t k, int32_t H, void* out,
+                        int out_dt) {
+    if ((H % 128) != 0) return -1;
+    const int32_t nb = H / 128;
+    double* acc = (double*)malloc(sizeof(double) * (size_t)H);
+    for (int64_t t = 0; t < T; ++t) {
+        for (int32_t c = 0; c < H; ++c) acc[c] = 0.0;
+        for (int32_t j = 0; j < k; ++j) {
+            const int32_t s = slot_of_pair[t * k + j];
+            if (s < 0) continue;
+            const double w = (double)topk_w[t * k + j];
+            for (int32_t c = 0; c < H; ++c) {
+                const float yv = (float)(e4m3_to_double(q[(int64_t)s * H + c]) *
+                                         (double)scales[(int64_t)s * nb + c / 128]);
+                acc[c] += w * (double)yv;
+            }
+        }
+        for (int32_t c = 0; c < H; ++c) store_elem(out, out_dt, t * H + c, acc[c]);
+    }
+    free(acc);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
 /* S5 combine: out[t] = sum_j w[t,j] * y[slot_of_pair[t*k+j]]          */
 /* ------------------------------------------------------------------ */
 /* The un-permute of the aiwiki sketch (y[order] = back) fused with the
