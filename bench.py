@@ -184,7 +184,10 @@ def oracle_sample(wl, target_s: float = 12.0, max_tokens: int | None = None):
         sub = wl.replace(T=S)
         lg, x = logits_all[:S].contiguous(), x_all[:S].contiguous()
         t0 = time.perf_counter()
-        idx, w = oracle.route_topk(lg, wl.k)
+        if wl.route_groups:
+            idx, w = oracle.route_topk_grouped(lg, wl.k, wl.route_groups, wl.route_max_groups)
+        else:
+            idx, w = oracle.route_topk(lg, wl.k)
         if wl.capacity_factor is None:
             lay = oracle.dispatch_layout(idx, wl.E, wl.W)
         else:
@@ -276,6 +279,8 @@ def _config(wl):
             "logical_ranks": wl.W, "activations": wl.act, "payload": wl.payload,
             "gemm": wl.wdt, "y": wl.ydt, "router": wl.router, "seed": wl.seed, "l2": l2,
             **({"capacity_factor": wl.capacity_factor} if wl.capacity_factor is not None else {}),
+            **({"route_groups": wl.route_groups, "route_max_groups": wl.route_max_groups}
+               if wl.route_groups else {}),
             "parallelism": "replicas (one independent layer per GPU)"}
 
 
@@ -383,8 +388,8 @@ def run_ours(args, wl):
             "route_topk": {"us": avg["route_topk"] * 1e3,
                            "gbs": gbs(kb["route_topk"], avg["route_topk"])},
             "dispatch_layout": {"us": avg["dispatch_layout"] * 1e3},
-            "permute": {"us": avg["permute"] * 1e3, "bytes": kb["permute"],
-                        "gbs": gbs(kb["permute"], avg["permute"])},
+            "permute": {"us": avg["permute"] * 1e3, "bytes": kb["permute_layer"],
+                        "gbs": gbs(kb["permute_layer"], avg["permute"])},
             "grouped_gemm": {"us": gemm_ms * 1e3, "flops": fl["total"],
                              "tflops": tf(fl["total"], gemm_ms),
                              "dequant_e4m3_us": avg["dequant_e4m3"] * 1e3,

@@ -69,7 +69,8 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
                 raise RuntimeError("nvcc failed: " + " ".join(cmd))
     if force or _stale(LIB, objs):
         tmp = LIB + f".tmp{os.getpid()}"
-        subprocess.check_call([NVCC, *ARCH, "-shared", "--cudart", "static", "-o", tmp, *objs])
+        subprocess.check_call([NVCC, *ARCH, "-shared", "--cudart", "static", "-Xlinker",
+                               "--no-undefined", "-o", tmp, *objs])
         os.replace(tmp, LIB)
     return LIB
 

@@ -11,14 +11,16 @@
 #include "common.cuh"
 
 namespace moe {
-cudaError_t launch_route_topk(const float*, int64_t, int, int, int32_t*, float*, cudaStream_t);
+cudaError_t launch_route_topk(const float*, int64_t, int, int, int, int, int32_t*, float*,
+                              cudaStream_t);
 size_t layout_workspace_bytes(int64_t T, int k, int E);
 cudaError_t launch_dispatch_layout(const int32_t*, int64_t, int, int, int, int, int32_t*,
                                    int32_t*, int32_t*, int32_t*, int32_t*, int32_t*, void*,
                                    int32_t*, cudaStream_t);
 cudaError_t launch_permute(const void*, moe_dtype, int64_t, int, int, const int32_t*, void*,
-                           moe_dtype, float*, cudaStream_t);
-cudaError_t launch_combine(const void*, moe_dtype, const int32_t*, const float*, int64_t, int,
+                           moe_dtype, float*, __nv_bfloat16*, cudaStream_t);
+cudaError_t launch_combine(const void*, moe_dtype, const float*, const int32_t*, const float*,
+                           int64_t, int,
                            int, void*, moe_dtype, cudaStream_t);
 cudaError_t launch_dequant_e4m3(const uint8_t*, const float*, const int32_t*, int, int, int64_t,
                                 int, __nv_bfloat16*, cudaStream_t);
@@ -27,7 +29,7 @@ cudaError_t launch_grouped_gemm_simt_f32(const float*, const int32_t*, const int
                                          float*, cudaEvent_t, cudaStream_t);
 cudaError_t launch_grouped_gemm_tc(const __nv_bfloat16*, const int32_t*, const int32_t*, int, int,
                                    int64_t, int, int, const __nv_bfloat16*, const __nv_bfloat16*,
-                                   __nv_bfloat16*, void*, bool, int32_t*, cudaEvent_t,
+                                   __nv_bfloat16*, void*, moe_dtype, float*, int32_t*, cudaEvent_t,
                                    cudaStream_t);
 }  // namespace moe
 
@@ -60,6 +62,15 @@ moe_status check_route(const float* logits, int64_t T, int32_t E, int32_t k,
     if (E > MOE_MAX_EXPERTS || k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
     if (T == 0) return *noop = true, MOE_OK;
     if (!logits || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+// Group-limited routing: G equal groups (G | E, 1 <= G <= 32), at most M
+// of them per token (1 <= M <= G) with enough experts for k picks.
+moe_status check_route_groups(int32_t E, int32_t k, int32_t G, int32_t M) {
+    if (G < 1 || M < 1 || M > G || (E % G) != 0) return MOE_ERR_INVALID_ARG;
+    if ((int64_t)k > (int64_t)M * (E / G)) return MOE_ERR_INVALID_ARG;
+    if (G > 32) return MOE_ERR_UNSUPPORTED;
     return MOE_OK;
 }
 
@@ -103,8 +114,8 @@ moe_status check_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_scales
                       const int32_t* expert_offsets, int32_t expert_begin, int32_t n_experts,
                       int64_t n_rows, int32_t H, int32_t I, const void* w13, const void* w2,
                       moe_dtype w_dtype, const void* h, const void* y, moe_dtype y_dtype,
-                      const void* workspace, size_t workspace_bytes, const int32_t* dev_status,
-                      bool* noop) {
+                      const float* y_scales, const void* workspace, size_t workspace_bytes,
+                      const int32_t* dev_status, bool* noop) {
     *noop = false;
     if (n_rows < 0 || H < 1 || I < 1 || (H % 8) != 0 || (I % 8) != 0) return MOE_ERR_INVALID_ARG;
     if (expert_begin < 0 || n_experts < 1) return MOE_ERR_INVALID_ARG;
@@ -112,7 +123,10 @@ moe_status check_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_scales
     const bool f32 = (w_dtype == MOE_F32 && xp_dtype == MOE_F32);
     const bool bf16 = (w_dtype == MOE_BF16 && (xp_dtype == MOE_BF16 || xp_dtype == MOE_E4M3));
     if (!f32 && !bf16) return MOE_ERR_INVALID_ARG;
-    if (y_dtype != MOE_F32 && !(bf16 && y_dtype == MOE_BF16)) return MOE_ERR_INVALID_ARG;
+    // y: fp32 (either path), bf16 or the FP8 combine payload (bf16 path only)
+    if (y_dtype != MOE_F32 && !(bf16 && (y_dtype == MOE_BF16 || y_dtype == MOE_E4M3)))
+        return MOE_ERR_INVALID_ARG;
+    if (y_dtype == MOE_E4M3 && ((H % 128) != 0 || !y_scales)) return MOE_ERR_INVALID_ARG;
     if (xp_dtype == MOE_E4M3 && ((H % 128) != 0 || !xp_scales)) return MOE_ERR_INVALID_ARG;
     if (!expert_offsets || !w13 || !w2 || !dev_status) return MOE_ERR_INVALID_ARG;
     if (n_rows == 0) return *noop = true, MOE_OK;
@@ -125,12 +139,14 @@ moe_status check_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_scales
     return MOE_OK;
 }
 
-moe_status check_combine(const void* y, moe_dtype y_dtype, const int32_t* slot_of_pair,
-                         const float* topk_w, int64_t T, int32_t k, int32_t H, const void* out,
-                         moe_dtype out_dtype, bool* noop) {
+moe_status check_combine(const void* y, moe_dtype y_dtype, const float* y_scales,
+                         const int32_t* slot_of_pair, const float* topk_w, int64_t T, int32_t k,
+                         int32_t H, const void* out, moe_dtype out_dtype, bool* noop) {
     *noop = false;
     if (T < 0 || H < 1 || k < 1 || (H % 8) != 0) return MOE_ERR_INVALID_ARG;
-    if (!is_act_dtype(y_dtype) || !is_act_dtype(out_dtype)) return MOE_ERR_INVALID_ARG;
+    if (!(is_act_dtype(y_dtype) || y_dtype == MOE_E4M3) || !is_act_dtype(out_dtype))
+        return MOE_ERR_INVALID_ARG;
+    if (y_dtype == MOE_E4M3 && ((H % 128) != 0 || !y_scales)) return MOE_ERR_INVALID_ARG;
     if (k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
     if (T == 0) return *noop = true, MOE_OK;
     if (!y || !slot_of_pair || !topk_w || !out || !aligned16(y) || !aligned16(out))
@@ -144,9 +160,10 @@ cudaError_t run_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_scales,
                      const int32_t* expert_offsets, const int32_t* expert_counts,
                      int32_t expert_begin, int32_t n_experts,
                      int64_t n_rows, int32_t H, int32_t I, const void* w13, const void* w2,
-                     moe_dtype w_dtype, void* h, void* y, moe_dtype y_dtype, void* workspace,
-                     int32_t* dev_status, cudaStream_t s, cudaEvent_t ev_a = nullptr,
-                     cudaEvent_t ev_b = nullptr) {
+                     moe_dtype w_dtype, void* h, void* y, moe_dtype y_dtype, float* y_scales,
+                     void* workspace, int32_t* dev_status, cudaStream_t s,
+                     cudaEvent_t ev_a = nullptr, cudaEvent_t ev_b = nullptr,
+                     bool a_ready = false) {
     cudaError_t e = cudaSuccess;
     if (w_dtype == MOE_F32) {
         if (ev_a) e = cudaEventRecord(ev_a, s);
@@ -158,8 +175,10 @@ cudaError_t run_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_scales,
     }
     const __nv_bfloat16* a = (const __nv_bfloat16*)xp;
     if (xp_dtype == MOE_E4M3) {
-        e = launch_dequant_e4m3((const uint8_t*)xp, xp_scales, expert_offsets, expert_begin,
-                                n_experts, n_rows, H, (__nv_bfloat16*)workspace, s);
+        // the FP8 rows' bf16 operand, unless the permute already wrote it
+        if (!a_ready)
+            e = launch_dequant_e4m3((const uint8_t*)xp, xp_scales, expert_offsets, expert_begin,
+                                    n_experts, n_rows, H, (__nv_bfloat16*)workspace, s);
         if (e != cudaSuccess) return e;
         a = (const __nv_bfloat16*)workspace;
     }
@@ -168,7 +187,7 @@ cudaError_t run_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_scales,
     return launch_grouped_gemm_tc(a, expert_offsets, expert_counts, expert_begin, n_experts,
                                   n_rows, H, I,
                                   (const __nv_bfloat16*)w13, (const __nv_bfloat16*)w2,
-                                  (__nv_bfloat16*)h, y, y_dtype == MOE_F32, dev_status, ev_b, s);
+                                  (__nv_bfloat16*)h, y, y_dtype, y_scales, dev_status, ev_b, s);
 }
 
 }  // namespace
@@ -181,7 +200,18 @@ moe_status moe_route_topk(const float* logits, int64_t T, int32_t E, int32_t k,
     const moe_status st = check_route(logits, T, E, k, topk_idx, topk_w, &noop);
     if (st != MOE_OK || noop) return st;
     return cuda_status(
-        launch_route_topk(logits, T, E, k, topk_idx, topk_w, (cudaStream_t)stream));
+        launch_route_topk(logits, T, E, k, 0, 0, topk_idx, topk_w, (cudaStream_t)stream));
+}
+
+moe_status moe_route_topk_grouped(const float* logits, int64_t T, int32_t E, int32_t k,
+                                  int32_t groups, int32_t max_groups, int32_t* topk_idx,
+                                  float* topk_w, void* stream) {
+    bool noop;
+    moe_status st = check_route_groups(E, k, groups, max_groups);
+    if (st == MOE_OK) st = check_route(logits, T, E, k, topk_idx, topk_w, &noop);
+    if (st != MOE_OK || noop) return st;
+    return cuda_status(launch_route_topk(logits, T, E, k, groups, max_groups, topk_idx, topk_w,
+                                         (cudaStream_t)stream));
 }
 
 size_t moe_dispatch_layout_workspace_bytes(int64_t T, int32_t k, int32_t E) {
@@ -232,7 +262,7 @@ moe_status moe_permute(const void* x, moe_dtype x_dtype, int64_t T, int32_t H, i
         check_permute(x, x_dtype, T, H, k, slot_of_pair, xp, xp_dtype, xp_scales, &noop);
     if (st != MOE_OK || noop) return st;
     return cuda_status(launch_permute(x, x_dtype, T, H, k, slot_of_pair, xp, xp_dtype, xp_scales,
-                                      (cudaStream_t)stream));
+                                      nullptr, (cudaStream_t)stream));
 }
 
 size_t moe_grouped_gemm_workspace_bytes(int64_t n_rows, int32_t H, int32_t I, moe_dtype xp_dtype,
@@ -247,28 +277,28 @@ moe_status moe_grouped_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_
                             int32_t expert_begin,
                             int32_t n_experts, int64_t n_rows, int32_t H, int32_t I,
                             const void* w13, const void* w2, moe_dtype w_dtype, void* h, void* y,
-                            moe_dtype y_dtype, void* workspace, size_t workspace_bytes,
-                            int32_t* dev_status, void* stream) {
+                            moe_dtype y_dtype, float* y_scales, void* workspace,
+                            size_t workspace_bytes, int32_t* dev_status, void* stream) {
     bool noop;
     const moe_status st =
         check_gemm(xp, xp_dtype, xp_scales, expert_offsets, expert_begin, n_experts, n_rows, H,
-                   I, w13, w2, w_dtype, h, y, y_dtype, workspace, workspace_bytes, dev_status,
-                   &noop);
+                   I, w13, w2, w_dtype, h, y, y_dtype, y_scales, workspace, workspace_bytes,
+                   dev_status, &noop);
     if (st != MOE_OK || noop) return st;
     return cuda_status(run_gemm(xp, xp_dtype, xp_scales, expert_offsets, expert_counts,
                                 expert_begin, n_experts, n_rows, H, I, w13, w2, w_dtype, h, y,
-                                y_dtype, workspace, dev_status, (cudaStream_t)stream));
+                                y_dtype, y_scales, workspace, dev_status, (cudaStream_t)stream));
 }
 
-moe_status moe_combine(const void* y, moe_dtype y_dtype, const int32_t* slot_of_pair,
-                       const float* topk_w, int64_t T, int32_t k, int32_t H, void* out,
-                       moe_dtype out_dtype, void* stream) {
+moe_status moe_combine(const void* y, moe_dtype y_dtype, const float* y_scales,
+                       const int32_t* slot_of_pair, const float* topk_w, int64_t T, int32_t k,
+                       int32_t H, void* out, moe_dtype out_dtype, void* stream) {
     bool noop;
-    const moe_status st =
-        check_combine(y, y_dtype, slot_of_pair, topk_w, T, k, H, out, out_dtype, &noop);
+    const moe_status st = check_combine(y, y_dtype, y_scales, slot_of_pair, topk_w, T, k, H, out,
+                                        out_dtype, &noop);
     if (st != MOE_OK || noop) return st;
-    return cuda_status(launch_combine(y, y_dtype, slot_of_pair, topk_w, T, k, H, out, out_dtype,
-                                      (cudaStream_t)stream));
+    return cuda_status(launch_combine(y, y_dtype, y_scales, slot_of_pair, topk_w, T, k, H, out,
+                                      out_dtype, (cudaStream_t)stream));
 }
 
 // Rows of the permuted buffers: T*k (dropless) or E*capacity (fixed slabs).
@@ -276,15 +306,23 @@ static int64_t layer_slots(int64_t T, int32_t k, int32_t E, int32_t capacity) {
     return capacity < 0 ? T * k : (int64_t)E * capacity;
 }
 
+static moe_layer_options resolve(const moe_layer_options* o) {
+    return o ? *o : moe_layer_options{-1, 0, 0};
+}
+
 static moe_status check_layer(const float* logits, const void* x, moe_dtype x_dtype, int64_t T,
                               int32_t H, int32_t E, int32_t k, int32_t W, int32_t I,
                               const void* w13, const void* w2, moe_dtype w_dtype,
-                              moe_dtype payload_dtype, moe_dtype y_dtype, int32_t capacity,
-                              const moe_layer_buffers* b, const void* out) {
+                              moe_dtype payload_dtype, moe_dtype y_dtype,
+                              const moe_layer_options& o, const moe_layer_buffers* b,
+                              const void* out) {
     if (!b) return MOE_ERR_INVALID_ARG;
+    const int32_t capacity = o.capacity;
     if (capacity >= 0 && (int64_t)E * capacity >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
     bool noop;
-    moe_status st = check_route(logits, T, E, k, b->topk_idx, b->topk_w, &noop);
+    moe_status st = MOE_OK;
+    if (o.route_groups != 0) st = check_route_groups(E, k, o.route_groups, o.route_max_groups);
+    if (st == MOE_OK) st = check_route(logits, T, E, k, b->topk_idx, b->topk_w, &noop);
     if (st == MOE_OK)
         st = check_layout(b->topk_idx, T, k, E, W, b->expert_counts, b->expert_offsets,
                           b->rank_offsets, b->slot_of_pair, b->pair_of_slot,
@@ -295,26 +333,30 @@ static moe_status check_layer(const float* logits, const void* x, moe_dtype x_dt
     if (st == MOE_OK)
         st = check_gemm(b->xp, payload_dtype, b->xp_scales, b->expert_offsets, 0, E,
                         layer_slots(T, k, E, capacity), H, I, w13, w2, w_dtype, b->h, b->y,
-                        y_dtype, b->gemm_workspace, b->gemm_workspace_bytes, b->dev_status,
+                        y_dtype, b->y_scales, b->gemm_workspace, b->gemm_workspace_bytes,
+                        b->dev_status,
                         &noop);
     if (st == MOE_OK)
-        st = check_combine(b->y, y_dtype, b->slot_of_pair, b->topk_w, T, k, H, out, x_dtype,
-                           &noop);
+        st = check_combine(b->y, y_dtype, b->y_scales, b->slot_of_pair, b->topk_w, T, k, H, out,
+                           x_dtype, &noop);
     return st;
 }
 
 static cudaError_t launch_layer(const float* logits, const void* x, moe_dtype x_dtype, int64_t T,
                                 int32_t H, int32_t E, int32_t k, int32_t W, int32_t I,
                                 const void* w13, const void* w2, moe_dtype w_dtype,
-                                moe_dtype payload_dtype, moe_dtype y_dtype, int32_t capacity,
-                                const moe_layer_buffers* b, void* out, void* const* ev,
-                                cudaStream_t s) {
+                                moe_dtype payload_dtype, moe_dtype y_dtype,
+                                const moe_layer_options& o, const moe_layer_buffers* b, void* out,
+                                void* const* ev, cudaStream_t s) {
+    const int32_t capacity = o.capacity;
     const int64_t n_slots = layer_slots(T, k, E, capacity);
     auto mark = [&](int i) {
         return ev ? cudaEventRecord((cudaEvent_t)ev[i], s) : cudaSuccess;
     };
     cudaError_t e = mark(0);
-    if (e == cudaSuccess && T > 0) e = launch_route_topk(logits, T, E, k, b->topk_idx, b->topk_w, s);
+    if (e == cudaSuccess && T > 0)
+        e = launch_route_topk(logits, T, E, k, o.route_groups, o.route_max_groups, b->topk_idx,
+                              b->topk_w, s);
     if (e == cudaSuccess) e = mark(1);
     if (e == cudaSuccess)
         e = launch_dispatch_layout(b->topk_idx, T, k, E, W, capacity < 0 ? -1 : capacity,
@@ -325,20 +367,24 @@ static cudaError_t launch_layer(const float* logits, const void* x, moe_dtype x_
     if (e == cudaSuccess) e = mark(2);
     if (e == cudaSuccess && T > 0)
         e = launch_permute(x, x_dtype, T, H, k, b->slot_of_pair, b->xp, payload_dtype,
-                           b->xp_scales, s);
+                           b->xp_scales,
+                           payload_dtype == MOE_E4M3 ? (__nv_bfloat16*)b->gemm_workspace : nullptr,
+                           s);
     if (e == cudaSuccess) e = mark(3);
     if (e == cudaSuccess && T > 0 && n_slots > 0) {
         e = run_gemm(b->xp, payload_dtype, b->xp_scales, b->expert_offsets,
                      capacity < 0 ? nullptr : b->expert_counts, 0, E, n_slots, H, I, w13, w2,
-                     w_dtype, b->h, b->y, y_dtype, b->gemm_workspace, b->dev_status, s,
-                     ev ? (cudaEvent_t)ev[4] : nullptr, ev ? (cudaEvent_t)ev[5] : nullptr);
+                     w_dtype, b->h, b->y, y_dtype, b->y_scales, b->gemm_workspace, b->dev_status,
+                     s, ev ? (cudaEvent_t)ev[4] : nullptr, ev ? (cudaEvent_t)ev[5] : nullptr,
+                     /*a_ready=*/true);
     } else if (e == cudaSuccess) {
         e = mark(4);
         if (e == cudaSuccess) e = mark(5);
     }
     if (e == cudaSuccess) e = mark(6);
     if (e == cudaSuccess && T > 0)
-        e = launch_combine(b->y, y_dtype, b->slot_of_pair, b->topk_w, T, k, H, out, x_dtype, s);
+        e = launch_combine(b->y, y_dtype, b->y_scales, b->slot_of_pair, b->topk_w, T, k, H, out,
+                           x_dtype, s);
     if (e == cudaSuccess) e = mark(7);
     return e;
 }
@@ -346,14 +392,15 @@ static cudaError_t launch_layer(const float* logits, const void* x, moe_dtype x_
 moe_status moe_layer_forward(const float* logits, const void* x, moe_dtype x_dtype, int64_t T,
                              int32_t H, int32_t E, int32_t k, int32_t W, int32_t I,
                              const void* w13, const void* w2, moe_dtype w_dtype,
-                             moe_dtype payload_dtype, moe_dtype y_dtype, int32_t capacity,
-                             const moe_layer_buffers* b, void* out, void* const* step_events,
-                             void* stream) {
+                             moe_dtype payload_dtype, moe_dtype y_dtype,
+                             const moe_layer_options* opts, const moe_layer_buffers* b, void* out,
+                             void* const* step_events, void* stream) {
+    const moe_layer_options o = resolve(opts);
     const moe_status st = check_layer(logits, x, x_dtype, T, H, E, k, W, I, w13, w2, w_dtype,
-                                      payload_dtype, y_dtype, capacity, b, out);
+                                      payload_dtype, y_dtype, o, b, out);
     if (st != MOE_OK) return st;
     return cuda_status(launch_layer(logits, x, x_dtype, T, H, E, k, W, I, w13, w2, w_dtype,
-                                    payload_dtype, y_dtype, capacity, b, out, step_events,
+                                    payload_dtype, y_dtype, o, b, out, step_events,
                                     (cudaStream_t)stream));
 }
 
@@ -362,10 +409,11 @@ moe_status moe_layer_forward_host(const float* logits_host, const void* x_host, 
                                   moe_dtype x_dtype, int64_t T, int32_t H, int32_t E, int32_t k,
                                   int32_t W, int32_t I, const void* w13, const void* w2,
                                   moe_dtype w_dtype, moe_dtype payload_dtype, moe_dtype y_dtype,
-                                  int32_t capacity, const moe_layer_buffers* b,
+                                  const moe_layer_options* opts, const moe_layer_buffers* b,
                                   void* const* step_events, void* stream) {
+    const moe_layer_options o = resolve(opts);
     const moe_status st = check_layer(logits_dev, x_dev, x_dtype, T, H, E, k, W, I, w13, w2,
-                                      w_dtype, payload_dtype, y_dtype, capacity, b, out_dev);
+                                      w_dtype, payload_dtype, y_dtype, o, b, out_dev);
     if (st != MOE_OK) return st;
     if (T > 0 && (!logits_host || !x_host || !out_host)) return MOE_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
@@ -378,7 +426,7 @@ moe_status moe_layer_forward_host(const float* logits_host, const void* x_host, 
     }
     if (e == cudaSuccess)
         e = launch_layer(logits_dev, x_dev, x_dtype, T, H, E, k, W, I, w13, w2, w_dtype,
-                         payload_dtype, y_dtype, capacity, b, out_dev, step_events, s);
+                         payload_dtype, y_dtype, o, b, out_dev, step_events, s);
     if (e == cudaSuccess && T > 0)
         e = cudaMemcpyAsync(out_host, out_dev, xb, cudaMemcpyDeviceToHost, s);
     return cuda_status(e);

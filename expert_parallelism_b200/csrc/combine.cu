@@ -10,6 +10,11 @@
 // elements; for every pick j it loads that piece of row y[slot_of_pair[t*k
 // + j]] (16-byte vector loads, all k issued before the sums), accumulates
 // w_j * y in fp32 with fused multiply-adds in j order, and rounds once.
+//
+// With the FP8 combine payload ("Expert parallelism and all-to-all",
+// "Traffic math": 1-byte activations both ways) y holds e4m3 codes with one
+// fp32 scale per 128 elements; a piece is 8 codes (one 8-byte load) and its
+// block's scale, used as decode(q) * scale, an fp32 product.
 #include "common.cuh"
 
 namespace moe {
@@ -41,8 +46,33 @@ __device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&f)[8]) {
                         pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7])));
 }
 
+// Piece c (8 elements) of row s of y as fp32.
+template <typename TY>
+__device__ __forceinline__ void load_piece(const TY* y, const float* y_scales, int64_t s, int H,
+                                           int c, float (&f)[8]) {
+    (void)y_scales;
+    load8_row(y + s * H + c * 8, f);
+}
+template <>
+__device__ __forceinline__ void load_piece<uint8_t>(const uint8_t* y, const float* y_scales,
+                                                    int64_t s, int H, int c, float (&f)[8]) {
+    const uint2 q = ld_nc_v2(y + s * H + c * 8);
+    const float sc = __ldg(y_scales + s * (H / 128) + (c * 8) / 128);
+    const uint32_t w[2] = {q.x, q.y};
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const float2 a = decode2_e4m3((uint16_t)(w[i] & 0xFFFFu));
+        const float2 b = decode2_e4m3((uint16_t)(w[i] >> 16));
+        f[4 * i + 0] = a.x * sc;
+        f[4 * i + 1] = a.y * sc;
+        f[4 * i + 2] = b.x * sc;
+        f[4 * i + 3] = b.y * sc;
+    }
+}
+
 template <typename TY, typename TO>
 __global__ void __launch_bounds__(256) combine_kernel(const TY* __restrict__ y,
+                                                      const float* __restrict__ y_scales,
                                                       const int32_t* __restrict__ slot_of_pair,
                                                       const float* __restrict__ topk_w, int64_t T,
                                                       int k, int H, TO* __restrict__ out) {
@@ -66,7 +96,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const TY* __restrict__ y,
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const int32_t s = s_slot[j + u];
-                    if (s >= 0) load8_row(y + (int64_t)s * H + c * 8, v[u]);
+                    if (s >= 0) load_piece(y, y_scales, s, H, c, v[u]);
                 }
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
@@ -80,7 +110,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const TY* __restrict__ y,
                 const int32_t s = s_slot[j];
                 if (s < 0) continue;
                 float v[8];
-                load8_row(y + (int64_t)s * H + c * 8, v);
+                load_piece(y, y_scales, s, H, c, v);
                 const float w = s_w[j];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) acc[i] = fmaf(w, v[i], acc[i]);
@@ -91,9 +121,9 @@ __global__ void __launch_bounds__(256) combine_kernel(const TY* __restrict__ y,
     }
 }
 
-cudaError_t launch_combine(const void* y, moe_dtype ydt, const int32_t* slot_of_pair,
-                           const float* topk_w, int64_t T, int k, int H, void* out,
-                           moe_dtype odt, cudaStream_t s) {
+cudaError_t launch_combine(const void* y, moe_dtype ydt, const float* y_scales,
+                           const int32_t* slot_of_pair, const float* topk_w, int64_t T, int k,
+                           int H, void* out, moe_dtype odt, cudaStream_t s) {
     if (T == 0) return cudaSuccess;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -102,10 +132,12 @@ cudaError_t launch_combine(const void* y, moe_dtype ydt, const int32_t* slot_of_
     const unsigned grid = (unsigned)(T < cap ? T : cap);
     int threads = ((H / 8 + 31) / 32) * 32;
     threads = threads < 32 ? 32 : (threads > 256 ? 256 : threads);
-#define MOE_COMBINE(TY, TO)                                                                    \
-    combine_kernel<TY, TO><<<grid, threads, 0, s>>>((const TY*)y, slot_of_pair, topk_w, T, k, \
-                                                    H, (TO*)out)
-    if (ydt == MOE_BF16 && odt == MOE_BF16) MOE_COMBINE(__nv_bfloat16, __nv_bfloat16);
+#define MOE_COMBINE(TY, TO)                                                               \
+    combine_kernel<TY, TO><<<grid, threads, 0, s>>>((const TY*)y, y_scales, slot_of_pair, \
+                                                    topk_w, T, k, H, (TO*)out)
+    if (ydt == MOE_E4M3 && odt == MOE_BF16) MOE_COMBINE(uint8_t, __nv_bfloat16);
+    else if (ydt == MOE_E4M3) MOE_COMBINE(uint8_t, float);
+    else if (ydt == MOE_BF16 && odt == MOE_BF16) MOE_COMBINE(__nv_bfloat16, __nv_bfloat16);
     else if (ydt == MOE_BF16) MOE_COMBINE(__nv_bfloat16, float);
     else if (odt == MOE_BF16) MOE_COMBINE(float, __nv_bfloat16);
     else MOE_COMBINE(float, float);

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -73,10 +74,43 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
                  : "l"(p));
     return r;
 }
+__device__ __forceinline__ uint2 ld_nc_v2(const void* p) {
+    uint2 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+                 : "=r"(r.x), "=r"(r.y)
+                 : "l"(p));
+    return r;
+}
 __device__ __forceinline__ void st_v4(void* p, const uint4& v) {
     asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y),
                  "r"(v.z), "r"(v.w)
                  : "memory");
+}
+
+// The FP8 payload rule, shared by the dispatch payload (permute) and the
+// combine payload (the down GEMM's epilogue): for a block with largest
+// magnitude amax, scale = amax / 448 (IEEE fp32 division; 1 for an all-zero
+// block), and each value is encoded as e4m3(v / scale) (IEEE division, then
+// the hardware's round-to-nearest-even, saturating conversion).
+__device__ __forceinline__ float e4m3_block_scale(float amax) {
+    const float s = __fdiv_rn(amax, 448.0f);
+    return s == 0.0f ? 1.0f : s;
+}
+
+// Four e4m3 codes of a / scale .. d / scale, packed low byte first.
+__device__ __forceinline__ uint32_t quant4_e4m3(float a, float b, float c, float d, float scale) {
+    const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
+        make_float2(__fdiv_rn(a, scale), __fdiv_rn(b, scale)), __NV_SATFINITE, __NV_E4M3);
+    const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+        make_float2(__fdiv_rn(c, scale), __fdiv_rn(d, scale)), __NV_SATFINITE, __NV_E4M3);
+    return (uint32_t)lo | ((uint32_t)hi << 16);
+}
+
+// Two e4m3 codes (low byte first) decoded to fp32 (exact: e4m3 values are
+// fp16 values).
+__device__ __forceinline__ float2 decode2_e4m3(uint16_t two) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two, __NV_E4M3);
+    return __half22float2(*reinterpret_cast<const __half2*>(&h));
 }
 
 inline int ceil_div(int64_t a, int64_t b) { return (int)((a + b - 1) / b); }

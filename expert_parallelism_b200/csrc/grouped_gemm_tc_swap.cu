@@ -32,7 +32,12 @@
 // receives its 128 weight rows (lanes) x the chunk's rows (columns).  Phase
 // 1 stages, per CTA, 64 gate rows and the 64 matching up rows, so lanes
 // 0..63 hold gate and 64..127 up for the same 64 features; the epilogue
-// pairs them through shared memory.  Phase 2 stages 128 rows of W2 per CTA.
+// pairs them through shared memory.  Phase 2 stages 128 rows of W2 per CTA;
+// its output y is fp32, bf16, or the FP8 combine payload: e4m3 codes with one
+// fp32 scale per 128 features ("Expert parallelism and all-to-all", "Traffic
+// math": 1-byte activations both ways).  A CTA's 128 weight rows are exactly
+// one such block, so each block's amax is a max over one epilogue group's
+// four warps.
 //
 // Rows come in expert segments [off[j], off[j+1]) read from device memory
 // (tile_schedule.cuh).  Chunk rows past the segment are loaded (TMA
@@ -85,6 +90,9 @@ constexpr int kEpiBytes = kEpiGroups * kGluGroupBytes > kEpiWarps * kOutWarpByte
                               ? kEpiGroups * kGluGroupBytes
                               : kEpiWarps * kOutWarpBytes;
 
+// FP8 y: per-token partial amax of each warp's 32 features, double-buffered
+constexpr int kAmaxBytes = 2 * kEpiGroups * 4 * 32 * 4;
+
 struct Smem {
     static constexpr int w = 0;
     static constexpr int t = w + kStages * kWBytes;
@@ -94,7 +102,8 @@ struct Smem {
     static constexpr int prefix = misc + 16;                 // int32 [MOE_MAX_EXPERTS + 1]
     static constexpr int warp_sums = prefix + (MOE_MAX_EXPERTS + 1) * 4;
     static constexpr int epi = ((warp_sums + (kThreads / 32) * 4 + 127) / 128) * 128;
-    static constexpr int total = epi + kEpiBytes;
+    static constexpr int amax = epi + kEpiBytes;
+    static constexpr int total = amax + kAmaxBytes;
     static constexpr size_t alloc = total + 1024;            // + alignment slack
 };
 static_assert(Smem::alloc <= 232448, "smem budget");
@@ -110,6 +119,7 @@ struct Params {
     int n_wtiles;             // weight tiles per pass
     int n_rows;               // rows of A and out: stores never go past it
     void* out;                // h (phase 1, bf16) or y (phase 2, OutT), row stride n_out
+    float* out_scales;        // y's block scales [n_rows, n_out / 128] when OutT is e4m3
     int32_t* dev_status;
 };
 
@@ -349,6 +359,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         float* glu_stage = reinterpret_cast<float*>(smem + Smem::epi + group * kGluGroupBytes);
         float* out_stage = reinterpret_cast<float*>(smem + Smem::epi + ew * kOutWarpBytes);
         OutT* out = reinterpret_cast<OutT*>(p.out);
+        constexpr bool kFP8 = sizeof(OutT) == 1;          // e4m3 codes + block scales
+        float* s_amax = reinterpret_cast<float*>(smem + Smem::amax);
+        uint32_t piece = 0;                               // FP8: amax buffer parity
         uint32_t nslot = 0;
         for (int t = unit; t < n_tiles && !aborted; t += n_units) {
             const TileInfo ti = tile_info(p, s_prefix, t);
@@ -358,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int ncols = c == 0 ? ti.n0 : ti.n1;
                 const int crow0 = ti.row0 + c * kMainN;      // chunk's first routed row
                 bool ok = mbar_wait(tfull_bar(nslot & 1), (nslot >> 1) & 1, s_abort, p.dev_status);
-                if (GLU) ok = group_all(group, ok);
+                if (GLU || kFP8) ok = group_all(group, ok);
                 if (!ok) {
                     aborted = true;
                     break;
@@ -397,6 +410,51 @@ __global__ void __launch_bounds__(kThreads, 1)
                                       make_uint4(pack_bf16x2(hv[0], hv[1]), pack_bf16x2(hv[2], hv[3]),
                                                  pack_bf16x2(hv[4], hv[5]), pack_bf16x2(hv[6], hv[7])));
                         }
+                    } else if constexpr (kFP8) {
+                        // this warp: 32 outputs (its lanes) x 32 chunk rows (v); lane l
+                        // then takes chunk row l: its amax over this warp's 32
+                        // outputs, the block amax over the group's four warps, and
+                        // 32 codes (32 bytes) of the row's 128-wide block
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) out_stage[i * kOutPitch + lane] = v[i];
+                        __syncwarp();
+                        float rv[32];
+                        float part = 0.0f;
+#pragma unroll
+                        for (int q4 = 0; q4 < 8; ++q4) {
+                            const float4 f =
+                                *reinterpret_cast<const float4*>(out_stage + lane * kOutPitch + 4 * q4);
+                            rv[4 * q4 + 0] = f.x;
+                            rv[4 * q4 + 1] = f.y;
+                            rv[4 * q4 + 2] = f.z;
+                            rv[4 * q4 + 3] = f.w;
+                            part = fmaxf(part, fmaxf(fmaxf(fabsf(f.x), fabsf(f.y)),
+                                                     fmaxf(fabsf(f.z), fabsf(f.w))));
+                        }
+                        float* amax_buf = s_amax + ((piece & 1) * kEpiGroups + group) * 128;
+                        amax_buf[quarter * 32 + lane] = part;
+                        group_bar(group);
+                        const float amax = fmaxf(fmaxf(amax_buf[lane], amax_buf[32 + lane]),
+                                                 fmaxf(amax_buf[64 + lane], amax_buf[96 + lane]));
+                        const float scale = e4m3_block_scale(amax);
+                        const int64_t row = crow0 + col + lane;
+                        const int blk0 = ti.wt * 2 * kWRows + (int)rank * kWRows;   // block start
+                        if (row < row_end && blk0 < p.n_out) {
+                            uint8_t* dst =
+                                reinterpret_cast<uint8_t*>(out) + row * p.n_out + blk0 + quarter * 32;
+                            st_v4(dst, make_uint4(quant4_e4m3(rv[0], rv[1], rv[2], rv[3], scale),
+                                                  quant4_e4m3(rv[4], rv[5], rv[6], rv[7], scale),
+                                                  quant4_e4m3(rv[8], rv[9], rv[10], rv[11], scale),
+                                                  quant4_e4m3(rv[12], rv[13], rv[14], rv[15], scale)));
+                            st_v4(dst + 16,
+                                  make_uint4(quant4_e4m3(rv[16], rv[17], rv[18], rv[19], scale),
+                                             quant4_e4m3(rv[20], rv[21], rv[22], rv[23], scale),
+                                             quant4_e4m3(rv[24], rv[25], rv[26], rv[27], scale),
+                                             quant4_e4m3(rv[28], rv[29], rv[30], rv[31], scale)));
+                            if (quarter == 0) p.out_scales[row * (p.n_out / 128) + blk0 / 128] = scale;
+                        }
+                        ++piece;
+                        __syncwarp();
                     } else {
                         // this warp: 32 outputs (its lanes) x 32 chunk rows (v)
 #pragma unroll
@@ -542,14 +600,16 @@ static bool make_row_maps(CUtensorMap* m, const void* base, int K, int64_t n_row
 }  // namespace tcs
 
 // A [n_rows, H] bf16; W13 [n_exp, 2I, H]; W2 [n_exp, H, I]; h [n_rows, I]
-// bf16; y [n_rows, H] in y_f32 ? fp32 : bf16.  counts (may be null) cuts
+// bf16; y [n_rows, H] in y_dtype (fp32, bf16, or e4m3 codes with fp32
+// y_scales [n_rows, H/128]).  counts (may be null) cuts
 // each expert's segment to its first counts[j] rows.  ev_mid (may be null)
 // is recorded between the two phases.
 cudaError_t launch_grouped_gemm_tc_swap(const __nv_bfloat16* a, const int32_t* offsets,
                                         const int32_t* counts, int expert_begin, int n_experts,
                                         int64_t n_rows, int H, int I, const __nv_bfloat16* w13,
                                         const __nv_bfloat16* w2, __nv_bfloat16* h, void* y,
-                                        bool y_f32, int32_t* dev_status, cudaEvent_t ev_mid,
+                                        moe_dtype y_dtype, float* y_scales, int32_t* dev_status,
+                                        cudaEvent_t ev_mid,
                                         cudaStream_t s) {
     using namespace tcs;
     CUtensorMap mw1, mt1[3], mw2, mt2[3];
@@ -570,14 +630,15 @@ cudaError_t launch_grouped_gemm_tc_swap(const __nv_bfloat16* a, const int32_t* o
     if (!make_row_maps(mt2, h, I, n_rows)) return cudaErrorInvalidValue;
 
     Params p1{offsets, counts, expert_begin, n_experts, H, I, (I + kWRows - 1) / kWRows,
-              (int)n_rows, h, dev_status};
+              (int)n_rows, h, nullptr, dev_status};
     cudaError_t e = launch_phase<true, __nv_bfloat16>(mw1, mt1, p1, s);
     if (e == cudaSuccess && ev_mid) e = cudaEventRecord(ev_mid, s);
     if (e != cudaSuccess) return e;
     Params p2{offsets, counts, expert_begin, n_experts, I, H, (H + 2 * kWRows - 1) / (2 * kWRows),
-              (int)n_rows, y, dev_status};
-    e = y_f32 ? launch_phase<false, float>(mw2, mt2, p2, s)
-              : launch_phase<false, __nv_bfloat16>(mw2, mt2, p2, s);
+              (int)n_rows, y, y_scales, dev_status};
+    e = y_dtype == MOE_F32    ? launch_phase<false, float>(mw2, mt2, p2, s)
+        : y_dtype == MOE_BF16 ? launch_phase<false, __nv_bfloat16>(mw2, mt2, p2, s)
+                              : launch_phase<false, uint8_t>(mw2, mt2, p2, s);
     note_launches(2);
     return e;
 }

@@ -55,16 +55,6 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&f)[8]) {
     unpack16(ld_nc_v4(p), f);
 }
 
-// Four e4m3 codes of a / scale (IEEE divisions, RNE, saturating), packed
-// low byte first.
-__device__ __forceinline__ uint32_t quant4(float a, float b, float c, float d, float scale) {
-    const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
-        make_float2(__fdiv_rn(a, scale), __fdiv_rn(b, scale)), __NV_SATFINITE, __NV_E4M3);
-    const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
-        make_float2(__fdiv_rn(c, scale), __fdiv_rn(d, scale)), __NV_SATFINITE, __NV_E4M3);
-    return (uint32_t)lo | ((uint32_t)hi << 16);
-}
-
 constexpr int kQuantThreads = 256;
 constexpr int kMaxBlocks = 64;           // scales staged in shared memory: H <= 8192
 
@@ -72,11 +62,14 @@ constexpr int kMaxBlocks = 64;           // scales staged in shared memory: H <=
 // block (16 elements each): amax by shuffles, scale = amax / 448, and
 // 16-byte stores of codes to each of the token's k slots.  The token's
 // scales are staged in shared memory and written as 16-byte vectors per
-// slot once the row is done.
+// slot once the row is done.  With `a` non-null (the layer call), the
+// kernel also writes what the grouped GEMM consumes, bf16(decode(q) *
+// scale) (an fp32 product rounded to bf16), to each slot's row of `a`,
+// so the GEMM needs no separate dequantisation pass.
 template <typename T>
 __global__ void __launch_bounds__(kQuantThreads) permute_e4m3_kernel(
     const T* __restrict__ x, int64_t T_, int H, int k, const int32_t* __restrict__ slot_of_pair,
-    uint8_t* __restrict__ xp, float* __restrict__ xp_scales) {
+    uint8_t* __restrict__ xp, float* __restrict__ xp_scales, __nv_bfloat16* __restrict__ a) {
     __shared__ int32_t s_slot[kMaxTopK];
     __shared__ __align__(16) float s_scale[kMaxBlocks];
     const int nblk = H / 128;
@@ -110,15 +103,35 @@ __global__ void __launch_bounds__(kQuantThreads) permute_e4m3_kernel(
             for (int off = 4; off > 0; off >>= 1)
                 amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
             if (!live) continue;
-            float scale = __fdiv_rn(amax, 448.0f);
-            if (scale == 0.0f) scale = 1.0f;
-            const uint4 q = make_uint4(quant4(f[0], f[1], f[2], f[3], scale),
-                                       quant4(f[4], f[5], f[6], f[7], scale),
-                                       quant4(f[8], f[9], f[10], f[11], scale),
-                                       quant4(f[12], f[13], f[14], f[15], scale));
+            const float scale = e4m3_block_scale(amax);
+            const uint4 q = make_uint4(quant4_e4m3(f[0], f[1], f[2], f[3], scale),
+                                       quant4_e4m3(f[4], f[5], f[6], f[7], scale),
+                                       quant4_e4m3(f[8], f[9], f[10], f[11], scale),
+                                       quant4_e4m3(f[12], f[13], f[14], f[15], scale));
             for (int j = 0; j < k; ++j) {
                 const int32_t s = s_slot[j];
                 if (s >= 0) st_v4(xp + (int64_t)s * H + g * 128 + l8 * 16, q);
+            }
+            if (a) {
+                // the GEMM's operand: each code decoded (exact) times the scale
+                const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+                uint32_t bw[8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 lo = decode2_e4m3((uint16_t)(qw[i] & 0xFFFFu));
+                    const float2 hi = decode2_e4m3((uint16_t)(qw[i] >> 16));
+                    bw[2 * i] = pack_bf16x2(__fmul_rn(lo.x, scale), __fmul_rn(lo.y, scale));
+                    bw[2 * i + 1] = pack_bf16x2(__fmul_rn(hi.x, scale), __fmul_rn(hi.y, scale));
+                }
+                const uint4 b0 = make_uint4(bw[0], bw[1], bw[2], bw[3]);
+                const uint4 b1 = make_uint4(bw[4], bw[5], bw[6], bw[7]);
+                for (int j = 0; j < k; ++j) {
+                    const int32_t s = s_slot[j];
+                    if (s < 0) continue;
+                    __nv_bfloat16* dst = a + (int64_t)s * H + g * 128 + l8 * 16;
+                    st_v4(dst, b0);
+                    st_v4(dst + 8, b1);
+                }
             }
             if (l8 == 0) {
                 if (vec_scales) {
@@ -152,18 +165,20 @@ static unsigned permute_grid(int64_t T) {
     return (unsigned)(T < cap ? T : cap);
 }
 
+// a_bf16 (may be null; FP8 payload only): also write the GEMM's bf16
+// operand bf16(decode(q) * scale) for every slot.
 cudaError_t launch_permute(const void* x, moe_dtype xdt, int64_t T, int H, int k,
                            const int32_t* slot_of_pair, void* xp, moe_dtype xpdt,
-                           float* xp_scales, cudaStream_t s) {
+                           float* xp_scales, __nv_bfloat16* a_bf16, cudaStream_t s) {
     if (T == 0) return cudaSuccess;
     const unsigned grid = permute_grid(T);
     if (xpdt == MOE_E4M3) {
         if (xdt == MOE_BF16)
             permute_e4m3_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-                (const __nv_bfloat16*)x, T, H, k, slot_of_pair, (uint8_t*)xp, xp_scales);
+                (const __nv_bfloat16*)x, T, H, k, slot_of_pair, (uint8_t*)xp, xp_scales, a_bf16);
         else
-            permute_e4m3_kernel<float><<<grid, 256, 0, s>>>((const float*)x, T, H, k,
-                                                            slot_of_pair, (uint8_t*)xp, xp_scales);
+            permute_e4m3_kernel<float><<<grid, 256, 0, s>>>(
+                (const float*)x, T, H, k, slot_of_pair, (uint8_t*)xp, xp_scales, a_bf16);
     } else if (xdt == MOE_BF16) {
         permute_copy_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
             (const __nv_bfloat16*)x, T, H, k, slot_of_pair, (__nv_bfloat16*)xp);

@@ -29,6 +29,7 @@ _P, _I64, _I32, _SZ, _I = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctyp
                            ctypes.c_int)
 SIGNATURES = {
     "moe_route_topk": ([_P, _I64, _I32, _I32, _P, _P, _P], _I),
+    "moe_route_topk_grouped": ([_P, _I64, _I32, _I32, _I32, _I32, _P, _P, _P], _I),
     "moe_dispatch_layout_workspace_bytes": ([_I64, _I32, _I32], _SZ),
     "moe_dispatch_layout": ([_P, _I64, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _SZ, _P, _P], _I),
     "moe_dispatch_layout_capacity": ([_P, _I64, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P,
@@ -38,16 +39,21 @@ SIGNATURES = {
     "moe_permute": ([_P, _I, _I64, _I32, _I32, _P, _P, _I, _P, _P], _I),
     "moe_grouped_gemm_workspace_bytes": ([_I64, _I32, _I32, _I, _I], _SZ),
     "moe_grouped_gemm": ([_P, _I, _P, _P, _P, _I32, _I32, _I64, _I32, _I32, _P, _P, _I, _P, _P,
-                          _I, _P, _SZ, _P, _P], _I),
-    "moe_combine": ([_P, _I, _P, _P, _I64, _I32, _I32, _P, _I, _P], _I),
+                          _I, _P, _P, _SZ, _P, _P], _I),
+    "moe_combine": ([_P, _I, _P, _P, _P, _I64, _I32, _I32, _P, _I, _P], _I),
     "moe_layer_forward": ([_P, _P, _I, _I64, _I32, _I32, _I32, _I32, _I32, _P, _P, _I, _I, _I,
-                           _I32, _P, _P, _P, _P], _I),
+                           _P, _P, _P, _P, _P], _I),
     "moe_layer_forward_host": ([_P, _P, _P, _P, _P, _P, _I, _I64, _I32, _I32, _I32, _I32, _I32,
-                                _P, _P, _I, _I, _I, _I32, _P, _P, _P], _I),
+                                _P, _P, _I, _I, _I, _P, _P, _P, _P], _I),
     "moe_check_status": ([_P, _P], _I),
     "moe_status_str": ([_I], ctypes.c_char_p),
     "moe_launch_count": ([], ctypes.c_uint64),
 }
+
+
+class LayerOptionsC(ctypes.Structure):
+    """moe_layer_options (include/moe.h)."""
+    _fields_ = [("capacity", _I32), ("route_groups", _I32), ("route_max_groups", _I32)]
 
 
 class LayerBuffersC(ctypes.Structure):
@@ -56,7 +62,7 @@ class LayerBuffersC(ctypes.Structure):
                 ("expert_offsets", _P), ("rank_offsets", _P), ("slot_of_pair", _P),
                 ("pair_of_slot", _P), ("layout_workspace", _P),
                 ("layout_workspace_bytes", _SZ), ("xp", _P), ("xp_scales", _P), ("h", _P),
-                ("y", _P), ("gemm_workspace", _P), ("gemm_workspace_bytes", _SZ),
+                ("y", _P), ("y_scales", _P), ("gemm_workspace", _P), ("gemm_workspace_bytes", _SZ),
                 ("dev_status", _P), ("n_dropped", _P)]
 
 
@@ -113,6 +119,14 @@ def moe_route_topk(logits, topk_idx, topk_w, stream=None):
         _ptr(logits), T, E, k, _ptr(topk_idx), _ptr(topk_w), _stream(stream)))
 
 
+def moe_route_topk_grouped(logits, groups, max_groups, topk_idx, topk_w, stream=None):
+    T, E = logits.shape
+    k = topk_idx.shape[1]
+    _check("moe_route_topk_grouped", load_library().moe_route_topk_grouped(
+        _ptr(logits), T, E, k, groups, max_groups, _ptr(topk_idx), _ptr(topk_w),
+        _stream(stream)))
+
+
 def moe_dispatch_layout_workspace_bytes(T, k, E) -> int:
     return int(load_library().moe_dispatch_layout_workspace_bytes(T, k, E))
 
@@ -160,7 +174,7 @@ def moe_grouped_gemm_workspace_bytes(n_rows, H, I, xp_dtype, w_dtype) -> int:
 
 
 def moe_grouped_gemm(xp, xp_scales, expert_offsets, expert_begin, n_experts, w13, w2, h, y,
-                     workspace, dev_status, stream=None, expert_counts=None):
+                     workspace, dev_status, stream=None, expert_counts=None, y_scales=None):
     n_rows, H = xp.shape
     I = w2.shape[2]
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
@@ -168,15 +182,16 @@ def moe_grouped_gemm(xp, xp_scales, expert_offsets, expert_begin, n_experts, w13
         _ptr(xp), dtype_code(xp), _ptr(xp_scales), _ptr(expert_offsets), _ptr(expert_counts),
         expert_begin,
         n_experts, n_rows, H, I, _ptr(w13), _ptr(w2), dtype_code(w13), _ptr(h), _ptr(y),
-        dtype_code(y), _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream)))
+        dtype_code(y), _ptr(y_scales), _ptr(workspace), ws_bytes, _ptr(dev_status),
+        _stream(stream)))
 
 
-def moe_combine(y, slot_of_pair, topk_w, out, stream=None):
+def moe_combine(y, slot_of_pair, topk_w, out, stream=None, y_scales=None):
     T, k = topk_w.shape
     H = y.shape[1]
     _check("moe_combine", load_library().moe_combine(
-        _ptr(y), dtype_code(y), _ptr(slot_of_pair), _ptr(topk_w), T, k, H, _ptr(out),
-        dtype_code(out), _stream(stream)))
+        _ptr(y), dtype_code(y), _ptr(y_scales), _ptr(slot_of_pair), _ptr(topk_w), T, k, H,
+        _ptr(out), dtype_code(out), _stream(stream)))
 
 
 def moe_check_status(dev_status, stream=None) -> int:
@@ -235,6 +250,8 @@ class LayerBuffers:
         wdt = TORCH_DTYPE[wl.wdt]
         self.h = torch.empty(N, I, dtype=wdt, device=dev)
         self.y = torch.empty(N, H, dtype=TORCH_DTYPE[wl.ydt], device=dev)
+        self.y_scales = (torch.empty(N, H // 128, dtype=torch.float32, device=dev)
+                         if wl.ydt == "e4m3" else None)
         gb = moe_grouped_gemm_workspace_bytes(N, H, I, pdt, wdt)
         self.gemm_ws = torch.empty(gb, dtype=torch.uint8, device=dev) if gb else None
         self.out = torch.empty(T, H, dtype=TORCH_DTYPE[wl.act], device=dev)
@@ -249,7 +266,8 @@ def layer_buffers_c(buf: "LayerBuffers") -> LayerBuffersC:
         _ptr(buf.topk_idx), _ptr(buf.topk_w), _ptr(buf.expert_counts), _ptr(buf.expert_offsets),
         _ptr(buf.rank_offsets), _ptr(buf.slot_of_pair), _ptr(buf.pair_of_slot),
         _ptr(buf.layout_ws), _nbytes(buf.layout_ws), _ptr(buf.xp), _ptr(buf.xp_scales),
-        _ptr(buf.h), _ptr(buf.y), _ptr(buf.gemm_ws), _nbytes(buf.gemm_ws), _ptr(buf.dev_status),
+        _ptr(buf.h), _ptr(buf.y), _ptr(buf.y_scales), _ptr(buf.gemm_ws), _nbytes(buf.gemm_ws),
+        _ptr(buf.dev_status),
         _ptr(buf.n_dropped))
 
 
@@ -265,6 +283,10 @@ def _events(step_events, stream=None):
     return ctypes.cast(arr, ctypes.c_void_p), arr
 
 
+def layer_options(wl, buf: "LayerBuffers") -> LayerOptionsC:
+    return LayerOptionsC(buf.capacity, wl.route_groups, wl.route_max_groups)
+
+
 def moe_layer_forward(wl, logits, x, w13, w2, buf: "LayerBuffers", step_events=None,
                       stream=None):
     """The whole hot path in one C call (route, layout, permute, grouped
@@ -274,8 +296,9 @@ def moe_layer_forward(wl, logits, x, w13, w2, buf: "LayerBuffers", step_events=N
     ev = _events(step_events, stream)
     _check("moe_layer_forward", load_library().moe_layer_forward(
         _ptr(logits), _ptr(x), dtype_code(x), wl.T, wl.H, wl.E, wl.k, wl.W, wl.I, _ptr(w13),
-        _ptr(w2), dtype_code(w13), dtype_code(buf.xp), dtype_code(buf.y), buf.capacity,
-        ctypes.byref(cb), _ptr(buf.out), ev[0] if ev else None, _stream(stream)))
+        _ptr(w2), dtype_code(w13), dtype_code(buf.xp), dtype_code(buf.y),
+        ctypes.byref(layer_options(wl, buf)), ctypes.byref(cb), _ptr(buf.out),
+        ev[0] if ev else None, _stream(stream)))
     return buf.out
 
 
@@ -287,8 +310,9 @@ def moe_layer_forward_host(wl, logits_host, x_host, out_host, logits_dev, x_dev,
     _check("moe_layer_forward_host", load_library().moe_layer_forward_host(
         _ptr(logits_host), _ptr(x_host), _ptr(out_host), _ptr(logits_dev), _ptr(x_dev),
         _ptr(buf.out), dtype_code(x_dev), wl.T, wl.H, wl.E, wl.k, wl.W, wl.I, _ptr(w13), _ptr(w2),
-        dtype_code(w13), dtype_code(buf.xp), dtype_code(buf.y), buf.capacity, ctypes.byref(cb),
-        ev[0] if ev else None, _stream(stream)))
+        dtype_code(w13), dtype_code(buf.xp), dtype_code(buf.y),
+        ctypes.byref(layer_options(wl, buf)), ctypes.byref(cb), ev[0] if ev else None,
+        _stream(stream)))
 
 
 def layer_forward(wl, logits, x, w13, w2, buf: "LayerBuffers", stream=None):

@@ -34,7 +34,11 @@ def kernel_bytes(wl: Workload, rows: int | None = None) -> dict:
         "route_topk": T * E * 4 + T * k * 8,
         "dispatch_layout": N * 4 + N * 8 + (2 * E + 1) * 4 + (wl.W + 1) * 4,
         "permute": T * H * xb + N * H * pb + scales,
-        "combine": N * H * yb + T * k * 8 + T * H * xb,
+        # inside moe_layer_forward an FP8 permute also writes the GEMM's bf16 rows
+        "permute_layer": T * H * xb + N * H * pb + scales
+                         + (N * H * 2 if wl.payload == "e4m3" else 0),
+        "combine": N * H * yb + (N * (H // 128) * 4 if wl.ydt == "e4m3" else 0)
+                   + T * k * 8 + T * H * xb,
     }
 
 

@@ -60,6 +60,8 @@ class Workload:
     seed: int = 0
     ydt: str = "f32"         # storage of the experts' outputs y (combine's input)
     capacity_factor: float | None = None   # None: dropless; else fixed slabs per expert
+    route_groups: int = 0                  # 0: plain top-k; G: group-limited routing
+    route_max_groups: int = 0              # M: groups a token may reach (with route_groups)
 
     @property
     def N(self) -> int:
@@ -86,6 +88,12 @@ WORKLOADS = {
                          capacity_factor=1.0),
     "skew_cap": Workload("skew_cap", 16384, 2880, 128, 4, 2880, 8, "bf16", "bf16", "bf16",
                          router="zipf", capacity_factor=1.25),
+    # FP8 combine payload: the experts' outputs travel back as e4m3 + block scales
+    "dsv3_fp8y": Workload("dsv3_fp8y", 8192, 7168, 256, 8, 2048, 8, "bf16", "e4m3", "bf16",
+                          ydt="e4m3"),
+    # group-limited routing: each token reaches at most 4 of the 8 rank groups
+    "dsv3_grouped": Workload("dsv3_grouped", 8192, 7168, 256, 8, 2048, 8, "bf16", "e4m3",
+                             "bf16", route_groups=8, route_max_groups=4),
 }
 
 TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16,

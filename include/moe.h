@@ -18,8 +18,14 @@
  *   moe_permute          x[T,H], slot_of_pair        -> xp[N,H] (+ FP8 block scales)
  *   moe_grouped_gemm     xp, offsets, W13, W2        -> h[N,I], y[N,H]  (SwiGLU FFN)
  *   moe_combine          y, slot_of_pair, topk_w     -> out[T,H]
+ *   moe_layer_forward    the five calls in one, with per-step events
  *
  * with N = T*k routed pairs; pair p = t*k + j is token t's j-th pick.
+ * Variants the pages discuss: moe_route_topk_grouped (at most M expert
+ * groups per token), moe_dispatch_layout_capacity (fixed slabs of C rows per
+ * expert, dropping the rest), an FP8 combine payload (y as e4m3 + block
+ * scales), and moe_dispatch_layout_noalloc (the layout without a caller
+ * workspace).
  *
  * Conventions shared by every call:
  *  - All arrays are dense, row-major, and live in device memory (except
@@ -67,7 +73,7 @@ typedef enum moe_status {
 typedef enum moe_dtype {
     MOE_F32 = 0,  /* IEEE binary32 */
     MOE_BF16 = 1, /* bfloat16 */
-    MOE_E4M3 = 2  /* OCP FP8 E4M3 (no infinities, max 448), payload only */
+    MOE_E4M3 = 2  /* OCP FP8 E4M3 (no infinities, max 448): payloads (xp, y) only */
 } moe_dtype;
 
 /* Bits of the device status word. */
@@ -97,6 +103,29 @@ typedef enum moe_dtype {
  */
 moe_status moe_route_topk(const float* logits, int64_t T, int32_t E, int32_t k,
                           int32_t* topk_idx, float* topk_w, void* stream);
+
+/*
+ * moe_route_topk_grouped -- moe_route_topk restricted to at most
+ * `max_groups` expert groups per token.
+ *
+ * Source: "Expert Parallelism" (aiwiki), "Hiding the latency",
+ * topology-aware routing: DeepSeek-V3's router sends each token to at most
+ * 4 nodes, bounding the inter-node fan-out.  The page does not say how the
+ * nodes are chosen; this library reads it as: the E experts form `groups`
+ * equal groups of consecutive ids (a node holds a logical rank's block); a
+ * group's score is its largest logit; each token keeps the `max_groups`
+ * groups with the highest scores (ties: lower group id) and takes its top k
+ * among their experts with the rule of moe_route_topk (logit descending,
+ * expert id ascending); the weights are the softmax over the k picks.
+ * max_groups == groups gives moe_route_topk's result.
+ *
+ * Arguments as moe_route_topk.  Requires groups | E, 1 <= max_groups <=
+ * groups, k <= max_groups * E / groups (MOE_ERR_INVALID_ARG otherwise) and
+ * groups <= 32 (MOE_ERR_UNSUPPORTED).
+ */
+moe_status moe_route_topk_grouped(const float* logits, int64_t T, int32_t E, int32_t k,
+                                  int32_t groups, int32_t max_groups, int32_t* topk_idx,
+                                  float* topk_w, void* stream);
 
 /*
  * moe_dispatch_layout -- the dispatch plan: a per-expert histogram, its
@@ -253,11 +282,18 @@ moe_status moe_permute(const void* x, moe_dtype x_dtype, int64_t T, int32_t H, i
  *   h              [n_rows, I] in w_dtype, written for the experts' rows (the
  *                  down projection's operand, so it has the GEMM's dtype).
  *   y              [n_rows, H] in y_dtype, written for the experts' rows:
- *                  MOE_F32 (either path) or MOE_BF16 (bf16 path only).  fp32
- *                  keeps the combine within 2e-2 of a row's RMS of the exact
- *                  layer output; a bf16 y adds a second bf16 rounding before
- *                  the weighted sum, which alone can take the largest
- *                  elements of a row past that bound.
+ *                  MOE_F32 (either path), MOE_BF16 or MOE_E4M3 (bf16 path
+ *                  only).  fp32 keeps the combine within 2e-2 of a row's RMS
+ *                  of the exact layer output; a bf16 y adds a second bf16
+ *                  rounding before the weighted sum, which alone can take the
+ *                  largest elements of a row past that bound.  MOE_E4M3 is
+ *                  the FP8 combine payload ("Expert parallelism and
+ *                  all-to-all", "Traffic math": 1-byte activations both
+ *                  ways): per 128 outputs of a row, scale = amax/448 of the
+ *                  fp32 values and the codes e4m3(y/scale), by the same rule
+ *                  as moe_permute's FP8 payload; requires H % 128 == 0.
+ *   y_scales       [n_rows, H/128] fp32, written when y_dtype == MOE_E4M3,
+ *                  else ignored (may be NULL).
  *   workspace      device scratch of moe_grouped_gemm_workspace_bytes(...)
  *                  bytes (may be 0 / NULL when that is 0), 128-byte aligned.
  *   dev_status     int32 device word (MOE_DEV_TIMEOUT on a bounded wait
@@ -275,7 +311,7 @@ moe_status moe_grouped_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_
                             int32_t expert_begin,
                             int32_t n_experts, int64_t n_rows, int32_t H, int32_t I,
                             const void* w13, const void* w2, moe_dtype w_dtype, void* h,
-                            void* y, moe_dtype y_dtype, void* workspace,
+                            void* y, moe_dtype y_dtype, float* y_scales, void* workspace,
                             size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /*
@@ -289,15 +325,19 @@ moe_status moe_grouped_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_
  * weighted sum into the residual stream); Transformers docs (the weighted
  * expert output for each token).
  *
- *   y            [>= max slot + 1, H] in y_dtype (MOE_F32 / MOE_BF16), device.
+ *   y            [>= max slot + 1, H] in y_dtype (MOE_F32 / MOE_BF16, or MOE_E4M3
+ *                codes: each element used as decode(q) * scale of its
+ *                128-element block, an fp32 product), device.
+ *   y_scales     [>= max slot + 1, H/128] fp32 when y_dtype == MOE_E4M3
+ *                (H % 128 == 0), else ignored (may be NULL).
  *   slot_of_pair [T*k] int32, device.
  *   topk_w       [T, k] fp32, device.
  *   out          [T, H] in out_dtype (MOE_F32 / MOE_BF16), device, written.
  * Requires H % 8 == 0, k >= 1.
  */
-moe_status moe_combine(const void* y, moe_dtype y_dtype, const int32_t* slot_of_pair,
-                       const float* topk_w, int64_t T, int32_t k, int32_t H, void* out,
-                       moe_dtype out_dtype, void* stream);
+moe_status moe_combine(const void* y, moe_dtype y_dtype, const float* y_scales,
+                       const int32_t* slot_of_pair, const float* topk_w, int64_t T, int32_t k,
+                       int32_t H, void* out, moe_dtype out_dtype, void* stream);
 
 /*
  * moe_layer_forward -- the whole hot path in one call: moe_route_topk,
@@ -312,17 +352,27 @@ moe_status moe_combine(const void* y, moe_dtype y_dtype, const int32_t* slot_of_
  *   b holds every intermediate buffer and workspace (device, caller
  *   owned); b->xp is in payload_dtype (x_dtype or MOE_E4M3), b->y in
  *   y_dtype.
- *   capacity: -1 for the dropless layout (moe_dispatch_layout; the
- *   permuted buffers have T*k rows), or C >= 0 for fixed slabs of C rows
- *   per expert (moe_dispatch_layout_capacity; E*C rows, dropped pairs add
- *   nothing, b->n_dropped receives their number when not NULL).
+ *   opts (may be NULL: capacity -1, route_groups 0):
+ *     capacity: -1 for the dropless layout (moe_dispatch_layout; the
+ *     permuted buffers have T*k rows), or C >= 0 for fixed slabs of C rows
+ *     per expert (moe_dispatch_layout_capacity; E*C rows, dropped pairs
+ *     add nothing, b->n_dropped receives their number when not NULL);
+ *     route_groups, route_max_groups: 0 for plain routing (moe_route_topk),
+ *     or G and M for moe_route_topk_grouped.
  *   step_events: NULL, or 8 cudaEvent_t handles recorded on `stream` at:
  *   0 before routing, 1 after routing, 2 after the layout, 3 after the
- *   permute, 4 after the FP8 dequantisation inside the GEMM (the same point
- *   as 3 without an FP8 payload), 5 after the gate/up GEMM, 6 after the down
- *   GEMM, 7 after combine -- so that a caller can time each kernel on the
- *   stream it runs on, without launch gaps between them.
+ *   permute, 4 when the GEMM's bf16 operand is ready (inside this call an
+ *   FP8 permute writes it as well, so 4 follows 3 directly), 5 after the
+ *   gate/up GEMM, 6 after the down GEMM, 7 after combine -- so that a caller
+ *   can time each kernel on the stream it runs on, without launch gaps
+ *   between them.
  */
+typedef struct moe_layer_options {
+    int32_t capacity;          /* -1: dropless; C >= 0: fixed slabs of C rows per expert */
+    int32_t route_groups;      /* 0: plain top-k; G: group-limited routing over G groups */
+    int32_t route_max_groups;  /* M: groups each token may reach (with route_groups) */
+} moe_layer_options;
+
 typedef struct moe_layer_buffers {
     int32_t* topk_idx;       /* [T, k] */
     float* topk_w;           /* [T, k] */
@@ -337,6 +387,7 @@ typedef struct moe_layer_buffers {
     float* xp_scales;        /* [S, H/128] (FP8 payload only) */
     void* h;                 /* [S, I] in w_dtype */
     void* y;                 /* [S, H] in y_dtype */
+    float* y_scales;         /* [S, H/128] (FP8 y only) */
     void* gemm_workspace;    /* moe_grouped_gemm_workspace_bytes(S, ...) */
     size_t gemm_workspace_bytes;
     int32_t* dev_status;     /* int32, zero-initialised */
@@ -346,9 +397,9 @@ typedef struct moe_layer_buffers {
 moe_status moe_layer_forward(const float* logits, const void* x, moe_dtype x_dtype, int64_t T,
                              int32_t H, int32_t E, int32_t k, int32_t W, int32_t I,
                              const void* w13, const void* w2, moe_dtype w_dtype,
-                             moe_dtype payload_dtype, moe_dtype y_dtype, int32_t capacity,
-                             const moe_layer_buffers* b, void* out, void* const* step_events,
-                             void* stream);
+                             moe_dtype payload_dtype, moe_dtype y_dtype,
+                             const moe_layer_options* opts, const moe_layer_buffers* b, void* out,
+                             void* const* step_events, void* stream);
 
 /*
  * moe_layer_forward_host -- moe_layer_forward with the inputs and the
@@ -363,7 +414,7 @@ moe_status moe_layer_forward_host(const float* logits_host, const void* x_host, 
                                   moe_dtype x_dtype, int64_t T, int32_t H, int32_t E, int32_t k,
                                   int32_t W, int32_t I, const void* w13, const void* w2,
                                   moe_dtype w_dtype, moe_dtype payload_dtype, moe_dtype y_dtype,
-                                  int32_t capacity, const moe_layer_buffers* b,
+                                  const moe_layer_options* opts, const moe_layer_buffers* b,
                                   void* const* step_events, void* stream);
 
 /*

@@ -106,21 +106,24 @@ def test_permute_combine_gemm_reject_before_launch(lib):
     assert p(ctypes.c_void_p(4098), moe.MOE_BF16, 10, 128, 2, FAKE, FAKE, moe.MOE_BF16, None,
              None) == 1                                                                 # align
     c = lib.moe_combine
-    assert c(FAKE, moe.MOE_E4M3, FAKE, FAKE, 10, 2, 128, FAKE, moe.MOE_BF16, None) == 1
-    assert c(FAKE, moe.MOE_BF16, FAKE, FAKE, 10, 0, 128, FAKE, moe.MOE_BF16, None) == 1
-    assert c(FAKE, moe.MOE_BF16, FAKE, FAKE, 10, 17, 128, FAKE, moe.MOE_BF16, None) == 2
+    assert c(FAKE, moe.MOE_E4M3, None, FAKE, FAKE, 10, 2, 128, FAKE, moe.MOE_BF16, None) == 1  # scales
+    assert c(FAKE, moe.MOE_E4M3, FAKE, FAKE, FAKE, 10, 2, 136, FAKE, moe.MOE_BF16, None) == 1  # H%128
+    assert c(FAKE, moe.MOE_BF16, None, FAKE, FAKE, 10, 0, 128, FAKE, moe.MOE_BF16, None) == 1
+    assert c(FAKE, moe.MOE_BF16, None, FAKE, FAKE, 10, 17, 128, FAKE, moe.MOE_BF16, None) == 2
     g = lib.moe_grouped_gemm
     base = [FAKE, moe.MOE_BF16, None, FAKE, None, 0, 8, 100, 256, 64, FAKE, FAKE, moe.MOE_BF16,
-            FAKE, FAKE, moe.MOE_F32, None, 0, FAKE, None]
+            FAKE, FAKE, moe.MOE_F32, None, None, 0, FAKE, None]
     bad = list(base); bad[9] = 60                      # I % 8
     assert g(*bad) == 1
     bad = list(base); bad[1] = moe.MOE_F32             # f32 payload with bf16 weights
     assert g(*bad) == 1
     bad = list(base); bad[1] = moe.MOE_E4M3            # FP8 payload needs scales
     assert g(*bad) == 1
-    bad = list(base); bad[18] = None                   # status word
+    bad = list(base); bad[19] = None                   # status word
     assert g(*bad) == 1
-    bad = list(base); bad[15] = moe.MOE_E4M3           # y storage must be fp32 or bf16
+    bad = list(base); bad[15] = moe.MOE_E4M3           # FP8 y needs its block scales
+    assert g(*bad) == 1
+    bad = list(base); bad[15] = moe.MOE_E4M3; bad[16] = FAKE; bad[8] = 200   # and H % 128
     assert g(*bad) == 1
     bad = list(base); bad[1] = moe.MOE_F32; bad[12] = moe.MOE_F32; bad[15] = moe.MOE_BF16
     assert g(*bad) == 1                                # fp32 GEMM stores y in fp32
@@ -142,11 +145,28 @@ def test_layer_call_rejects_before_launch(lib):
     f = lib.moe_layer_forward
     # no buffer struct
     assert f(FAKE, FAKE, moe.MOE_BF16, 10, 128, 8, 2, 2, 64, FAKE, FAKE, moe.MOE_BF16,
-             moe.MOE_BF16, moe.MOE_F32, -1, None, FAKE, None, None) == 1
-    cb = moe.LayerBuffersC(*([FAKE] * 8 + [0] + [FAKE] * 5 + [0] + [FAKE, None]))
+             moe.MOE_BF16, moe.MOE_F32, None, None, FAKE, None, None) == 1
+    cb = moe.LayerBuffersC(*([FAKE] * 8 + [0] + [FAKE] * 6 + [0] + [FAKE, None]))
     # E % W != 0 is caught before anything runs (workspace size 0 too)
     assert f(FAKE, FAKE, moe.MOE_BF16, 10, 128, 8, 2, 3, 64, FAKE, FAKE, moe.MOE_BF16,
-             moe.MOE_BF16, moe.MOE_F32, -1, ctypes.byref(cb), FAKE, None, None) == 1
+             moe.MOE_BF16, moe.MOE_F32, None, ctypes.byref(cb), FAKE, None, None) == 1
     # a capacity whose E * C rows do not fit int32
+    big = moe.LayerOptionsC(1 << 28, 0, 0)
     assert f(FAKE, FAKE, moe.MOE_BF16, 10, 128, 8, 2, 2, 64, FAKE, FAKE, moe.MOE_BF16,
-             moe.MOE_BF16, moe.MOE_F32, 1 << 28, ctypes.byref(cb), FAKE, None, None) == 2
+             moe.MOE_BF16, moe.MOE_F32, ctypes.byref(big), ctypes.byref(cb), FAKE, None,
+             None) == 2
+    # group-limited routing that cannot give k picks (2 groups of 4, 1 kept, k = 5)
+    grp = moe.LayerOptionsC(-1, 2, 1)
+    assert f(FAKE, FAKE, moe.MOE_BF16, 10, 128, 8, 5, 2, 64, FAKE, FAKE, moe.MOE_BF16,
+             moe.MOE_BF16, moe.MOE_F32, ctypes.byref(grp), ctypes.byref(cb), FAKE, None,
+             None) == 1
+
+
+def test_grouped_route_rejects_before_launch(lib):
+    f = lib.moe_route_topk_grouped
+    assert f(FAKE, 10, 8, 2, 3, 1, FAKE, FAKE, None) == 1      # groups must divide E
+    assert f(FAKE, 10, 8, 5, 4, 2, FAKE, FAKE, None) == 1      # 2 groups of 2: < 5 experts
+    assert f(FAKE, 10, 8, 2, 4, 5, FAKE, FAKE, None) == 1      # more kept groups than groups
+    assert f(FAKE, 10, 8, 2, 4, 0, FAKE, FAKE, None) == 1
+    assert f(FAKE, 10, 128, 2, 64, 4, FAKE, FAKE, None) == 2   # more than 32 groups
+    assert f(None, 0, 8, 2, 4, 2, None, None, None) == 0       # empty batch: no-op

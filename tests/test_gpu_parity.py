@@ -22,12 +22,16 @@ from parity_helpers import (BF16_TOL, F32_TOL, GpuLayer, bits, h_ok, oracle_gemm
 SMALL = ["tiny", "small_f32", "small_bf16", "small_fp8", "small_fp8v", "ragged_bf16", "pair_bf16",
          "pair_fp8"]
 FULL = {"decode": 64, "mid": 192, "skew": 128, "dsv3": 96,    # name -> sampled tokens
-        "dsv3_cap": 96, "skew_cap": 128}
+        "dsv3_cap": 96, "skew_cap": 128, "dsv3_grouped": 96}
 
 
 def _check_route_layout(wl, g: GpuLayer):
     b = g.buf
-    idx_o, w_o = oracle.route_topk(g.inputs["logits"], wl.k)
+    if wl.route_groups:
+        idx_o, w_o = oracle.route_topk_grouped(g.inputs["logits"], wl.k, wl.route_groups,
+                                               wl.route_max_groups)
+    else:
+        idx_o, w_o = oracle.route_topk(g.inputs["logits"], wl.k)
     assert torch.equal(b.topk_idx.cpu(), idx_o), "topk_idx differs"
     wg = b.topk_w.cpu().double()
     assert bool(((wg - w_o.double()).abs() <= 1e-5 * w_o.double().abs()).all()), "topk_w"
