@@ -239,7 +239,8 @@ def combine(y: torch.Tensor, slot_of_pair: torch.Tensor, topk_w: torch.Tensor,
 
 def quantize_rows_e4m3(v: torch.Tensor):
     """Per-128 block FP8 e4m3 quantisation of rows of fp32 values (the
-    dispatch payload's rule): returns (codes as float8_e4m3fn, fp32 scales)."""
+    combine payload's rule: scale = amax / 448, codes e4m3(v * (1 / scale)));
+    returns (codes as float8_e4m3fn, fp32 scales)."""
     v = v.to(torch.float32).contiguous()
     rows, H = v.shape
     q = torch.empty(rows, H, dtype=torch.uint8)

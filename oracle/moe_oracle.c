@@ -442,11 +442,14 @@ int64_t oracle_grouped_gemm(const void* xp, int xp_dt, const float* xp_scales,
 /* ------------------------------------------------------------------ */
 /* "Expert parallelism and all-to-all", "Traffic math": the figure of
  * 2 * k * H * bytes per token assumes 1-byte activations both ways, i.e.
- * the experts' outputs also travel back as FP8.  Reading: each y row is
- * quantised exactly like the dispatch payload (per 128-element block of
- * the fp32 value: scale = amax / 448 by fp32 IEEE division, 1 when amax is
- * 0; q = e4m3(y / scale), fp32 IEEE division, round-to-nearest-even,
- * saturating), and the combine uses decode(q) * scale as an fp32 product.
+ * the experts' outputs also travel back as FP8.  Reading: per 128-element
+ * block of each y row's fp32 values, scale = amax / 448 (fp32 IEEE
+ * division; 1 when amax is 0) as for the dispatch payload, and q =
+ * e4m3(y * r) with r = 1 / scale (one fp32 IEEE division per block, then an
+ * fp32 product per element; round-to-nearest-even, saturating): the
+ * combine payload has as many elements as the GEMM's outputs, so the
+ * per-element IEEE division of the dispatch payload is replaced by a
+ * product.  The combine uses decode(q) * scale as an fp32 product.
  * oracle_quantize_rows_e4m3 quantises rows of fp32 values; the caller
  * passes fp32(y). */
 int oracle_quantize_rows_e4m3(const float* v, int64_t rows, int32_t H, uint8_t* q,
@@ -462,7 +465,8 @@ int oracle_quantize_rows_e4m3(const float* v, int64_t rows, int32_t H, uint8_t* 
             float scale = amax / 448.0f;
             if (scale == 0.0f) scale = 1.0f;
             scales[r * nb + b] = scale;
-            for (int32_t i = 0; i < 128; ++i) q[r * H + b * 128 + i] = e4m3_from_float(blk[i] / scale);
+            const float rs = 1.0f / scale;
+            for (int32_t i = 0; i < 128; ++i) q[r * H + b * 128 + i] = e4m3_from_float(blk[i] * rs);
         }
     }
     return 0;

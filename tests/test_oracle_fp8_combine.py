@@ -1,5 +1,6 @@
 """Pins of the oracle's FP8 combine payload: per-128 block e4m3 quantisation
-of y (the dispatch payload's rule) and the combine that dequantises it.
+of y (scale = amax / 448, codes e4m3(y * (1 / scale))) and the combine that
+dequantises it.
 
 Source: "Expert parallelism and all-to-all", "Traffic math": 1-byte
 activations both ways (dispatch and combine).
@@ -20,7 +21,8 @@ def test_codes_equal_torch_e4m3_of_the_scaled_values():
     q, sc = oracle.quantize_rows_e4m3(v)
     amax = v.abs().view(64, 4, 128).amax(dim=2)
     assert torch.equal(sc, amax / 448.0)                    # fp32 IEEE division
-    scaled = v / sc.repeat_interleave(128, dim=1)           # every |value| <= 448 (+ rounding)
+    recip = 1.0 / sc                                        # one IEEE division per block
+    scaled = v * recip.repeat_interleave(128, dim=1)        # every |value| <= 448 (+ rounding)
     ref = scaled.clamp(-448, 448).to(torch.float8_e4m3fn)   # torch: round to nearest even
     assert torch.equal(q.view(torch.uint8), ref.view(torch.uint8))
 
