@@ -363,6 +363,9 @@ def run_ours(args, wl):
             e2e_ms.append(e0.elapsed_time(e1))
     e2e = statistics.mean(e2e_ms)
     (e2e,) = max_over_ranks([e2e], dev)
+    # the permute alone (moe_permute: the send buffer only, as a standalone
+    # call), L2 flushed before each launch
+    perm_alone_us = _permute_alone_us(wl, x, buf, 10)
     # the whole layer captured once in a CUDA graph and replayed: median
     # device time per replay (launch overhead of the separate calls removed)
     graph_us, replays = _graph_replay_us(wl, logits, x, w13, w2, buf, 100 if wl.T <= 1024 else 20)
@@ -389,7 +392,12 @@ def run_ours(args, wl):
                            "gbs": gbs(kb["route_topk"], avg["route_topk"])},
             "dispatch_layout": {"us": avg["dispatch_layout"] * 1e3},
             "permute": {"us": avg["permute"] * 1e3, "bytes": kb["permute_layer"],
-                        "gbs": gbs(kb["permute_layer"], avg["permute"])},
+                        "gbs": gbs(kb["permute_layer"], avg["permute"]),
+                        "note": "inside the layer call an FP8 permute also writes the GEMM's "
+                                "bf16 rows" if wl.payload == "e4m3" else "send buffer only"},
+            "permute_standalone": {"us": perm_alone_us, "bytes": kb["permute"],
+                                   "gbs": gbs(kb["permute"], perm_alone_us * 1e-3),
+                                   "l2": "flushed before each launch"},
             "grouped_gemm": {"us": gemm_ms * 1e3, "flops": fl["total"],
                              "tflops": tf(fl["total"], gemm_ms),
                              "dequant_e4m3_us": avg["dequant_e4m3"] * 1e3,
@@ -402,7 +410,7 @@ def run_ours(args, wl):
             "combine": {"us": avg["combine"] * 1e3, "bytes": kb["combine"],
                         "gbs": gbs(kb["combine"], avg["combine"])},
         }
-        for n in ["permute", "combine", "route_topk"]:
+        for n in ["permute", "permute_standalone", "combine", "route_topk"]:
             kernels[n]["hbm_frac"] = kernels[n]["gbs"] / peaks["hbm_gbs"]
         # the dominant kernel: the gate/up grouped GEMM (SwiGLU fused)
         achieved = tf(fl["gate_up"], avg["gemm_gate_up"])
@@ -438,6 +446,25 @@ def run_ours(args, wl):
     if ws > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
+
+
+def _permute_alone_us(wl, x, buf, iters):
+    """Mean device time of moe_permute on the step's routing (its send
+    buffer, payload dtype of the workload), with a 512 MiB write before each
+    launch so x starts outside L2."""
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=x.device)
+    ts = []
+    for i in range(iters + 2):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        moe.moe_permute(x, wl.k, buf.slot_of_pair, buf.xp, buf.xp_scales)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= 2:
+            ts.append(e0.elapsed_time(e1) * 1e3)
+    del flush
+    return statistics.mean(ts)
 
 
 def _graph_replay_us(wl, logits, x, w13, w2, buf, replays):

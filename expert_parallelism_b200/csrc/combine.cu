@@ -46,29 +46,53 @@ __device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&f)[8]) {
                         pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7])));
 }
 
-// Piece c (8 elements) of row s of y as fp32.
+// One thread's piece of a y row: load() issues its global loads (all picks'
+// loads are issued before any sum), add() folds w * piece into the fp32
+// accumulators in element order.  fp32 / bf16 y: 8 elements (16 bytes),
+// converted at load.  e4m3 y: 16 codes (16 bytes) and the block's scale,
+// kept raw until add() (decode(q) * scale, an fp32 product), so four picks
+// in flight hold 4 x 5 registers instead of 4 x 16.
 template <typename TY>
-__device__ __forceinline__ void load_piece(const TY* y, const float* y_scales, int64_t s, int H,
-                                           int c, float (&f)[8]) {
-    (void)y_scales;
-    load8_row(y + s * H + c * 8, f);
-}
-template <>
-__device__ __forceinline__ void load_piece<uint8_t>(const uint8_t* y, const float* y_scales,
-                                                    int64_t s, int H, int c, float (&f)[8]) {
-    const uint2 q = ld_nc_v2(y + s * H + c * 8);
-    const float sc = __ldg(y_scales + s * (H / 128) + (c * 8) / 128);
-    const uint32_t w[2] = {q.x, q.y};
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const float2 a = decode2_e4m3((uint16_t)(w[i] & 0xFFFFu));
-        const float2 b = decode2_e4m3((uint16_t)(w[i] >> 16));
-        f[4 * i + 0] = a.x * sc;
-        f[4 * i + 1] = a.y * sc;
-        f[4 * i + 2] = b.x * sc;
-        f[4 * i + 3] = b.y * sc;
+struct Piece {
+    static constexpr int N = 8;
+    struct Raw {
+        float f[8];
+    };
+    static __device__ __forceinline__ void load(const TY* y, const float*, int64_t s, int H, int c,
+                                                Raw& r) {
+        load8_row(y + s * H + c * 8, r.f);
     }
-}
+    static __device__ __forceinline__ void add(float (&acc)[8], const Raw& r, float w) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = fmaf(w, r.f[i], acc[i]);
+    }
+};
+
+template <>
+struct Piece<uint8_t> {
+    static constexpr int N = 16;
+    struct Raw {
+        uint4 q;
+        float sc;
+    };
+    static __device__ __forceinline__ void load(const uint8_t* y, const float* y_scales, int64_t s,
+                                                int H, int c, Raw& r) {
+        r.q = ld_nc_v4(y + s * H + c * 16);
+        r.sc = __ldg(y_scales + s * (H / 128) + (c * 16) / 128);
+    }
+    static __device__ __forceinline__ void add(float (&acc)[16], const Raw& r, float w) {
+        const uint32_t q[4] = {r.q.x, r.q.y, r.q.z, r.q.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 a = decode2_e4m3((uint16_t)(q[i] & 0xFFFFu));
+            const float2 b = decode2_e4m3((uint16_t)(q[i] >> 16));
+            acc[4 * i + 0] = fmaf(w, __fmul_rn(a.x, r.sc), acc[4 * i + 0]);
+            acc[4 * i + 1] = fmaf(w, __fmul_rn(a.y, r.sc), acc[4 * i + 1]);
+            acc[4 * i + 2] = fmaf(w, __fmul_rn(b.x, r.sc), acc[4 * i + 2]);
+            acc[4 * i + 3] = fmaf(w, __fmul_rn(b.y, r.sc), acc[4 * i + 3]);
+        }
+    }
+};
 
 template <typename TY, typename TO>
 __global__ void __launch_bounds__(256) combine_kernel(const TY* __restrict__ y,
@@ -76,9 +100,11 @@ __global__ void __launch_bounds__(256) combine_kernel(const TY* __restrict__ y,
                                                       const int32_t* __restrict__ slot_of_pair,
                                                       const float* __restrict__ topk_w, int64_t T,
                                                       int k, int H, TO* __restrict__ out) {
+    using P = Piece<TY>;
+    constexpr int EPT = P::N;
     __shared__ int32_t s_slot[kCombineMaxTopK];
     __shared__ float s_w[kCombineMaxTopK];
-    const int nchunk = H / 8;
+    const int nchunk = H / EPT;
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
         if (threadIdx.x < k) {
             s_slot[threadIdx.x] = slot_of_pair[t * k + threadIdx.x];
@@ -86,36 +112,32 @@ __global__ void __launch_bounds__(256) combine_kernel(const TY* __restrict__ y,
         }
         __syncthreads();
         for (int c = threadIdx.x; c < nchunk; c += blockDim.x) {
-            float acc[8];
+            float acc[EPT];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+            for (int i = 0; i < EPT; ++i) acc[i] = 0.0f;
             int j = 0;
             // four picks at a time: their loads are in flight together
             for (; j + 4 <= k; j += 4) {
-                float v[4][8];
+                typename P::Raw v[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const int32_t s = s_slot[j + u];
-                    if (s >= 0) load_piece(y, y_scales, s, H, c, v[u]);
+                    if (s >= 0) P::load(y, y_scales, s, H, c, v[u]);
                 }
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    if (s_slot[j + u] < 0) continue;
-                    const float w = s_w[j + u];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) acc[i] = fmaf(w, v[u][i], acc[i]);
-                }
+                for (int u = 0; u < 4; ++u)
+                    if (s_slot[j + u] >= 0) P::add(acc, v[u], s_w[j + u]);
             }
             for (; j < k; ++j) {
                 const int32_t s = s_slot[j];
                 if (s < 0) continue;
-                float v[8];
-                load_piece(y, y_scales, s, H, c, v);
-                const float w = s_w[j];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = fmaf(w, v[i], acc[i]);
+                typename P::Raw v;
+                P::load(y, y_scales, s, H, c, v);
+                P::add(acc, v, s_w[j]);
             }
-            store8(out + t * H + c * 8, acc);
+#pragma unroll
+            for (int h = 0; h < EPT / 8; ++h)
+                store8(out + t * H + c * EPT + 8 * h, *reinterpret_cast<float(*)[8]>(acc + 8 * h));
         }
         __syncthreads();
     }
@@ -130,7 +152,8 @@ cudaError_t launch_combine(const void* y, moe_dtype ydt, const float* y_scales,
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t cap = (int64_t)sms * 8;
     const unsigned grid = (unsigned)(T < cap ? T : cap);
-    int threads = ((H / 8 + 31) / 32) * 32;
+    const int ept = ydt == MOE_E4M3 ? 16 : 8;
+    int threads = ((H / ept + 31) / 32) * 32;
     threads = threads < 32 ? 32 : (threads > 256 ? 256 : threads);
 #define MOE_COMBINE(TY, TO)                                                               \
     combine_kernel<TY, TO><<<grid, threads, 0, s>>>((const TY*)y, y_scales, slot_of_pair, \

@@ -106,6 +106,17 @@ __device__ __forceinline__ uint32_t quant4_e4m3(float a, float b, float c, float
     return (uint32_t)lo | ((uint32_t)hi << 16);
 }
 
+// The FP8 combine payload's encoding: four e4m3 codes of a * r .. d * r,
+// r = 1 / scale (fp32 products, then the round-to-nearest-even,
+// saturating conversion), packed low byte first.
+__device__ __forceinline__ uint32_t quant4_e4m3_mul(float a, float b, float c, float d, float r) {
+    const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
+        make_float2(__fmul_rn(a, r), __fmul_rn(b, r)), __NV_SATFINITE, __NV_E4M3);
+    const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+        make_float2(__fmul_rn(c, r), __fmul_rn(d, r)), __NV_SATFINITE, __NV_E4M3);
+    return (uint32_t)lo | ((uint32_t)hi << 16);
+}
+
 // Two e4m3 codes (low byte first) decoded to fp32 (exact: e4m3 values are
 // fp16 values).
 __device__ __forceinline__ float2 decode2_e4m3(uint16_t two) {

@@ -33,9 +33,9 @@
 // 1 stages, per CTA, 64 gate rows and the 64 matching up rows, so lanes
 // 0..63 hold gate and 64..127 up for the same 64 features; the epilogue
 // pairs them through shared memory.  Phase 2 stages 128 rows of W2 per CTA;
-// its output y is fp32, bf16, or the FP8 combine payload: e4m3 codes with one
-// fp32 scale per 128 features ("Expert parallelism and all-to-all", "Traffic
-// math": 1-byte activations both ways).  A CTA's 128 weight rows are exactly
+// its output y is fp32, bf16, or the FP8 combine payload: e4m3 codes of
+// y * (1/scale) with one fp32 scale (amax / 448) per 128 features ("Expert
+// parallelism and all-to-all", "Traffic math": 1-byte activations both ways).  A CTA's 128 weight rows are exactly
 // one such block, so each block's amax is a max over one epilogue group's
 // four warps.
 //
@@ -437,20 +437,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float amax = fmaxf(fmaxf(amax_buf[lane], amax_buf[32 + lane]),
                                                  fmaxf(amax_buf[64 + lane], amax_buf[96 + lane]));
                         const float scale = e4m3_block_scale(amax);
+                        const float rs = __frcp_rn(scale);       // codes: e4m3(y * (1/scale))
                         const int64_t row = crow0 + col + lane;
                         const int blk0 = ti.wt * 2 * kWRows + (int)rank * kWRows;   // block start
                         if (row < row_end && blk0 < p.n_out) {
                             uint8_t* dst =
                                 reinterpret_cast<uint8_t*>(out) + row * p.n_out + blk0 + quarter * 32;
-                            st_v4(dst, make_uint4(quant4_e4m3(rv[0], rv[1], rv[2], rv[3], scale),
-                                                  quant4_e4m3(rv[4], rv[5], rv[6], rv[7], scale),
-                                                  quant4_e4m3(rv[8], rv[9], rv[10], rv[11], scale),
-                                                  quant4_e4m3(rv[12], rv[13], rv[14], rv[15], scale)));
+                            st_v4(dst, make_uint4(quant4_e4m3_mul(rv[0], rv[1], rv[2], rv[3], rs),
+                                                  quant4_e4m3_mul(rv[4], rv[5], rv[6], rv[7], rs),
+                                                  quant4_e4m3_mul(rv[8], rv[9], rv[10], rv[11], rs),
+                                                  quant4_e4m3_mul(rv[12], rv[13], rv[14], rv[15], rs)));
                             st_v4(dst + 16,
-                                  make_uint4(quant4_e4m3(rv[16], rv[17], rv[18], rv[19], scale),
-                                             quant4_e4m3(rv[20], rv[21], rv[22], rv[23], scale),
-                                             quant4_e4m3(rv[24], rv[25], rv[26], rv[27], scale),
-                                             quant4_e4m3(rv[28], rv[29], rv[30], rv[31], scale)));
+                                  make_uint4(quant4_e4m3_mul(rv[16], rv[17], rv[18], rv[19], rs),
+                                             quant4_e4m3_mul(rv[20], rv[21], rv[22], rv[23], rs),
+                                             quant4_e4m3_mul(rv[24], rv[25], rv[26], rv[27], rs),
+                                             quant4_e4m3_mul(rv[28], rv[29], rv[30], rv[31], rs)));
                             if (quarter == 0) p.out_scales[row * (p.n_out / 128) + blk0 / 128] = scale;
                         }
                         ++piece;
