@@ -281,6 +281,7 @@ def _config(wl):
             **({"capacity_factor": wl.capacity_factor} if wl.capacity_factor is not None else {}),
             **({"route_groups": wl.route_groups, "route_max_groups": wl.route_max_groups}
                if wl.route_groups else {}),
+            "fused_gather": wl.fused_gather,
             "parallelism": "replicas (one independent layer per GPU)"}
 
 
@@ -386,15 +387,17 @@ def run_ours(args, wl):
         counts = buf.expert_counts.cpu()
         touched = int((counts > 0).sum())
         tf = lambda flops, ms: flops / (ms * 1e-3) / 1e12
-        gbs = lambda b, ms: b / (ms * 1e-3) / 1e9
+        gbs = lambda b, ms: b / (ms * 1e-3) / 1e9 if b and ms > 0 else None
         kernels = {
             "route_topk": {"us": avg["route_topk"] * 1e3,
                            "gbs": gbs(kb["route_topk"], avg["route_topk"])},
             "dispatch_layout": {"us": avg["dispatch_layout"] * 1e3},
             "permute": {"us": avg["permute"] * 1e3, "bytes": kb["permute_layer"],
                         "gbs": gbs(kb["permute_layer"], avg["permute"]),
-                        "note": "inside the layer call an FP8 permute also writes the GEMM's "
-                                "bf16 rows" if wl.payload == "e4m3" else "send buffer only"},
+                        "note": ("fused gather: one bf16 round trip per token (FP8 payload), "
+                                 "no permuted copy" if wl.fused_gather else
+                                 "inside the layer call an FP8 permute also writes the GEMM's "
+                                 "bf16 rows" if wl.payload == "e4m3" else "send buffer only")},
             "permute_standalone": {"us": perm_alone_us, "bytes": kb["permute"],
                                    "gbs": gbs(kb["permute"], perm_alone_us * 1e-3),
                                    "l2": "flushed before each launch"},
@@ -411,7 +414,8 @@ def run_ours(args, wl):
                         "gbs": gbs(kb["combine"], avg["combine"])},
         }
         for n in ["permute", "permute_standalone", "combine", "route_topk"]:
-            kernels[n]["hbm_frac"] = kernels[n]["gbs"] / peaks["hbm_gbs"]
+            g = kernels[n]["gbs"]
+            kernels[n]["hbm_frac"] = g / peaks["hbm_gbs"] if g is not None else None
         # the dominant kernel: the gate/up grouped GEMM (SwiGLU fused)
         achieved = tf(fl["gate_up"], avg["gemm_gate_up"])
         # timed inside a long run of back-to-back steps under the 1000 W cap:

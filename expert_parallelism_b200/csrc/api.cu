@@ -29,8 +29,11 @@ cudaError_t launch_grouped_gemm_simt_f32(const float*, const int32_t*, const int
                                          float*, cudaEvent_t, cudaStream_t);
 cudaError_t launch_grouped_gemm_tc(const __nv_bfloat16*, const int32_t*, const int32_t*, int, int,
                                    int64_t, int, int, const __nv_bfloat16*, const __nv_bfloat16*,
-                                   __nv_bfloat16*, void*, moe_dtype, float*, int32_t*, cudaEvent_t,
-                                   cudaStream_t);
+                                   __nv_bfloat16*, void*, moe_dtype, float*, int32_t*,
+                                   const gemm_gather*, cudaEvent_t, cudaStream_t);
+bool grouped_gemm_tc_uses_swap(int64_t n_rows, int n_experts, moe_dtype y_dtype);
+cudaError_t launch_quantize_tokens_e4m3(const void*, moe_dtype, int64_t, int, __nv_bfloat16*,
+                                       cudaStream_t);
 }  // namespace moe
 
 namespace moe {
@@ -155,7 +158,8 @@ moe_status check_combine(const void* y, moe_dtype y_dtype, const float* y_scales
 }
 
 // ev_a (after the FP8 dequantisation, or at the start) and ev_b (between
-// the two GEMM phases) may be null.
+// the two GEMM phases) may be null.  g (bf16 weights, operand-swapped
+// kernel only): the gate/up rows are gathered from g->src; xp is not read.
 cudaError_t run_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_scales,
                      const int32_t* expert_offsets, const int32_t* expert_counts,
                      int32_t expert_begin, int32_t n_experts,
@@ -163,7 +167,7 @@ cudaError_t run_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_scales,
                      moe_dtype w_dtype, void* h, void* y, moe_dtype y_dtype, float* y_scales,
                      void* workspace, int32_t* dev_status, cudaStream_t s,
                      cudaEvent_t ev_a = nullptr, cudaEvent_t ev_b = nullptr,
-                     bool a_ready = false) {
+                     bool a_ready = false, const gemm_gather* g = nullptr) {
     cudaError_t e = cudaSuccess;
     if (w_dtype == MOE_F32) {
         if (ev_a) e = cudaEventRecord(ev_a, s);
@@ -174,7 +178,7 @@ cudaError_t run_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_scales,
                                             (float*)y, ev_b, s);
     }
     const __nv_bfloat16* a = (const __nv_bfloat16*)xp;
-    if (xp_dtype == MOE_E4M3) {
+    if (xp_dtype == MOE_E4M3 && !g) {
         // the FP8 rows' bf16 operand, unless the permute already wrote it
         if (!a_ready)
             e = launch_dequant_e4m3((const uint8_t*)xp, xp_scales, expert_offsets, expert_begin,
@@ -187,7 +191,8 @@ cudaError_t run_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_scales,
     return launch_grouped_gemm_tc(a, expert_offsets, expert_counts, expert_begin, n_experts,
                                   n_rows, H, I,
                                   (const __nv_bfloat16*)w13, (const __nv_bfloat16*)w2,
-                                  (__nv_bfloat16*)h, y, y_dtype, y_scales, dev_status, ev_b, s);
+                                  (__nv_bfloat16*)h, y, y_dtype, y_scales, dev_status, g, ev_b,
+                                  s);
 }
 
 }  // namespace
@@ -307,7 +312,7 @@ static int64_t layer_slots(int64_t T, int32_t k, int32_t E, int32_t capacity) {
 }
 
 static moe_layer_options resolve(const moe_layer_options* o) {
-    return o ? *o : moe_layer_options{-1, 0, 0};
+    return o ? *o : moe_layer_options{-1, 0, 0, 0};
 }
 
 static moe_status check_layer(const float* logits, const void* x, moe_dtype x_dtype, int64_t T,
@@ -339,6 +344,11 @@ static moe_status check_layer(const float* logits, const void* x, moe_dtype x_dt
     if (st == MOE_OK)
         st = check_combine(b->y, y_dtype, b->y_scales, b->slot_of_pair, b->topk_w, T, k, H, out,
                            x_dtype, &noop);
+    // the fused gather's FP8 source, one bf16 row per token, lives in the
+    // GEMM workspace
+    if (st == MOE_OK && o.fused_gather != 0 && payload_dtype == MOE_E4M3 && T > 0 &&
+        (b->gemm_workspace_bytes < (size_t)T * H * 2 || !b->gemm_workspace))
+        st = MOE_ERR_INVALID_ARG;
     return st;
 }
 
@@ -350,6 +360,14 @@ static cudaError_t launch_layer(const float* logits, const void* x, moe_dtype x_
                                 void* const* ev, cudaStream_t s) {
     const int32_t capacity = o.capacity;
     const int64_t n_slots = layer_slots(T, k, E, capacity);
+    // Fused gather: the gate/up GEMM reads each routed row from a token-major
+    // source (x itself for a bf16 payload; each token's FP8 round trip,
+    // bf16(decode(q) * scale), for an FP8 payload) instead of a permuted copy.
+    const bool gather = o.fused_gather != 0 && w_dtype == MOE_BF16 && n_slots > 0 &&
+                        grouped_gemm_tc_uses_swap(n_slots, E, y_dtype);
+    const gemm_gather gsrc{payload_dtype == MOE_E4M3 ? (const __nv_bfloat16*)b->gemm_workspace
+                                                     : (const __nv_bfloat16*)x,
+                           b->pair_of_slot, k};
     auto mark = [&](int i) {
         return ev ? cudaEventRecord((cudaEvent_t)ev[i], s) : cudaSuccess;
     };
@@ -365,7 +383,9 @@ static cudaError_t launch_layer(const float* logits, const void* x, moe_dtype x_
                                    capacity < 0 ? nullptr : b->n_dropped, b->layout_workspace,
                                    b->dev_status, s);
     if (e == cudaSuccess) e = mark(2);
-    if (e == cudaSuccess && T > 0)
+    if (e == cudaSuccess && T > 0 && gather && payload_dtype == MOE_E4M3)
+        e = launch_quantize_tokens_e4m3(x, x_dtype, T, H, (__nv_bfloat16*)b->gemm_workspace, s);
+    else if (e == cudaSuccess && T > 0 && !gather)
         e = launch_permute(x, x_dtype, T, H, k, b->slot_of_pair, b->xp, payload_dtype,
                            b->xp_scales,
                            payload_dtype == MOE_E4M3 ? (__nv_bfloat16*)b->gemm_workspace : nullptr,
@@ -376,7 +396,7 @@ static cudaError_t launch_layer(const float* logits, const void* x, moe_dtype x_
                      capacity < 0 ? nullptr : b->expert_counts, 0, E, n_slots, H, I, w13, w2,
                      w_dtype, b->h, b->y, y_dtype, b->y_scales, b->gemm_workspace, b->dev_status,
                      s, ev ? (cudaEvent_t)ev[4] : nullptr, ev ? (cudaEvent_t)ev[5] : nullptr,
-                     /*a_ready=*/true);
+                     /*a_ready=*/true, gather ? &gsrc : nullptr);
     } else if (e == cudaSuccess) {
         e = mark(4);
         if (e == cudaSuccess) e = mark(5);

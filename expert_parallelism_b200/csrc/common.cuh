@@ -126,6 +126,15 @@ __device__ __forceinline__ float2 decode2_e4m3(uint16_t two) {
 
 inline int ceil_div(int64_t a, int64_t b) { return (int)((a + b - 1) / b); }
 
+// Source of the grouped GEMM's fused gather: row s of the gate/up operand
+// is row pair_of_slot[s] / top_k of src (token-major, bf16); a slot holding
+// no pair (-1) reads zeros.
+struct gemm_gather {
+    const __nv_bfloat16* src;
+    const int32_t* pair_of_slot;
+    int top_k;
+};
+
 // Host-side count of kernel launches (reported by moe_launch_count).
 void note_launches(int n);
 

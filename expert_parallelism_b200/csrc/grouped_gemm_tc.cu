@@ -505,7 +505,7 @@ cudaError_t launch_grouped_gemm_tc_swap(const __nv_bfloat16* a, const int32_t* o
                                         int64_t n_rows, int H, int I, const __nv_bfloat16* w13,
                                         const __nv_bfloat16* w2, __nv_bfloat16* h, void* y,
                                         moe_dtype y_dtype, float* y_scales, int32_t* dev_status,
-                                        cudaEvent_t ev_mid, cudaStream_t s);
+                                        const gemm_gather* g, cudaEvent_t ev_mid, cudaStream_t s);
 
 // Kernel choice, from the average rows per expert (known on the host
 // without reading the device offsets).  The operand-swapped pair kernel
@@ -519,22 +519,30 @@ static bool gemm_use_swap(int64_t n_rows, int n_experts) {
     return n_rows >= (int64_t)16 * n_experts;
 }
 
+// Whether launch_grouped_gemm_tc runs the operand-swapped kernel, the one
+// with the fused gather.
+bool grouped_gemm_tc_uses_swap(int64_t n_rows, int n_experts, moe_dtype y_dtype) {
+    return y_dtype == MOE_E4M3 || gemm_use_swap(n_rows, n_experts);
+}
+
 // A [n_rows, H] bf16 (the payload, or its dequantised copy); W13 [n_exp, 2I,
 // H]; W2 [n_exp, H, I]; h [n_rows, I] bf16; y [n_rows, H] in y_dtype: fp32,
 // bf16, or e4m3 codes with fp32 block scales y_scales [n_rows, H/128] (the
 // operand-swapped kernel only).  counts (may be null) cuts each expert's
-// segment to its first counts[j] rows.  ev_mid (may be null) is recorded
-// between the two phases.
+// segment to its first counts[j] rows.  g (may be null; the operand-swapped
+// kernel only): the gate/up operand's rows are gathered from g->src instead
+// of read from A.  ev_mid (may be null) is recorded between the two phases.
 cudaError_t launch_grouped_gemm_tc(const __nv_bfloat16* a, const int32_t* offsets,
                                    const int32_t* counts, int expert_begin, int n_experts,
                                    int64_t n_rows, int H, int I, const __nv_bfloat16* w13,
                                    const __nv_bfloat16* w2, __nv_bfloat16* h, void* y,
                                    moe_dtype y_dtype, float* y_scales, int32_t* dev_status,
-                                   cudaEvent_t ev_mid, cudaStream_t s) {
-    if (y_dtype == MOE_E4M3 || gemm_use_swap(n_rows, n_experts))
+                                   const gemm_gather* g, cudaEvent_t ev_mid, cudaStream_t s) {
+    if (grouped_gemm_tc_uses_swap(n_rows, n_experts, y_dtype))
         return launch_grouped_gemm_tc_swap(a, offsets, counts, expert_begin, n_experts, n_rows, H,
-                                           I, w13, w2, h, y, y_dtype, y_scales, dev_status, ev_mid,
-                                           s);
+                                           I, w13, w2, h, y, y_dtype, y_scales, dev_status, g,
+                                           ev_mid, s);
+    if (g) return cudaErrorInvalidValue;
     return tc::run_gemm<1>(a, offsets, counts, expert_begin, n_experts, n_rows, H, I, w13, w2, h,
                            y, y_dtype == MOE_F32, dev_status, ev_mid, s);
 }

@@ -79,6 +79,20 @@ constexpr int kStages = 5;
 constexpr int kSlotCols = 256;
 constexpr int kTmemCols = 2 * kSlotCols;
 
+// Fused gather (phase 1): the routed rows are read from a token-major
+// source through pair_of_slot by two teams of four warps per CTA that take
+// alternate k-steps; each thread owns one 16-byte piece (8 bf16) of ten of
+// the stage's 160 rows.
+constexpr int kGatherTeams = 2;
+constexpr int kTeamWarps = 4;
+constexpr int kGatherThreads = kGatherTeams * kTeamWarps * 32;
+constexpr int kGatherWarp0 = kThreads / 32;                      // warps 10..17
+constexpr int kGatherRows = kTRows * 8 / (kTeamWarps * 32);      // rows per thread per stage
+constexpr int kMaxThreads = kThreads + kGatherThreads;
+static_assert(kTRows * 8 % (kTeamWarps * 32) == 0, "gather pieces divide evenly");
+template <bool GATHER>
+constexpr int threads_of() { return GATHER ? kMaxThreads : kThreads; }
+
 // Epilogue staging.  Phase 1: per group, 128 lanes x 32 chunk rows as fp32,
 // row pitch 33 words (conflict-free both ways).  Phase 2: per warp 32 chunk
 // rows x 32 outputs as fp32, row pitch 36 words (16-byte aligned rows).
@@ -101,7 +115,7 @@ struct Smem {
     static constexpr int misc = bars + n_bars * 8;           // tmem addr, abort flag
     static constexpr int prefix = misc + 16;                 // int32 [MOE_MAX_EXPERTS + 1]
     static constexpr int warp_sums = prefix + (MOE_MAX_EXPERTS + 1) * 4;
-    static constexpr int epi = ((warp_sums + (kThreads / 32) * 4 + 127) / 128) * 128;
+    static constexpr int epi = ((warp_sums + (kMaxThreads / 32) * 4 + 127) / 128) * 128;
     static constexpr int amax = epi + kEpiBytes;
     static constexpr int total = amax + kAmaxBytes;
     static constexpr size_t alloc = total + 1024;            // + alignment slack
@@ -121,6 +135,11 @@ struct Params {
     void* out;                // h (phase 1, bf16) or y (phase 2, OutT), row stride n_out
     float* out_scales;        // y's block scales [n_rows, n_out / 128] when OutT is e4m3
     int32_t* dev_status;
+    // fused gather (phase 1 only): row s of A is row pair_of_slot[s] / top_k
+    // of gather_src [*, K] (zeros for a slot holding no pair)
+    const __nv_bfloat16* gather_src;
+    const int32_t* pair_of_slot;
+    int top_k;
 };
 
 // Passes an expert with `rows` routed rows takes.
@@ -200,8 +219,8 @@ __device__ __forceinline__ void load_rows(uint32_t dst, const CUtensorMap* m128,
     tma_load_2d<2>(dst, b == 128 ? m128 : b == 32 ? m32 : m8, bar, k0, r0);
 }
 
-template <bool GLU, typename OutT>
-__global__ void __launch_bounds__(kThreads, 1)
+template <bool GLU, typename OutT, bool GATHER>
+__global__ void __launch_bounds__(threads_of<GATHER>(), 1)
     grouped_gemm_swap_kernel(const __grid_constant__ CUtensorMap tmap_w,
                              const __grid_constant__ CUtensorMap tmap_t128,
                              const __grid_constant__ CUtensorMap tmap_t32,
@@ -226,7 +245,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(full_bar(s), 1);            // the leader's expect_tx (both CTAs' bytes)
+            // the leader's expect_tx (both CTAs' TMA bytes), and with the
+            // fused gather one arrival per gathering warp of both CTAs
+            mbar_init(full_bar(s), GATHER ? 1 + 2 * kTeamWarps : 1);
             mbar_init(empty_bar(s), 1);           // the leader's MMA commit
         }
         for (int b = 0; b < 2; ++b) {
@@ -271,7 +292,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const TileInfo ti = tile_info(p, s_prefix, t);
             const int h0 = ti.n0 >> 1, h1 = ti.n1 >> 1;       // rows this CTA multiplies per chunk
             const uint32_t tx =
-                2u * (uint32_t)(kWBytes + (box_rows(h0) + (h1 ? box_rows(h1) : 0)) * kRowBytes);
+                GATHER ? 2u * (uint32_t)kWBytes
+                       : 2u * (uint32_t)(kWBytes +
+                                         (box_rows(h0) + (h1 ? box_rows(h1) : 0)) * kRowBytes);
             for (int kb = 0; kb < nk; ++kb) {
                 if (!mbar_wait(empty_bar(stage), phase ^ 1u, s_abort, p.dev_status)) {
                     aborted = true;
@@ -287,9 +310,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_4d<2>(sw, &tmap_w, cfb, k0, w_row(ti), 0, ti.j);
                 else
                     tma_load_3d<2>(sw, &tmap_w, cfb, k0, w_row(ti), ti.j);
-                load_rows(st, &tmap_t128, &tmap_t32, &tmap_t8, cfb, k0, ti.row0 + (int)rank * h0,
-                          h0);
-                if (h1)
+                if (!GATHER)
+                    load_rows(st, &tmap_t128, &tmap_t32, &tmap_t8, cfb, k0,
+                              ti.row0 + (int)rank * h0, h0);
+                if (!GATHER && h1)
                     load_rows(st + kTailOff, &tmap_t128, &tmap_t32, &tmap_t8, cfb, k0,
                               ti.row0 + kMainN + (int)rank * h1, h1);
                 if (++stage == kStages) {
@@ -348,7 +372,73 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < ns; ++c) umma_commit<2>(tfull_bar((nslot + c) & 1));
             nslot += ns;
         }
-    } else if (warp >= 2) {
+    } else if (GATHER && warp >= kGatherWarp0) {
+        // ------------------------------------------------ row gather (both CTAs)
+        // Stage row q (q < 128: first chunk, q >= 128: second chunk) of this
+        // CTA is the routed row in slot row0 + rank * h0 + q (or row0 + 256
+        // + rank * h1 + q - 128); it is row pair_of_slot[slot] / top_k of the
+        // source.  Rows are written in the 128-byte-swizzled layout a TMA box
+        // would produce: 16-byte piece c of row q at q * 128 + ((c ^ (q % 8))
+        // * 16).  Rows past the pass (padding) are zeros.
+        const int gw = warp - kGatherWarp0;
+        const uint32_t team = (uint32_t)(gw / kTeamWarps);
+        const int lt = (gw % kTeamWarps) * 32 + lane;
+        const int piece = lt & 7;                  // 16-byte piece of each row
+        const int rb = lt >> 3;                    // rows rb, rb + 16, .., rb + 144
+        uint32_t g = 0;                            // k-steps so far, both teams
+        for (int t = unit; t < n_tiles && !aborted; t += n_units) {
+            const TileInfo ti = tile_info(p, s_prefix, t);
+            const int h0 = ti.n0 >> 1, h1 = ti.n1 >> 1;
+            const __nv_bfloat16* src[kGatherRows];
+            uint32_t need = 0;                     // bit m: row rb + 16 m is multiplied
+#pragma unroll
+            for (int m = 0; m < kGatherRows; ++m) {
+                const int q = rb + 16 * m;
+                const bool first = q < kMainN / 2;
+                const int qi = first ? q : q - kMainN / 2;
+                const bool used = qi < (first ? h0 : h1);
+                const int ci = (int)rank * (first ? h0 : h1) + qi;        // row within the chunk
+                const int lim = first ? min(ti.rows, kMainN) : ti.rows - kMainN;
+                const int64_t slot = (int64_t)ti.row0 + (first ? 0 : kMainN) + ci;
+                src[m] = nullptr;
+                if (used) {
+                    need |= 1u << m;
+                    if (ci < lim && slot < p.n_rows) {
+                        const int32_t pr = __ldg(p.pair_of_slot + slot);
+                        if (pr >= 0)
+                            src[m] = p.gather_src + (int64_t)(pr / p.top_k) * p.K + piece * 8;
+                    }
+                }
+            }
+            for (int kb = 0; kb < nk; ++kb, ++g) {
+                if (g % kGatherTeams != team) continue;
+                const int stage = (int)(g % kStages);
+                const uint32_t phase = (g / kStages) & 1u;
+                const bool ok = __all_sync(
+                    0xffffffffu, mbar_wait(empty_bar(stage), phase ^ 1u, s_abort, p.dev_status));
+                if (!ok) {
+                    aborted = true;
+                    break;
+                }
+                const int k0 = kb * BK;
+                const bool kin = k0 + piece * 8 < p.K;
+                uint4 d[kGatherRows];
+#pragma unroll
+                for (int m = 0; m < kGatherRows; ++m)
+                    d[m] = (src[m] != nullptr && kin) ? ld_nc_v4(src[m] + k0) : make_uint4(0, 0, 0, 0);
+                const uint32_t st = sbase + Smem::t + stage * kTBytes;
+#pragma unroll
+                for (int m = 0; m < kGatherRows; ++m) {
+                    const int q = rb + 16 * m;
+                    if ((need >> m) & 1u)
+                        st_shared_v4(st + q * kRowBytes + ((piece ^ (q & 7)) << 4), d[m]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(map_to_rank(full_bar(stage), 0));
+            }
+        }
+    } else if (warp >= 2 && warp < 2 + kEpiWarps) {
         // ------------------------------------------------ epilogue (both CTAs)
         const int ew = warp - 2;                 // 0..7
         const int group = ew >> 2;               // takes every kEpiGroups-th 32-column piece
@@ -545,7 +635,7 @@ static void pair_cluster(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr) {
     cfg.numAttrs = 1;
 }
 
-template <bool GLU, typename OutT>
+template <bool GLU, typename OutT, bool GATHER>
 static int resident_pairs(size_t smem) {
     static int cached = -1;
     if (cached > 0) return cached;
@@ -555,12 +645,12 @@ static int resident_pairs(size_t smem) {
     int n = sms / 2;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(2 * n));
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(threads_of<GATHER>());
     cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr[1];
     pair_cluster(cfg, attr);
     int c = 0;
-    if (cudaOccupancyMaxActiveClusters(&c, grouped_gemm_swap_kernel<GLU, OutT>, &cfg) ==
+    if (cudaOccupancyMaxActiveClusters(&c, grouped_gemm_swap_kernel<GLU, OutT, GATHER>, &cfg) ==
             cudaSuccess &&
         c > 0)
         n = c;
@@ -568,17 +658,17 @@ static int resident_pairs(size_t smem) {
     return n;
 }
 
-template <bool GLU, typename OutT>
+template <bool GLU, typename OutT, bool GATHER = false>
 static cudaError_t launch_phase(const CUtensorMap& mw, const CUtensorMap* mt, const Params& p,
                                 cudaStream_t s) {
-    auto kern = grouped_gemm_swap_kernel<GLU, OutT>;
+    auto kern = grouped_gemm_swap_kernel<GLU, OutT, GATHER>;
     constexpr size_t smem = Smem::alloc;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(2 * resident_pairs<GLU, OutT>(smem)));
-    cfg.blockDim = dim3(kThreads);
+    cfg.gridDim = dim3((unsigned)(2 * resident_pairs<GLU, OutT, GATHER>(smem)));
+    cfg.blockDim = dim3(threads_of<GATHER>());
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -604,13 +694,15 @@ static bool make_row_maps(CUtensorMap* m, const void* base, int K, int64_t n_row
 // bf16; y [n_rows, H] in y_dtype (fp32, bf16, or e4m3 codes with fp32
 // y_scales [n_rows, H/128]).  counts (may be null) cuts
 // each expert's segment to its first counts[j] rows.  ev_mid (may be null)
-// is recorded between the two phases.
+// is recorded between the two phases.  With g (the fused gather) non-null,
+// A is not read: row s of the gate/up operand is row pair_of_slot[s] / k of
+// g.src [*, H] (16-byte aligned).
 cudaError_t launch_grouped_gemm_tc_swap(const __nv_bfloat16* a, const int32_t* offsets,
                                         const int32_t* counts, int expert_begin, int n_experts,
                                         int64_t n_rows, int H, int I, const __nv_bfloat16* w13,
                                         const __nv_bfloat16* w2, __nv_bfloat16* h, void* y,
                                         moe_dtype y_dtype, float* y_scales, int32_t* dev_status,
-                                        cudaEvent_t ev_mid,
+                                        const gemm_gather* g, cudaEvent_t ev_mid,
                                         cudaStream_t s) {
     using namespace tcs;
     CUtensorMap mw1, mt1[3], mw2, mt2[3];
@@ -621,7 +713,7 @@ cudaError_t launch_grouped_gemm_tc_swap(const __nv_bfloat16* a, const int32_t* o
         const cuuint32_t box[4] = {BK, kWRows / 2, 2, 1};
         if (!make_map(&mw1, w13, 4, dims, str, box)) return cudaErrorInvalidValue;
     }
-    if (!make_row_maps(mt1, a, H, n_rows)) return cudaErrorInvalidValue;
+    if (!g && !make_row_maps(mt1, a, H, n_rows)) return cudaErrorInvalidValue;
     {   // W2 as [E, H, I]: a box of 128 rows
         const cuuint64_t dims[3] = {(cuuint64_t)I, (cuuint64_t)H, (cuuint64_t)n_experts};
         const cuuint64_t str[2] = {(cuuint64_t)I * 2, (cuuint64_t)H * I * 2};
@@ -631,12 +723,21 @@ cudaError_t launch_grouped_gemm_tc_swap(const __nv_bfloat16* a, const int32_t* o
     if (!make_row_maps(mt2, h, I, n_rows)) return cudaErrorInvalidValue;
 
     Params p1{offsets, counts, expert_begin, n_experts, H, I, (I + kWRows - 1) / kWRows,
-              (int)n_rows, h, nullptr, dev_status};
-    cudaError_t e = launch_phase<true, __nv_bfloat16>(mw1, mt1, p1, s);
+              (int)n_rows, h, nullptr, dev_status, nullptr, nullptr, 0};
+    cudaError_t e;
+    if (g) {
+        p1.gather_src = g->src;
+        p1.pair_of_slot = g->pair_of_slot;
+        p1.top_k = g->top_k;
+        const CUtensorMap unused[3] = {mw1, mw1, mw1};   // no row boxes: the rows are gathered
+        e = launch_phase<true, __nv_bfloat16, true>(mw1, unused, p1, s);
+    } else {
+        e = launch_phase<true, __nv_bfloat16>(mw1, mt1, p1, s);
+    }
     if (e == cudaSuccess && ev_mid) e = cudaEventRecord(ev_mid, s);
     if (e != cudaSuccess) return e;
     Params p2{offsets, counts, expert_begin, n_experts, I, H, (H + 2 * kWRows - 1) / (2 * kWRows),
-              (int)n_rows, y, y_scales, dev_status};
+              (int)n_rows, y, y_scales, dev_status, nullptr, nullptr, 0};
     e = y_dtype == MOE_F32    ? launch_phase<false, float>(mw2, mt2, p2, s)
         : y_dtype == MOE_BF16 ? launch_phase<false, __nv_bfloat16>(mw2, mt2, p2, s)
                               : launch_phase<false, uint8_t>(mw2, mt2, p2, s);

@@ -65,7 +65,10 @@ constexpr int kMaxBlocks = 64;           // scales staged in shared memory: H <=
 // slot once the row is done.  With `a` non-null (the layer call), the
 // kernel also writes what the grouped GEMM consumes, bf16(decode(q) *
 // scale) (an fp32 product rounded to bf16), to each slot's row of `a`,
-// so the GEMM needs no separate dequantisation pass.
+// so the GEMM needs no separate dequantisation pass.  With xp null (the
+// token-major form, for the GEMM's fused gather) only `a` is written, at
+// the token's own row t: each token is quantised once and its k copies are
+// the same row.
 template <typename T>
 __global__ void __launch_bounds__(kQuantThreads) permute_e4m3_kernel(
     const T* __restrict__ x, int64_t T_, int H, int k, const int32_t* __restrict__ slot_of_pair,
@@ -76,9 +79,10 @@ __global__ void __launch_bounds__(kQuantThreads) permute_e4m3_kernel(
     const int l8 = threadIdx.x & 7;                 // lane within the block's 8
     const int grp = threadIdx.x >> 3;               // block handled in this pass
     const int ngrp = blockDim.x >> 3;
-    const bool vec_scales = (nblk % 4) == 0 && nblk <= kMaxBlocks;
+    const bool tok_major = xp == nullptr;
+    const bool vec_scales = !tok_major && (nblk % 4) == 0 && nblk <= kMaxBlocks;
     for (int64_t t = blockIdx.x; t < T_; t += gridDim.x) {
-        if (threadIdx.x < k) s_slot[threadIdx.x] = slot_of_pair[t * k + threadIdx.x];
+        if (!tok_major && threadIdx.x < k) s_slot[threadIdx.x] = slot_of_pair[t * k + threadIdx.x];
         __syncthreads();
         const T* row = x + t * H;
         // whole warps iterate together so the 8-lane shuffles stay converged
@@ -108,7 +112,7 @@ __global__ void __launch_bounds__(kQuantThreads) permute_e4m3_kernel(
                                        quant4_e4m3(f[4], f[5], f[6], f[7], scale),
                                        quant4_e4m3(f[8], f[9], f[10], f[11], scale),
                                        quant4_e4m3(f[12], f[13], f[14], f[15], scale));
-            for (int j = 0; j < k; ++j) {
+            for (int j = 0; j < k && !tok_major; ++j) {
                 const int32_t s = s_slot[j];
                 if (s >= 0) st_v4(xp + (int64_t)s * H + g * 128 + l8 * 16, q);
             }
@@ -125,7 +129,12 @@ __global__ void __launch_bounds__(kQuantThreads) permute_e4m3_kernel(
                 }
                 const uint4 b0 = make_uint4(bw[0], bw[1], bw[2], bw[3]);
                 const uint4 b1 = make_uint4(bw[4], bw[5], bw[6], bw[7]);
-                for (int j = 0; j < k; ++j) {
+                if (tok_major) {
+                    __nv_bfloat16* dst = a + t * H + g * 128 + l8 * 16;
+                    st_v4(dst, b0);
+                    st_v4(dst + 8, b1);
+                }
+                for (int j = 0; j < k && !tok_major; ++j) {
                     const int32_t s = s_slot[j];
                     if (s < 0) continue;
                     __nv_bfloat16* dst = a + (int64_t)s * H + g * 128 + l8 * 16;
@@ -133,7 +142,7 @@ __global__ void __launch_bounds__(kQuantThreads) permute_e4m3_kernel(
                     st_v4(dst + 8, b1);
                 }
             }
-            if (l8 == 0) {
+            if (l8 == 0 && !tok_major) {
                 if (vec_scales) {
                     s_scale[g] = scale;
                 } else {
@@ -186,6 +195,22 @@ cudaError_t launch_permute(const void* x, moe_dtype xdt, int64_t T, int H, int k
         permute_copy_kernel<float><<<grid, 256, 0, s>>>((const float*)x, T, H, k, slot_of_pair,
                                                         (float*)xp);
     }
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+// Token-major FP8 round trip for the GEMM's fused gather: a[t] =
+// bf16(decode(q) * scale) of x[t]'s FP8 payload, one row per token.
+cudaError_t launch_quantize_tokens_e4m3(const void* x, moe_dtype xdt, int64_t T, int H,
+                                       __nv_bfloat16* a, cudaStream_t s) {
+    if (T == 0) return cudaSuccess;
+    const unsigned grid = permute_grid(T);
+    if (xdt == MOE_BF16)
+        permute_e4m3_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+            (const __nv_bfloat16*)x, T, H, 1, nullptr, nullptr, nullptr, a);
+    else
+        permute_e4m3_kernel<float><<<grid, 256, 0, s>>>((const float*)x, T, H, 1, nullptr,
+                                                        nullptr, nullptr, a);
     note_launches(1);
     return cudaGetLastError();
 }

@@ -139,6 +139,20 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map
             : "memory");
 }
 
+// 16-byte store to this CTA's shared memory (32-bit shared address).
+__device__ __forceinline__ void st_shared_v4(uint32_t saddr, const uint4& v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(saddr), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// Orders this thread's ordinary (generic-proxy) writes to its CTA's shared
+// memory before later async-proxy accesses to it, such as the tensor core
+// reading an MMA operand; issued by the writer before it signals a barrier.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }

@@ -53,7 +53,8 @@ SIGNATURES = {
 
 class LayerOptionsC(ctypes.Structure):
     """moe_layer_options (include/moe.h)."""
-    _fields_ = [("capacity", _I32), ("route_groups", _I32), ("route_max_groups", _I32)]
+    _fields_ = [("capacity", _I32), ("route_groups", _I32), ("route_max_groups", _I32),
+                ("fused_gather", _I32)]
 
 
 class LayerBuffersC(ctypes.Structure):
@@ -253,6 +254,8 @@ class LayerBuffers:
         self.y_scales = (torch.empty(N, H // 128, dtype=torch.float32, device=dev)
                          if wl.ydt == "e4m3" else None)
         gb = moe_grouped_gemm_workspace_bytes(N, H, I, pdt, wdt)
+        if wl.fused_gather and wl.payload == "e4m3":
+            gb = max(gb, T * H * 2)            # the fused gather's one bf16 row per token
         self.gemm_ws = torch.empty(gb, dtype=torch.uint8, device=dev) if gb else None
         self.out = torch.empty(T, H, dtype=TORCH_DTYPE[wl.act], device=dev)
 
@@ -284,7 +287,8 @@ def _events(step_events, stream=None):
 
 
 def layer_options(wl, buf: "LayerBuffers") -> LayerOptionsC:
-    return LayerOptionsC(buf.capacity, wl.route_groups, wl.route_max_groups)
+    return LayerOptionsC(buf.capacity, wl.route_groups, wl.route_max_groups,
+                         1 if wl.fused_gather else 0)
 
 
 def moe_layer_forward(wl, logits, x, w13, w2, buf: "LayerBuffers", step_events=None,

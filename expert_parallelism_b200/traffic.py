@@ -34,9 +34,14 @@ def kernel_bytes(wl: Workload, rows: int | None = None) -> dict:
         "route_topk": T * E * 4 + T * k * 8,
         "dispatch_layout": N * 4 + N * 8 + (2 * E + 1) * 4 + (wl.W + 1) * 4,
         "permute": T * H * xb + N * H * pb + scales,
-        # inside moe_layer_forward an FP8 permute also writes the GEMM's bf16 rows
-        "permute_layer": T * H * xb + N * H * pb + scales
-                         + (N * H * 2 if wl.payload == "e4m3" else 0),
+        # inside moe_layer_forward an FP8 permute also writes the GEMM's bf16
+        # rows; with the fused gather the permuted copy is never made: an FP8
+        # payload's tokens make one bf16 round trip each (T rows), a bf16
+        # payload has no step here at all
+        "permute_layer": ((T * H * xb + T * H * 2 if wl.payload == "e4m3" else 0)
+                          if wl.fused_gather else
+                          T * H * xb + N * H * pb + scales
+                          + (N * H * 2 if wl.payload == "e4m3" else 0)),
         "combine": N * H * yb + (N * (H // 128) * 4 if wl.ydt == "e4m3" else 0)
                    + T * k * 8 + T * H * xb,
     }

@@ -62,6 +62,7 @@ class Workload:
     capacity_factor: float | None = None   # None: dropless; else fixed slabs per expert
     route_groups: int = 0                  # 0: plain top-k; G: group-limited routing
     route_max_groups: int = 0              # M: groups a token may reach (with route_groups)
+    fused_gather: bool = False             # the gate/up GEMM gathers rows from x (no xp copy)
 
     @property
     def N(self) -> int:
@@ -94,6 +95,14 @@ WORKLOADS = {
     # group-limited routing: each token reaches at most 4 of the 8 rank groups
     "dsv3_grouped": Workload("dsv3_grouped", 8192, 7168, 256, 8, 2048, 8, "bf16", "e4m3",
                              "bf16", route_groups=8, route_max_groups=4),
+    # fused gather: the gate/up GEMM reads each routed row from the token-major
+    # activations through pair_of_slot, with no permuted copy in between
+    "dsv3_fused": Workload("dsv3_fused", 8192, 7168, 256, 8, 2048, 8, "bf16", "e4m3", "bf16",
+                           fused_gather=True),
+    "mid_fused": Workload("mid_fused", 4096, 2048, 64, 6, 1408, 4, "bf16", "bf16", "bf16",
+                          fused_gather=True),
+    "skew_fused": Workload("skew_fused", 16384, 2880, 128, 4, 2880, 8, "bf16", "bf16", "bf16",
+                           router="zipf", fused_gather=True),
 }
 
 TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16,

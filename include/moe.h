@@ -352,17 +352,28 @@ moe_status moe_combine(const void* y, moe_dtype y_dtype, const float* y_scales,
  *   b holds every intermediate buffer and workspace (device, caller
  *   owned); b->xp is in payload_dtype (x_dtype or MOE_E4M3), b->y in
  *   y_dtype.
- *   opts (may be NULL: capacity -1, route_groups 0):
+ *   opts (may be NULL: capacity -1, route_groups 0, fused_gather 0):
  *     capacity: -1 for the dropless layout (moe_dispatch_layout; the
  *     permuted buffers have T*k rows), or C >= 0 for fixed slabs of C rows
  *     per expert (moe_dispatch_layout_capacity; E*C rows, dropped pairs
  *     add nothing, b->n_dropped receives their number when not NULL);
  *     route_groups, route_max_groups: 0 for plain routing (moe_route_topk),
  *     or G and M for moe_route_topk_grouped.
+ *     fused_gather: 0 runs moe_permute and hands b->xp to the GEMM.  1 (bf16
+ *     weights, where the GEMM takes its operand-swapped kernel: at least 16
+ *     rows per expert on average, or y_dtype MOE_E4M3) skips the permuted
+ *     copy: the gate/up GEMM reads routed row s from row pair_of_slot[s] / k
+ *     of a token-major source, x itself for a bf16 payload, or for an FP8
+ *     payload each token's round trip bf16(decode(q) * scale) (the rows
+ *     moe_permute's payload dequantises to), written once per token into
+ *     b->gemm_workspace.  h, y and out are the same; b->xp and b->xp_scales
+ *     are not written.  Elsewhere the flag is ignored.
  *   step_events: NULL, or 8 cudaEvent_t handles recorded on `stream` at:
  *   0 before routing, 1 after routing, 2 after the layout, 3 after the
- *   permute, 4 when the GEMM's bf16 operand is ready (inside this call an
- *   FP8 permute writes it as well, so 4 follows 3 directly), 5 after the
+ *   permute (with fused_gather: after the token-major FP8 round trip, or
+ *   at once for a bf16 payload), 4 when the GEMM's bf16 operand is ready
+ *   (inside this call an FP8 permute writes it as well, so 4 follows 3
+ *   directly), 5 after the
  *   gate/up GEMM, 6 after the down GEMM, 7 after combine -- so that a caller
  *   can time each kernel on the stream it runs on, without launch gaps
  *   between them.
@@ -371,6 +382,7 @@ typedef struct moe_layer_options {
     int32_t capacity;          /* -1: dropless; C >= 0: fixed slabs of C rows per expert */
     int32_t route_groups;      /* 0: plain top-k; G: group-limited routing over G groups */
     int32_t route_max_groups;  /* M: groups each token may reach (with route_groups) */
+    int32_t fused_gather;      /* 0: permute, then the GEMM; 1: the GEMM gathers the rows */
 } moe_layer_options;
 
 typedef struct moe_layer_buffers {

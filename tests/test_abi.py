@@ -162,6 +162,19 @@ def test_layer_call_rejects_before_launch(lib):
              None) == 1
 
 
+def test_fused_gather_needs_one_workspace_row_per_token(lib):
+    """With an FP8 payload the fused gather keeps one bf16 row per token in
+    the GEMM workspace: a workspace sized only for the GEMM's slots (here 8
+    slots from capacity 1, fewer than the 10 tokens) is rejected up front."""
+    T, H, E, k, W, I = 10, 128, 8, 2, 2, 64
+    lw = moe.moe_dispatch_layout_workspace_bytes(T, k, E)
+    cb = moe.LayerBuffersC(*([FAKE] * 8 + [lw] + [FAKE] * 6 + [E * 1 * H * 2] + [FAKE, None]))
+    fused = moe.LayerOptionsC(1, 0, 0, 1)
+    assert lib.moe_layer_forward(FAKE, FAKE, moe.MOE_BF16, T, H, E, k, W, I, FAKE, FAKE,
+                                 moe.MOE_BF16, moe.MOE_E4M3, moe.MOE_F32, ctypes.byref(fused),
+                                 ctypes.byref(cb), FAKE, None, None) == 1
+
+
 def test_grouped_route_rejects_before_launch(lib):
     f = lib.moe_route_topk_grouped
     assert f(FAKE, 10, 8, 2, 3, 1, FAKE, FAKE, None) == 1      # groups must divide E
