@@ -379,13 +379,23 @@ __global__ void __launch_bounds__(threads_of<GATHER>(), 1)
         // + rank * h1 + q - 128); it is row pair_of_slot[slot] / top_k of the
         // source.  Rows are written in the 128-byte-swizzled layout a TMA box
         // would produce: 16-byte piece c of row q at q * 128 + ((c ^ (q % 8))
-        // * 16).  Rows past the pass (padding) are zeros.
+        // * 16).  Rows past the pass (padding) are zeros.  The copies are
+        // cp.async: a team releases a k-step to the MMA (its copies landed,
+        // proxy fence, one arrival per warp) only after issuing its next one,
+        // so each team keeps two k-steps in flight -- four of the five stages
+        // with both teams, and a k-step waits only on stages five back.
         const int gw = warp - kGatherWarp0;
         const uint32_t team = (uint32_t)(gw / kTeamWarps);
         const int lt = (gw % kTeamWarps) * 32 + lane;
         const int piece = lt & 7;                  // 16-byte piece of each row
         const int rb = lt >> 3;                    // rows rb, rb + 16, .., rb + 144
         uint32_t g = 0;                            // k-steps so far, both teams
+        int pending = -1;                          // stage issued but not yet released
+        auto release = [&](int stg) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(map_to_rank(full_bar(stg), 0));
+        };
         for (int t = unit; t < n_tiles && !aborted; t += n_units) {
             const TileInfo ti = tile_info(p, s_prefix, t);
             const int h0 = ti.n0 >> 1, h1 = ti.n1 >> 1;
@@ -422,22 +432,27 @@ __global__ void __launch_bounds__(threads_of<GATHER>(), 1)
                 }
                 const int k0 = kb * BK;
                 const bool kin = k0 + piece * 8 < p.K;
-                uint4 d[kGatherRows];
-#pragma unroll
-                for (int m = 0; m < kGatherRows; ++m)
-                    d[m] = (src[m] != nullptr && kin) ? ld_nc_v4(src[m] + k0) : make_uint4(0, 0, 0, 0);
                 const uint32_t st = sbase + Smem::t + stage * kTBytes;
 #pragma unroll
                 for (int m = 0; m < kGatherRows; ++m) {
                     const int q = rb + 16 * m;
-                    if ((need >> m) & 1u)
-                        st_shared_v4(st + q * kRowBytes + ((piece ^ (q & 7)) << 4), d[m]);
+                    if ((need >> m) & 1u) {
+                        const bool live = src[m] != nullptr && kin;
+                        cp_async16(st + q * kRowBytes + ((piece ^ (q & 7)) << 4),
+                                   live ? (const void*)(src[m] + k0) : (const void*)p.gather_src,
+                                   live ? 16u : 0u);
+                    }
                 }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(map_to_rank(full_bar(stage), 0));
+                cp_async_commit();
+                if (pending >= 0) {
+                    cp_async_wait<1>();            // the previous k-step's copies landed
+                    release(pending);
+                }
+                pending = stage;
             }
         }
+        cp_async_wait<0>();
+        if (!aborted && pending >= 0) release(pending);
     } else if (warp >= 2 && warp < 2 + kEpiWarps) {
         // ------------------------------------------------ epilogue (both CTAs)
         const int ew = warp - 2;                 // 0..7

@@ -146,6 +146,22 @@ __device__ __forceinline__ void st_shared_v4(uint32_t saddr, const uint4& v) {
                  : "memory");
 }
 
+// 16-byte asynchronous copy global -> this CTA's shared memory through L2
+// (cp.async.cg); src_bytes 0 reads nothing and writes 16 zero bytes.
+__device__ __forceinline__ void cp_async16(uint32_t saddr, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// Waits until at most N of this thread's committed groups are in flight.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // Orders this thread's ordinary (generic-proxy) writes to its CTA's shared
 // memory before later async-proxy accesses to it, such as the tensor core
 // reading an MMA operand; issued by the writer before it signals a barrier.
