@@ -63,6 +63,10 @@ def _load():
         lib.oracle_grouped_gemm.restype = I64
         lib.oracle_combine.argtypes = [P, I, P, P, I64, I32, I32, P, I]
         lib.oracle_combine.restype = I
+        lib.oracle_combine_rank.argtypes = [P, I, P, P, I64, I32, I32, P, I32, I32, P, I]
+        lib.oracle_combine_rank.restype = I
+        lib.oracle_reduce_partials.argtypes = [P, I, I32, I64, P, I]
+        lib.oracle_reduce_partials.restype = I
         lib.oracle_e4m3_encode.argtypes = [P, I64, P]
         lib.oracle_e4m3_decode.argtypes = [P, I64, P]
         lib.oracle_bf16_round.argtypes = [P, I64, P]
@@ -234,6 +238,37 @@ def combine(y: torch.Tensor, slot_of_pair: torch.Tensor, topk_w: torch.Tensor,
     _load().oracle_combine(_p(y), _CODE[_dt_name(y)], _p(slot_of_pair.to(torch.int32).contiguous()),
                            _p(topk_w.to(torch.float32).contiguous()), T, k, H, _p(out),
                            _CODE[out_dtype])
+    return out
+
+
+def combine_rank(y: torch.Tensor, slot_of_pair: torch.Tensor, topk_w: torch.Tensor,
+                 rank_offsets: torch.Tensor, rank: int, out_dtype: str = "f64"):
+    """Rank ``rank``'s partial of the all_reduce form: each token's weighted
+    sum over only the picks whose slot lies in the rank's slab
+    [rank_offsets[rank], rank_offsets[rank+1]) (zero rows for tokens it does
+    not serve); fp64, "f64" unrounded."""
+    y = y.contiguous()
+    T, k = topk_w.shape
+    H = y.shape[1]
+    ro = rank_offsets.to(torch.int32).contiguous()
+    out = torch.empty(T, H, dtype=_TDT[out_dtype])
+    rc = _load().oracle_combine_rank(_p(y), _CODE[_dt_name(y)],
+                                     _p(slot_of_pair.to(torch.int32).contiguous()),
+                                     _p(topk_w.to(torch.float32).contiguous()), T, k, H, _p(ro),
+                                     ro.numel() - 1, rank, _p(out), _CODE[out_dtype])
+    if rc != 0:
+        raise ValueError("combine_rank: rank outside [0, world)")
+    return out
+
+
+def reduce_partials(partials: torch.Tensor, out_dtype: str = "f64"):
+    """Sum of the ranks' partials [n, T, H] (the all-reduce), in fp64,
+    rounded once to ``out_dtype``."""
+    p = partials.contiguous()
+    n = p.shape[0]
+    out = torch.empty(p.shape[1:], dtype=_TDT[out_dtype])
+    _load().oracle_reduce_partials(_p(p), _CODE[_dt_name(p)], n, p[0].numel(), _p(out),
+                                   _CODE[out_dtype])
     return out
 
 

@@ -521,3 +521,51 @@ int oracle_combine(const void* y, int y_dt, const int32_t* slot_of_pair,
     free(acc);
     return 0;
 }
+
+/* ------------------------------------------------------------------ */
+/* The all_reduce form of the layer: per-rank partial sums, then their  */
+/* sum over ranks                                                      */
+/* ------------------------------------------------------------------ */
+/* Transformers docs, "Expert parallelism", "Choosing an implementation",
+ * the all_reduce row: no token moves; every rank runs its own experts over
+ * the whole batch it shares with the other ranks, and the ranks' outputs
+ * are summed by an all-reduce.  Rank r's experts own the slots
+ * [rank_offsets[r], rank_offsets[r+1]) of the layout, so its contribution
+ * to token t is
+ *     partial_r[t] = sum over j with slot_of_pair[t*k+j] in that range of
+ *                    topk_w[t,j] * y[slot_of_pair[t*k+j]],
+ * zero for a token none of whose picks it owns.  fp64; out_dt fp64 returns
+ * it unrounded.  Returns 0, or -1 if rank is outside [0, world). */
+int oracle_combine_rank(const void* y, int y_dt, const int32_t* slot_of_pair,
+                        const float* topk_w, int64_t T, int32_t k, int32_t H,
+                        const int32_t* rank_offsets, int32_t world, int32_t rank, void* out,
+                        int out_dt) {
+    if (rank < 0 || rank >= world) return -1;
+    const int32_t lo = rank_offsets[rank], hi = rank_offsets[rank + 1];
+    double* acc = (double*)malloc(sizeof(double) * (size_t)H);
+    for (int64_t t = 0; t < T; ++t) {
+        for (int32_t c = 0; c < H; ++c) acc[c] = 0.0;
+        for (int32_t j = 0; j < k; ++j) {
+            const int32_t s = slot_of_pair[t * k + j];
+            if (s < lo || s >= hi) continue;   /* another rank's pick, or dropped (-1) */
+            const double w = (double)topk_w[t * k + j];
+            for (int32_t c = 0; c < H; ++c) acc[c] += w * load_elem(y, y_dt, (int64_t)s * H + c);
+        }
+        for (int32_t c = 0; c < H; ++c) store_elem(out, out_dt, t * H + c, acc[c]);
+    }
+    free(acc);
+    return 0;
+}
+
+/* The all-reduce's sum: out[i] = partials[0][i] + ... + partials[n-1][i],
+ * each partial read in its own dtype, summed in fp64 and rounded once to
+ * out_dt.  n_elems elements per partial.  Returns 0. */
+int oracle_reduce_partials(const void* partials, int p_dt, int32_t n, int64_t n_elems,
+                           void* out, int out_dt) {
+    for (int64_t i = 0; i < n_elems; ++i) {
+        double acc = 0.0;
+        for (int32_t r = 0; r < n; ++r) acc += load_elem(partials, p_dt, (int64_t)r * n_elems + i);
+        store_elem(out, out_dt, i, acc);
+    }
+    return 0;
+}
