@@ -282,6 +282,7 @@ def _config(wl):
             **({"route_groups": wl.route_groups, "route_max_groups": wl.route_max_groups}
                if wl.route_groups else {}),
             "fused_gather": wl.fused_gather,
+            **({"all_reduce_form": True} if wl.all_reduce_form else {}),
             "parallelism": "replicas (one independent layer per GPU)"}
 
 

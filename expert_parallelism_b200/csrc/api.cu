@@ -20,8 +20,9 @@ cudaError_t launch_dispatch_layout(const int32_t*, int64_t, int, int, int, int, 
 cudaError_t launch_permute(const void*, moe_dtype, int64_t, int, int, const int32_t*, void*,
                            moe_dtype, float*, __nv_bfloat16*, cudaStream_t);
 cudaError_t launch_combine(const void*, moe_dtype, const float*, const int32_t*, const float*,
-                           int64_t, int,
-                           int, void*, moe_dtype, cudaStream_t);
+                           int64_t, int, int, void*, moe_dtype, cudaStream_t,
+                           const int32_t* rank_offsets = nullptr, int rank = 0);
+cudaError_t launch_reduce_partials(const float*, int, int64_t, void*, moe_dtype, cudaStream_t);
 cudaError_t launch_dequant_e4m3(const uint8_t*, const float*, const int32_t*, int, int, int64_t,
                                 int, __nv_bfloat16*, cudaStream_t);
 cudaError_t launch_grouped_gemm_simt_f32(const float*, const int32_t*, const int32_t*, int, int,
@@ -306,13 +307,38 @@ moe_status moe_combine(const void* y, moe_dtype y_dtype, const float* y_scales,
                                       out_dtype, (cudaStream_t)stream));
 }
 
+moe_status moe_combine_rank(const void* y, moe_dtype y_dtype, const float* y_scales,
+                            const int32_t* slot_of_pair, const float* topk_w, int64_t T,
+                            int32_t k, int32_t H, const int32_t* rank_offsets, int32_t world,
+                            int32_t rank, float* partial, void* stream) {
+    bool noop;
+    const moe_status st = check_combine(y, y_dtype, y_scales, slot_of_pair, topk_w, T, k, H,
+                                        partial, MOE_F32, &noop);
+    if (st != MOE_OK) return st;
+    if (world < 1 || rank < 0 || rank >= world) return MOE_ERR_INVALID_ARG;
+    if (noop) return MOE_OK;
+    if (!rank_offsets) return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_combine(y, y_dtype, y_scales, slot_of_pair, topk_w, T, k, H, partial,
+                                      MOE_F32, (cudaStream_t)stream, rank_offsets, rank));
+}
+
+moe_status moe_reduce_partials(const float* partials, int32_t n_partials, int64_t T, int32_t H,
+                               void* out, moe_dtype out_dtype, void* stream) {
+    if (n_partials < 1 || T < 0 || H < 1 || (H % 8) != 0 || !is_act_dtype(out_dtype))
+        return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!partials || !out || !aligned16(partials) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+    return cuda_status(
+        launch_reduce_partials(partials, n_partials, T * H, out, out_dtype, (cudaStream_t)stream));
+}
+
 // Rows of the permuted buffers: T*k (dropless) or E*capacity (fixed slabs).
 static int64_t layer_slots(int64_t T, int32_t k, int32_t E, int32_t capacity) {
     return capacity < 0 ? T * k : (int64_t)E * capacity;
 }
 
 static moe_layer_options resolve(const moe_layer_options* o) {
-    return o ? *o : moe_layer_options{-1, 0, 0, 0};
+    return o ? *o : moe_layer_options{-1, 0, 0, 0, 0};
 }
 
 static moe_status check_layer(const float* logits, const void* x, moe_dtype x_dtype, int64_t T,
@@ -344,6 +370,9 @@ static moe_status check_layer(const float* logits, const void* x, moe_dtype x_dt
     if (st == MOE_OK)
         st = check_combine(b->y, y_dtype, b->y_scales, b->slot_of_pair, b->topk_w, T, k, H, out,
                            x_dtype, &noop);
+    // the all_reduce form: W fp32 partials of [T, H]
+    if (st == MOE_OK && o.all_reduce_form != 0 && T > 0 && (!b->partials || !aligned16(b->partials)))
+        st = MOE_ERR_INVALID_ARG;
     // the fused gather's FP8 source, one bf16 row per token, lives in the
     // GEMM workspace
     if (st == MOE_OK && o.fused_gather != 0 && payload_dtype == MOE_E4M3 && T > 0 &&
@@ -402,9 +431,17 @@ static cudaError_t launch_layer(const float* logits, const void* x, moe_dtype x_
         if (e == cudaSuccess) e = mark(5);
     }
     if (e == cudaSuccess) e = mark(6);
-    if (e == cudaSuccess && T > 0)
+    if (e == cudaSuccess && T > 0 && o.all_reduce_form != 0) {
+        // each logical rank's partial over its own slab, then their sum in
+        // rank order (on W GPUs: the all-reduce) rounded once
+        for (int r = 0; r < W && e == cudaSuccess; ++r)
+            e = launch_combine(b->y, y_dtype, b->y_scales, b->slot_of_pair, b->topk_w, T, k, H,
+                               b->partials + (int64_t)r * T * H, MOE_F32, s, b->rank_offsets, r);
+        if (e == cudaSuccess) e = launch_reduce_partials(b->partials, W, T * H, out, x_dtype, s);
+    } else if (e == cudaSuccess && T > 0) {
         e = launch_combine(b->y, y_dtype, b->y_scales, b->slot_of_pair, b->topk_w, T, k, H, out,
                            x_dtype, s);
+    }
     if (e == cudaSuccess) e = mark(7);
     return e;
 }

@@ -13,8 +13,16 @@
 //
 // With the FP8 combine payload ("Expert parallelism and all-to-all",
 // "Traffic math": 1-byte activations both ways) y holds e4m3 codes with one
-// fp32 scale per 128 elements; a piece is 8 codes (one 8-byte load) and its
-// block's scale, used as decode(q) * scale, an fp32 product.
+// fp32 scale per 128 elements; a piece is 16 codes (one 16-byte load) and
+// its block's scale, used as decode(q) * scale, an fp32 product.
+//
+// The all_reduce form of the layer (Transformers docs, "Expert
+// parallelism", "Choosing an implementation": no token moves, every rank
+// runs its experts over the whole batch, and the ranks' outputs are summed
+// by an all-reduce) uses the same kernel restricted to one rank's slab of
+// slots, [rank_offsets[r], rank_offsets[r+1]) read on the device, writing
+// an fp32 partial; reduce_partials_kernel sums the ranks' partials in rank
+// order and rounds once.
 #include "common.cuh"
 
 namespace moe {
@@ -94,20 +102,27 @@ struct Piece<uint8_t> {
     }
 };
 
+// rank_offsets null: every pick.  Otherwise only picks whose slot lies in
+// [rank_offsets[rank], rank_offsets[rank + 1]) (the others add nothing).
 template <typename TY, typename TO>
 __global__ void __launch_bounds__(256) combine_kernel(const TY* __restrict__ y,
                                                       const float* __restrict__ y_scales,
                                                       const int32_t* __restrict__ slot_of_pair,
                                                       const float* __restrict__ topk_w, int64_t T,
-                                                      int k, int H, TO* __restrict__ out) {
+                                                      int k, int H, TO* __restrict__ out,
+                                                      const int32_t* __restrict__ rank_offsets,
+                                                      int rank) {
     using P = Piece<TY>;
     constexpr int EPT = P::N;
     __shared__ int32_t s_slot[kCombineMaxTopK];
     __shared__ float s_w[kCombineMaxTopK];
     const int nchunk = H / EPT;
+    const int32_t lo = rank_offsets ? __ldg(rank_offsets + rank) : INT32_MIN;
+    const int32_t hi = rank_offsets ? __ldg(rank_offsets + rank + 1) : INT32_MAX;
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
         if (threadIdx.x < k) {
-            s_slot[threadIdx.x] = slot_of_pair[t * k + threadIdx.x];
+            const int32_t sl = slot_of_pair[t * k + threadIdx.x];
+            s_slot[threadIdx.x] = (sl >= lo && sl < hi) ? sl : -1;
             s_w[threadIdx.x] = topk_w[t * k + threadIdx.x];
         }
         __syncthreads();
@@ -143,21 +158,27 @@ __global__ void __launch_bounds__(256) combine_kernel(const TY* __restrict__ y,
     }
 }
 
-cudaError_t launch_combine(const void* y, moe_dtype ydt, const float* y_scales,
-                           const int32_t* slot_of_pair, const float* topk_w, int64_t T, int k,
-                           int H, void* out, moe_dtype odt, cudaStream_t s) {
-    if (T == 0) return cudaSuccess;
+static int64_t sm_grid_cap() {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t cap = (int64_t)sms * 8;
+    return (int64_t)sms * 8;   // 8 CTAs of <= 256 threads per SM
+}
+
+// rank_offsets (may be null): restrict to rank `rank`'s slab of slots.
+cudaError_t launch_combine(const void* y, moe_dtype ydt, const float* y_scales,
+                           const int32_t* slot_of_pair, const float* topk_w, int64_t T, int k,
+                           int H, void* out, moe_dtype odt, cudaStream_t s,
+                           const int32_t* rank_offsets, int rank) {
+    if (T == 0) return cudaSuccess;
+    const int64_t cap = sm_grid_cap();
     const unsigned grid = (unsigned)(T < cap ? T : cap);
     const int ept = ydt == MOE_E4M3 ? 16 : 8;
     int threads = ((H / ept + 31) / 32) * 32;
     threads = threads < 32 ? 32 : (threads > 256 ? 256 : threads);
 #define MOE_COMBINE(TY, TO)                                                               \
     combine_kernel<TY, TO><<<grid, threads, 0, s>>>((const TY*)y, y_scales, slot_of_pair, \
-                                                    topk_w, T, k, H, (TO*)out)
+                                                    topk_w, T, k, H, (TO*)out, rank_offsets, rank)
     if (ydt == MOE_E4M3 && odt == MOE_BF16) MOE_COMBINE(uint8_t, __nv_bfloat16);
     else if (ydt == MOE_E4M3) MOE_COMBINE(uint8_t, float);
     else if (ydt == MOE_BF16 && odt == MOE_BF16) MOE_COMBINE(__nv_bfloat16, __nv_bfloat16);
@@ -165,6 +186,45 @@ cudaError_t launch_combine(const void* y, moe_dtype ydt, const float* y_scales,
     else if (odt == MOE_BF16) MOE_COMBINE(float, __nv_bfloat16);
     else MOE_COMBINE(float, float);
 #undef MOE_COMBINE
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+// out[i] = (((p[0][i] + p[1][i]) + p[2][i]) + ...) in fp32, rounded once to
+// TO; each thread owns 8 consecutive elements (16-byte loads), n_elems % 8
+// == 0.  With one partial it is the rounding after an all-reduce.
+template <typename TO>
+__global__ void __launch_bounds__(256) reduce_partials_kernel(const float* __restrict__ p, int n,
+                                                              int64_t n_elems,
+                                                              TO* __restrict__ out) {
+    const int64_t nvec = n_elems / 8;
+    for (int64_t v = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; v < nvec;
+         v += (int64_t)gridDim.x * blockDim.x) {
+        float acc[8];
+        load8_row(p + v * 8, acc);
+        for (int r = 1; r < n; ++r) {
+            float f[8];
+            load8_row(p + (int64_t)r * n_elems + v * 8, f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], f[i]);
+        }
+        store8(out + v * 8, acc);
+    }
+}
+
+cudaError_t launch_reduce_partials(const float* partials, int n, int64_t n_elems, void* out,
+                                   moe_dtype odt, cudaStream_t s) {
+    if (n_elems == 0) return cudaSuccess;
+    const int64_t nvec = n_elems / 8;
+    int64_t grid = (nvec + 255) / 256;
+    const int64_t cap = sm_grid_cap();
+    if (grid > cap) grid = cap;
+    if (odt == MOE_BF16)
+        reduce_partials_kernel<__nv_bfloat16><<<(unsigned)grid, 256, 0, s>>>(
+            partials, n, n_elems, (__nv_bfloat16*)out);
+    else
+        reduce_partials_kernel<float><<<(unsigned)grid, 256, 0, s>>>(partials, n, n_elems,
+                                                                    (float*)out);
     note_launches(1);
     return cudaGetLastError();
 }

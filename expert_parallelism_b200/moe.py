@@ -41,6 +41,8 @@ SIGNATURES = {
     "moe_grouped_gemm": ([_P, _I, _P, _P, _P, _I32, _I32, _I64, _I32, _I32, _P, _P, _I, _P, _P,
                           _I, _P, _P, _SZ, _P, _P], _I),
     "moe_combine": ([_P, _I, _P, _P, _P, _I64, _I32, _I32, _P, _I, _P], _I),
+    "moe_combine_rank": ([_P, _I, _P, _P, _P, _I64, _I32, _I32, _P, _I32, _I32, _P, _P], _I),
+    "moe_reduce_partials": ([_P, _I32, _I64, _I32, _P, _I, _P], _I),
     "moe_layer_forward": ([_P, _P, _I, _I64, _I32, _I32, _I32, _I32, _I32, _P, _P, _I, _I, _I,
                            _P, _P, _P, _P, _P], _I),
     "moe_layer_forward_host": ([_P, _P, _P, _P, _P, _P, _I, _I64, _I32, _I32, _I32, _I32, _I32,
@@ -54,7 +56,7 @@ SIGNATURES = {
 class LayerOptionsC(ctypes.Structure):
     """moe_layer_options (include/moe.h)."""
     _fields_ = [("capacity", _I32), ("route_groups", _I32), ("route_max_groups", _I32),
-                ("fused_gather", _I32)]
+                ("fused_gather", _I32), ("all_reduce_form", _I32)]
 
 
 class LayerBuffersC(ctypes.Structure):
@@ -64,7 +66,7 @@ class LayerBuffersC(ctypes.Structure):
                 ("pair_of_slot", _P), ("layout_workspace", _P),
                 ("layout_workspace_bytes", _SZ), ("xp", _P), ("xp_scales", _P), ("h", _P),
                 ("y", _P), ("y_scales", _P), ("gemm_workspace", _P), ("gemm_workspace_bytes", _SZ),
-                ("dev_status", _P), ("n_dropped", _P)]
+                ("dev_status", _P), ("n_dropped", _P), ("partials", _P)]
 
 
 class MoEError(RuntimeError):
@@ -195,6 +197,24 @@ def moe_combine(y, slot_of_pair, topk_w, out, stream=None, y_scales=None):
         _ptr(out), dtype_code(out), _stream(stream)))
 
 
+def moe_combine_rank(y, slot_of_pair, topk_w, rank_offsets, rank, partial, stream=None,
+                     y_scales=None):
+    """Rank ``rank``'s fp32 partial of the all_reduce form (its own slab of
+    slots only); ``rank_offsets`` has world + 1 entries."""
+    T, k = topk_w.shape
+    H = y.shape[1]
+    _check("moe_combine_rank", load_library().moe_combine_rank(
+        _ptr(y), dtype_code(y), _ptr(y_scales), _ptr(slot_of_pair), _ptr(topk_w), T, k, H,
+        _ptr(rank_offsets), rank_offsets.numel() - 1, rank, _ptr(partial), _stream(stream)))
+
+
+def moe_reduce_partials(partials, out, stream=None):
+    """out = the sum of partials [n, T, H] (fp32, rank order), rounded once."""
+    n, T, H = partials.shape
+    _check("moe_reduce_partials", load_library().moe_reduce_partials(
+        _ptr(partials), n, T, H, _ptr(out), dtype_code(out), _stream(stream)))
+
+
 def moe_check_status(dev_status, stream=None) -> int:
     """Synchronises the stream; returns the raw status code (0 = OK)."""
     return int(load_library().moe_check_status(_ptr(dev_status), _stream(stream)))
@@ -258,6 +278,8 @@ class LayerBuffers:
             gb = max(gb, T * H * 2)            # the fused gather's one bf16 row per token
         self.gemm_ws = torch.empty(gb, dtype=torch.uint8, device=dev) if gb else None
         self.out = torch.empty(T, H, dtype=TORCH_DTYPE[wl.act], device=dev)
+        self.partials = (torch.empty(W, T, H, dtype=torch.float32, device=dev)
+                         if wl.all_reduce_form else None)
 
 
 def _nbytes(t):
@@ -271,7 +293,7 @@ def layer_buffers_c(buf: "LayerBuffers") -> LayerBuffersC:
         _ptr(buf.layout_ws), _nbytes(buf.layout_ws), _ptr(buf.xp), _ptr(buf.xp_scales),
         _ptr(buf.h), _ptr(buf.y), _ptr(buf.y_scales), _ptr(buf.gemm_ws), _nbytes(buf.gemm_ws),
         _ptr(buf.dev_status),
-        _ptr(buf.n_dropped))
+        _ptr(buf.n_dropped), _ptr(buf.partials))
 
 
 def _events(step_events, stream=None):
@@ -288,7 +310,7 @@ def _events(step_events, stream=None):
 
 def layer_options(wl, buf: "LayerBuffers") -> LayerOptionsC:
     return LayerOptionsC(buf.capacity, wl.route_groups, wl.route_max_groups,
-                         1 if wl.fused_gather else 0)
+                         1 if wl.fused_gather else 0, 1 if wl.all_reduce_form else 0)
 
 
 def moe_layer_forward(wl, logits, x, w13, w2, buf: "LayerBuffers", step_events=None,

@@ -42,8 +42,11 @@ def kernel_bytes(wl: Workload, rows: int | None = None) -> dict:
                           if wl.fused_gather else
                           T * H * xb + N * H * pb + scales
                           + (N * H * 2 if wl.payload == "e4m3" else 0)),
+        # the all_reduce form reads slot_of_pair and topk_w once per rank,
+        # writes W fp32 partials and reads them back for the sum
         "combine": N * H * yb + (N * (H // 128) * 4 if wl.ydt == "e4m3" else 0)
-                   + T * k * 8 + T * H * xb,
+                   + T * k * 8 * (wl.W if wl.all_reduce_form else 1) + T * H * xb
+                   + (2 * wl.W * T * H * 4 if wl.all_reduce_form else 0),
     }
 
 

@@ -63,6 +63,7 @@ class Workload:
     route_groups: int = 0                  # 0: plain top-k; G: group-limited routing
     route_max_groups: int = 0              # M: groups a token may reach (with route_groups)
     fused_gather: bool = False             # the gate/up GEMM gathers rows from x (no xp copy)
+    all_reduce_form: bool = False          # combine as W per-rank partials summed over ranks
 
     @property
     def N(self) -> int:
@@ -103,6 +104,12 @@ WORKLOADS = {
                           fused_gather=True),
     "skew_fused": Workload("skew_fused", 16384, 2880, 128, 4, 2880, 8, "bf16", "bf16", "bf16",
                            router="zipf", fused_gather=True),
+    # the all_reduce form: each logical rank's partial sum over its own
+    # experts' picks, then the sum over ranks (the all-reduce) rounded once
+    "dsv3_allreduce": Workload("dsv3_allreduce", 8192, 7168, 256, 8, 2048, 8, "bf16", "e4m3",
+                               "bf16", all_reduce_form=True),
+    "decode_allreduce": Workload("decode_allreduce", 64, 7168, 256, 8, 2048, 8, "bf16", "bf16",
+                                 "bf16", all_reduce_form=True),
 }
 
 TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16,

@@ -340,6 +340,40 @@ moe_status moe_combine(const void* y, moe_dtype y_dtype, const float* y_scales,
                        int32_t H, void* out, moe_dtype out_dtype, void* stream);
 
 /*
+ * moe_combine_rank -- rank `rank`'s partial in the all_reduce form of the
+ * layer, where no token moves: every rank holds the whole batch, runs its
+ * own experts, and the ranks' per-token outputs are summed by an
+ * all-reduce (Transformers docs, "Expert parallelism", "Choosing an
+ * implementation", the all_reduce row).  Rank r's experts own the slots
+ * [rank_offsets[r], rank_offsets[r+1]) of the layout, so
+ *     partial[t] = sum over j with slot_of_pair[t*k+j] in that range of
+ *                  topk_w[t,j] * y[slot_of_pair[t*k+j]],
+ * fp32 accumulation in j order, unrounded fp32 result (zeros for a token
+ * with no pick on the rank).  The bounds are read on the device, so the
+ * call needs no host synchronisation.
+ *
+ *   y, y_dtype, y_scales, slot_of_pair, topk_w, T, k, H: as moe_combine.
+ *   rank_offsets [world + 1] int32, device (moe_dispatch_layout's output).
+ *   rank         in [0, world).
+ *   partial      [T, H] fp32, device, written (16-byte aligned).
+ */
+moe_status moe_combine_rank(const void* y, moe_dtype y_dtype, const float* y_scales,
+                            const int32_t* slot_of_pair, const float* topk_w, int64_t T,
+                            int32_t k, int32_t H, const int32_t* rank_offsets, int32_t world,
+                            int32_t rank, float* partial, void* stream);
+
+/*
+ * moe_reduce_partials -- the all-reduce's sum of n_partials fp32 partials
+ * [n_partials, T, H] (contiguous): out = ((p[0] + p[1]) + p[2]) + ..., in
+ * fp32 in rank order, rounded once to out_dtype (MOE_F32 / MOE_BF16).
+ * With n_partials = 1 it is the rounding that follows an all-reduce done
+ * elsewhere (for example NCCL over W GPUs, on the fp32 partials).
+ * Requires H % 8 == 0; partials and out 16-byte aligned, device.
+ */
+moe_status moe_reduce_partials(const float* partials, int32_t n_partials, int64_t T, int32_t H,
+                               void* out, moe_dtype out_dtype, void* stream);
+
+/*
  * moe_layer_forward -- the whole hot path in one call: moe_route_topk,
  * moe_dispatch_layout, moe_permute, moe_grouped_gemm (every expert, local
  * expert j = global expert j) and moe_combine, in that order on `stream`,
@@ -352,7 +386,8 @@ moe_status moe_combine(const void* y, moe_dtype y_dtype, const float* y_scales,
  *   b holds every intermediate buffer and workspace (device, caller
  *   owned); b->xp is in payload_dtype (x_dtype or MOE_E4M3), b->y in
  *   y_dtype.
- *   opts (may be NULL: capacity -1, route_groups 0, fused_gather 0):
+ *   opts (may be NULL: capacity -1, route_groups 0, fused_gather 0,
+ *   all_reduce_form 0):
  *     capacity: -1 for the dropless layout (moe_dispatch_layout; the
  *     permuted buffers have T*k rows), or C >= 0 for fixed slabs of C rows
  *     per expert (moe_dispatch_layout_capacity; E*C rows, dropped pairs
@@ -368,6 +403,10 @@ moe_status moe_combine(const void* y, moe_dtype y_dtype, const float* y_scales,
  *     moe_permute's payload dequantises to), written once per token into
  *     b->gemm_workspace.  h, y and out are the same; b->xp and b->xp_scales
  *     are not written.  Elsewhere the flag is ignored.
+ *     all_reduce_form: 0 runs moe_combine.  1 runs the combine of the
+ *     all_reduce form on the W logical ranks: moe_combine_rank for r = 0..W-1
+ *     into b->partials[r], then moe_reduce_partials into out (the same sum,
+ *     associated by rank).
  *   step_events: NULL, or 8 cudaEvent_t handles recorded on `stream` at:
  *   0 before routing, 1 after routing, 2 after the layout, 3 after the
  *   permute (with fused_gather: after the token-major FP8 round trip, or
@@ -383,6 +422,7 @@ typedef struct moe_layer_options {
     int32_t route_groups;      /* 0: plain top-k; G: group-limited routing over G groups */
     int32_t route_max_groups;  /* M: groups each token may reach (with route_groups) */
     int32_t fused_gather;      /* 0: permute, then the GEMM; 1: the GEMM gathers the rows */
+    int32_t all_reduce_form;   /* 0: one combine; 1: W per-rank partials, then their sum */
 } moe_layer_options;
 
 typedef struct moe_layer_buffers {
@@ -404,6 +444,7 @@ typedef struct moe_layer_buffers {
     size_t gemm_workspace_bytes;
     int32_t* dev_status;     /* int32, zero-initialised */
     int32_t* n_dropped;      /* int32 or NULL: dropped pairs (capacity >= 0) */
+    float* partials;         /* [W, T, H] fp32 (all_reduce_form only), else NULL */
 } moe_layer_buffers;
 
 moe_status moe_layer_forward(const float* logits, const void* x, moe_dtype x_dtype, int64_t T,

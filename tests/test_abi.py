@@ -162,6 +162,28 @@ def test_layer_call_rejects_before_launch(lib):
              None) == 1
 
 
+def test_all_reduce_form_calls_reject_before_launch(lib):
+    cr = lib.moe_combine_rank
+    assert cr(FAKE, moe.MOE_BF16, None, FAKE, FAKE, 10, 2, 128, FAKE, 4, 4, FAKE, None) == 1  # rank
+    assert cr(FAKE, moe.MOE_BF16, None, FAKE, FAKE, 10, 2, 128, FAKE, 4, -1, FAKE, None) == 1
+    assert cr(FAKE, moe.MOE_BF16, None, FAKE, FAKE, 10, 2, 128, None, 4, 0, FAKE, None) == 1  # offsets
+    assert cr(FAKE, moe.MOE_BF16, None, FAKE, FAKE, 10, 2, 100, FAKE, 4, 0, FAKE, None) == 1  # H % 8
+    assert cr(FAKE, moe.MOE_BF16, None, FAKE, FAKE, 0, 2, 128, None, 4, 0, None, None) == 0   # empty
+    rp = lib.moe_reduce_partials
+    assert rp(FAKE, 0, 10, 128, FAKE, moe.MOE_BF16, None) == 1             # no partials
+    assert rp(FAKE, 2, 10, 100, FAKE, moe.MOE_BF16, None) == 1             # H % 8
+    assert rp(FAKE, 2, 10, 128, FAKE, moe.MOE_E4M3, None) == 1             # out dtype
+    assert rp(ctypes.c_void_p(4100), 2, 10, 128, FAKE, moe.MOE_BF16, None) == 1   # alignment
+    assert rp(None, 2, 0, 128, None, moe.MOE_BF16, None) == 0              # empty
+    # the layer's all_reduce form needs the partials buffer
+    lw = moe.moe_dispatch_layout_workspace_bytes(10, 2, 8)
+    cb = moe.LayerBuffersC(*([FAKE] * 8 + [lw] + [FAKE] * 6 + [0] + [FAKE, None, None]))
+    o = moe.LayerOptionsC(-1, 0, 0, 0, 1)
+    assert lib.moe_layer_forward(FAKE, FAKE, moe.MOE_BF16, 10, 128, 8, 2, 2, 64, FAKE, FAKE,
+                                 moe.MOE_BF16, moe.MOE_BF16, moe.MOE_F32, ctypes.byref(o),
+                                 ctypes.byref(cb), FAKE, None, None) == 1
+
+
 def test_fused_gather_needs_one_workspace_row_per_token(lib):
     """With an FP8 payload the fused gather keeps one bf16 row per token in
     the GEMM workspace: a workspace sized only for the GEMM's slots (here 8
@@ -169,7 +191,7 @@ def test_fused_gather_needs_one_workspace_row_per_token(lib):
     T, H, E, k, W, I = 10, 128, 8, 2, 2, 64
     lw = moe.moe_dispatch_layout_workspace_bytes(T, k, E)
     cb = moe.LayerBuffersC(*([FAKE] * 8 + [lw] + [FAKE] * 6 + [E * 1 * H * 2] + [FAKE, None]))
-    fused = moe.LayerOptionsC(1, 0, 0, 1)
+    fused = moe.LayerOptionsC(1, 0, 0, 1, 0)
     assert lib.moe_layer_forward(FAKE, FAKE, moe.MOE_BF16, T, H, E, k, W, I, FAKE, FAKE,
                                  moe.MOE_BF16, moe.MOE_E4M3, moe.MOE_F32, ctypes.byref(fused),
                                  ctypes.byref(cb), FAKE, None, None) == 1

@@ -1,10 +1,12 @@
-"""The N > 1 launch path of bench.py, on CPU ranks over gloo.
+"""The N > 1 paths, on CPU ranks over gloo.
 
-With N GPUs every rank runs an independent replica of the layer (the path
-has no exchange step on one GPU's data), so the only cross-rank work is the
-max over ranks of the device times and the whole-job rate computed from it.
-These tests run that logic with world_size 2 on the gloo backend, and run
-the reference arm under torchrun, where rank 0 alone times the oracle.
+With N GPUs bench.py runs an independent replica of the layer per rank, so
+its only cross-rank work is the max over ranks of the device times and the
+whole-job rate computed from it.  These tests run that logic with
+world_size 2 on the gloo backend, run the reference arm under torchrun
+(rank 0 alone times the oracle), and run the exchange step of the layer's
+all_reduce form (ep_allreduce.all_reduce_partial) on partials the oracle
+computes for each rank.
 """
 import json
 import os
@@ -81,3 +83,43 @@ def test_reference_arm_under_torchrun_world2():
     assert line["value"] > 0 and line["e2e"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert line["config"]["workload"] == "tiny"
+
+
+def _allreduce_rank_main(rank, world, port, q):
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import oracle
+    from expert_parallelism_b200 import ep_allreduce
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # the same batch on both ranks; dyadic values keep every sum exact
+        T, k, E, H = 50, 4, 8, 16
+        g = torch.Generator().manual_seed(31)
+        idx, _ = oracle.route_topk(torch.randn(T, E, generator=g), k)
+        lay = oracle.dispatch_layout(idx, E, world)
+        y = torch.randint(-64, 65, (T * k, H), generator=g).float() / 8
+        w = torch.randint(1, 16, (T, k), generator=g).float() / 16
+        part = oracle.combine_rank(y, lay["slot_of_pair"], w, lay["rank_offsets"], rank, "f32")
+        ep_allreduce.all_reduce_partial(part)
+        whole = oracle.combine(y, lay["slot_of_pair"], w, "f32")
+        q.put((rank, bool(torch.equal(part, whole)), int((part != 0).any(dim=1).sum())))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_all_reduce_form_exchange_gloo_world2():
+    """Each rank's partial covers its own experts' picks only; after the
+    all-reduce both ranks hold the full combine, bit for bit."""
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_allreduce_rank_main, args=(r, world, port, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(world))
+    assert [r[1] for r in res] == [True, True]
