@@ -44,6 +44,23 @@ def test_every_declared_symbol_is_exported_and_bound(lib):
         assert name in moe.SIGNATURES, f"binding lacks {name}"
 
 
+def _struct_fields(name):
+    """Field names of `typedef struct <name> {...} <name>;` in the header,
+    in order."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    body = re.search(r"typedef struct " + name + r"\s*\{(.*?)\}\s*" + name + ";", src, re.S)
+    assert body, name
+    return re.findall(r"(\w+)\s*;", body.group(1))      # each declaration ends "name;"
+
+
+def test_layer_structs_match_the_header():
+    """The ctypes mirrors of moe_layer_options and moe_layer_buffers list the
+    header's fields in the header's order (a drift would shift every later
+    field)."""
+    assert [f[0] for f in moe.LayerOptionsC._fields_] == _struct_fields("moe_layer_options")
+    assert [f[0] for f in moe.LayerBuffersC._fields_] == _struct_fields("moe_layer_buffers")
+
+
 def test_status_strings(lib):
     assert moe.moe_status_str(0) == "MOE_OK"
     assert moe.moe_status_str(1) == "MOE_ERR_INVALID_ARG"
