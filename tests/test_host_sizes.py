@@ -42,3 +42,16 @@ def test_buffers_for_the_options():
     opts = moe.layer_options(wl.replace(fused_gather=True, all_reduce_form=True), ar)
     assert (opts.capacity, opts.fused_gather, opts.all_reduce_form) == (ar.capacity, 1, 1)
     assert moe.layer_buffers_c(ar).partials == ar.partials.data_ptr()
+
+
+def test_permute_bytes_and_gemm_flops_of_the_five_workloads():
+    """Hand-computed: the permute reads x once and writes T*k payload rows
+    (plus fp32 scales per 128 for FP8); the expert FFN is 6 N H I flops."""
+    want_permute_mb = {"tiny": 0.393, "mid": 117.4, "dsv3": 601.9, "skew": 471.9, "decode": 8.26}
+    want_gflops = {"tiny": 0.1007, "mid": 425.2, "dsv3": 5772.0, "skew": 3261.4, "decode": 45.10}
+    for name in want_permute_mb:
+        wl = workloads.WORKLOADS[name]
+        mb = traffic.kernel_bytes(wl)["permute"] / 1e6
+        gf = traffic.gemm_flops(wl)["total"] / 1e9
+        assert abs(mb - want_permute_mb[name]) <= 0.002 * want_permute_mb[name], (name, mb)
+        assert abs(gf - want_gflops[name]) <= 0.002 * want_gflops[name], (name, gf)
