@@ -52,78 +52,78 @@ def _peaks():
 
 
 class ClockSampler:
-    """SM clock and clock-event (throttle) reasons sampled every 10 ms while
-    the timed region runs.  Reads NVML (the library nvidia-smi reports from),
-    for the device whose UUID the CUDA runtime gives; falls back to polling
-    nvidia-smi when NVML cannot be loaded.  Read-only: changes no setting."""
+    """SM clock and clock-event (throttle) reasons sampled while the timed
+    region runs, kept sample by sample.  Two read-only sources run side by
+    side: NVML polled every 5 ms from a thread (for the device whose UUID the
+    CUDA runtime gives), and ``nvidia-smi -lms 50`` (the tool the recipe's
+    clocks line uses).  Changes no setting."""
 
     REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
                "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
     SMI_FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
                   "clocks_event_reasons.hw_thermal_slowdown,"
                   "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    SMI_NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def __init__(self, device: torch.device, period_s: float = 0.01):
+    def __init__(self, device: torch.device, period_s: float = 0.005):
         self.device = device
         self.period = period_s
-        self.sm, self.max_mhz, self.reasons = [], None, set()
+        self.nvml, self.smi = [], []      # (ms since start, MHz, reason names)
+        self.max_mhz = None
         self.stop = threading.Event()
-        self.t = None
+        self.threads = []
         self.proc = None
-        self.source = None
+        self.t0 = None
 
-    def _nvml_handle(self):
-        import pynvml
-        pynvml.nvmlInit()
-        uuid = str(torch.cuda.get_device_properties(self.device).uuid)
-        if not uuid.startswith("GPU-"):
-            uuid = "GPU-" + uuid
-        return pynvml, pynvml.nvmlDeviceGetHandleByUUID(uuid)
+    def _uuid(self):
+        u = str(torch.cuda.get_device_properties(self.device).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+
+    def _now_ms(self):
+        return (time.perf_counter() - self.t0) * 1e3
 
     def _poll_nvml(self, nv, h):
         self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
         while not self.stop.is_set():
-            self.sm.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
+            mhz = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
             bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
-            for n, b in self.REASONS.items():
-                if bits & b:
-                    self.reasons.add(n)
+            names = [n for n, b in self.REASONS.items() if bits & b]
+            self.nvml.append((self._now_ms(), mhz, names))
             self.stop.wait(self.period)
 
     def _read_smi(self):
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in self.proc.stdout:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 6:
                 continue
             try:
-                self.sm.append(float(parts[0]))
-                self.max_mhz = float(parts[1])
+                mhz, mx = float(parts[0]), float(parts[1])
             except ValueError:
                 continue
-            for n, v in zip(names, parts[2:6]):
-                if v.lower() == "active":
-                    self.reasons.add(n)
+            self.max_mhz = self.max_mhz or mx
+            names = [n for n, v in zip(self.SMI_NAMES, parts[2:6]) if v.lower() == "active"]
+            self.smi.append((self._now_ms(), mhz, names))
 
     def __enter__(self):
+        self.t0 = time.perf_counter()
         try:
-            nv, h = self._nvml_handle()
-            self.t = threading.Thread(target=self._poll_nvml, args=(nv, h), daemon=True)
-            self.source = "nvml, 10 ms"
+            import pynvml as nv
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByUUID(self._uuid())
+            self.threads.append(threading.Thread(target=self._poll_nvml, args=(nv, h),
+                                                 daemon=True))
         except Exception:
-            try:
-                idx = str(torch.cuda.get_device_properties(self.device).uuid)
-                idx = idx if idx.startswith("GPU-") else "GPU-" + idx
-                self.proc = subprocess.Popen(
-                    ["nvidia-smi", "-i", idx, f"--query-gpu={self.SMI_FIELDS}",
-                     "--format=csv,noheader,nounits", "-lms", "100"],
-                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-                self.t = threading.Thread(target=self._read_smi, daemon=True)
-                self.source = "nvidia-smi, 100 ms"
-            except Exception:
-                self.t = None
-        if self.t is not None:
-            self.t.start()
+            pass
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self._uuid(), f"--query-gpu={self.SMI_FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.threads.append(threading.Thread(target=self._read_smi, daemon=True))
+        except Exception:
+            self.proc = None
+        for t in self.threads:
+            t.start()
         return self
 
     def __exit__(self, *a):
@@ -134,15 +134,37 @@ class ClockSampler:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
-        if self.t is not None:
-            self.t.join(timeout=5)
+        for t in self.threads:
+            t.join(timeout=5)
 
-    def summary(self):
-        sm = sorted(self.sm)
-        pct = lambda q: sm[min(len(sm) - 1, int(q * len(sm)))] if sm else None
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
-                "sm_mhz_p10": pct(0.1), "sm_mhz_min": sm[0] if sm else None,
-                "reasons": sorted(self.reasons), "samples": len(sm), "source": self.source}
+    @staticmethod
+    def _stats(samples):
+        if not samples:
+            return None
+        mhz = sorted(s[1] for s in samples)
+        cap = sum(1 for s in samples if "sw_power_cap" in s[2])
+        return {"samples": len(samples), "sm_mhz_median": statistics.median(mhz),
+                "sm_mhz_p10": mhz[min(len(mhz) - 1, int(0.1 * len(mhz)))], "sm_mhz_min": mhz[0],
+                "sw_power_cap_frac": cap / len(samples),
+                "reasons": sorted({n for s in samples for n in s[2]}),
+                # (ms from the start of the timed region, MHz, active reasons)
+                "trace": [[round(s[0], 1), s[1], s[2]] for s in samples[:64]]}
+
+    def summary(self, ms_per_step=None):
+        """Median and spread per source; the headline figures take
+        nvidia-smi's when it gave at least 3 samples, else NVML's.
+        ``ms_x_mhz`` (step time x median SM MHz) lets step times taken at
+        different clocks be compared."""
+        nv, smi = self._stats(self.nvml), self._stats(self.smi)
+        head = smi if smi and smi["samples"] >= 3 else (nv or smi)
+        out = {"sm_mhz": head["sm_mhz_median"] if head else None, "sm_max_mhz": self.max_mhz,
+               "reasons": sorted(set((nv or {}).get("reasons", [])) |
+                                 set((smi or {}).get("reasons", []))),
+               "source": ("nvidia-smi, 50 ms" if head is smi else "nvml, 5 ms") if head else None,
+               "nvml": nv, "nvidia_smi": smi}
+        if head and ms_per_step:
+            out["ms_x_mhz"] = ms_per_step * head["sm_mhz_median"]
+        return out
 
 
 def max_over_ranks(values, device):
@@ -170,20 +192,22 @@ def _dist():
 
 
 # ---------------------------------------------------------------- CPU oracle leg
-def oracle_sample(wl, target_s: float = 12.0, max_tokens: int | None = None):
-    """Time the CPU oracle on a token sample of the workload: all five steps
-    for the first S tokens (route, layout, permute, GEMM, combine).  S grows
-    (doubling) until the oracle's own time reaches ``target_s``/2; expert
-    weights are drawn on the host outside the timed calls."""
-    import oracle
-    logits_all = workloads.router_logits(wl)
-    x_all = workloads.hidden_states(wl)
-    cache = {}
+class OracleSample:
+    """The CPU oracle run on the first S tokens of a workload: all five
+    steps (route, layout, permute, GEMM, combine) in fp64.  The touched
+    experts' weights are drawn on the host once, outside the timed calls,
+    and kept for later runs of the same or a smaller sample."""
 
-    def run(S):
-        sub = wl.replace(T=S)
-        lg, x = logits_all[:S].contiguous(), x_all[:S].contiguous()
-        t0 = time.perf_counter()
+    def __init__(self, wl):
+        self.wl = wl
+        self.logits = workloads.router_logits(wl)
+        self.x = workloads.hidden_states(wl)
+        self.cache = {}
+
+    def _route_layout(self, S):
+        import oracle
+        wl = self.wl
+        lg, x = self.logits[:S].contiguous(), self.x[:S].contiguous()
         if wl.route_groups:
             idx, w = oracle.route_topk_grouped(lg, wl.k, wl.route_groups, wl.route_max_groups)
         else:
@@ -193,22 +217,41 @@ def oracle_sample(wl, target_s: float = 12.0, max_tokens: int | None = None):
         else:
             lay = oracle.dispatch_layout_capacity(
                 idx, wl.E, wl.W, oracle.capacity_rows(S, wl.k, wl.E, wl.capacity_factor))
+        return x, w, lay
+
+    def prepare(self, S):
+        """Draws (untimed) the weights of every expert the first S tokens
+        reach."""
+        import concurrent.futures as cf
+        _, _, lay = self._route_layout(S)
+        cnt = lay["expert_counts"].tolist()
+        need = [e for e in range(self.wl.E) if cnt[e] > 0 and e not in self.cache]
+        draw = lambda e: (e, workloads.expert_w13(self.wl, e), workloads.expert_w2(self.wl, e))
+        with cf.ThreadPoolExecutor(max(1, min(16, os.cpu_count() or 1))) as pool:
+            for e, a, b in pool.map(draw, need):
+                self.cache[e] = (a, b)
+
+    def run(self, S):
+        """Seconds of oracle work for the first S tokens (weight drawing
+        excluded)."""
+        import oracle
+        wl = self.wl
+        self.prepare(S)
+        t0 = time.perf_counter()
+        x, w, lay = self._route_layout(S)
         xp, sc = oracle.permute(x, wl.k, lay["pair_of_slot"], wl.payload)
         el = time.perf_counter() - t0
         off = lay["expert_offsets"].tolist()
         cnt = lay["expert_counts"].tolist()         # rows each expert computes
         touched = [e for e in range(wl.E) if cnt[e] > 0]
-        for e in touched:
-            if e not in cache:
-                cache[e] = (workloads.expert_w13(wl, e), workloads.expert_w2(wl, e))
         y = torch.zeros(xp.shape[0], wl.H, dtype=torch.float64)
         for i in range(0, len(touched), 32):
             grp = touched[i:i + 32]
             rows = torch.cat([torch.arange(off[e], off[e] + cnt[e]) for e in grp])
             oe = torch.tensor([0] + list(torch.tensor([cnt[e] for e in grp])
                                          .cumsum(0).tolist()), dtype=torch.int32)
-            a13 = torch.stack([cache[e][0] for e in grp])
-            a2 = torch.stack([cache[e][1] for e in grp])
+            a13 = torch.stack([self.cache[e][0] for e in grp])
+            a2 = torch.stack([self.cache[e][1] for e in grp])
             t0 = time.perf_counter()
             _, ye, _ = oracle.grouped_gemm(xp[rows].contiguous(),
                                            sc[rows].contiguous() if sc is not None else None,
@@ -220,38 +263,59 @@ def oracle_sample(wl, target_s: float = 12.0, max_tokens: int | None = None):
         el += time.perf_counter() - t0
         return el
 
-    S = 4
-    el = run(S)
-    cap = wl.T if max_tokens is None else min(wl.T, max_tokens)
-    while el < target_s / 2 and S < cap:
-        S = min(cap, S * 2)
-        cache_keep = len(cache)
-        el = run(S)
-        if len(cache) > 400 and cache_keep:
-            cache.clear()
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    return {"value": S / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+    def tokens_for(self, seconds, probe=8):
+        """Sample size whose oracle time is about ``seconds`` (the oracle's
+        time is linear in the tokens: one probe run, then scaled)."""
+        S = min(self.wl.T, probe)
+        el = self.run(S)
+        return max(1, min(self.wl.T, int(S * seconds / max(el, 1e-6))))
+
+
+def _cores():
+    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+
+def oracle_sample(wl, target_s: float = 12.0, max_tokens: int | None = None):
+    """cpu_baseline of the GPU line: the oracle on about ``target_s`` seconds
+    of work (a token sample of the workload)."""
+    o = OracleSample(wl)
+    S = o.tokens_for(target_s)
+    if max_tokens is not None:
+        S = min(S, max_tokens)
+    el = o.run(S)
+    return {"value": S / el, "unit": "tokens/s", "cores": _cores(), "kind": "oracle",
             "sample": f"first {S} of {wl.T} tokens of workload {wl.name}, all five steps "
                       f"(fp64 C oracle, OpenMP over GEMM rows); {el:.2f} s of oracle time"}
 
 
 def run_reference(args, wl):
+    """The reference arm: the oracle as it stands, on rank 0 only.  Each of
+    the W + K steps is the same bounded token sample S, sized once so that
+    the whole run takes about ``--ref-budget`` seconds; ``ms_per_step`` is the
+    measured time of those S-token steps, and ``value`` = S / that time."""
     ws, rank, local = _dist()
     if rank != 0:
         return
-    times = []
+    o = OracleSample(wl)
+    per_step = min(args.ref_seconds, args.ref_budget / max(1, args.steps + args.warmup))
+    S = o.tokens_for(per_step)
+    o.prepare(S)
     for _ in range(args.warmup):
-        oracle_sample(wl, target_s=2.0, max_tokens=8)
-    res = None
-    for _ in range(args.steps):
-        res = oracle_sample(wl, target_s=args.ref_seconds)
-        times.append(1.0 / res["value"] * wl.T)
-    v = res["value"]
+        o.run(S)
+    times = [o.run(S) for _ in range(args.steps)]
+    sec = statistics.mean(times)
+    v = S / sec
+    sample = (f"first {S} of {wl.T} tokens of workload {wl.name} per step, all five steps "
+              f"(fp64 C oracle, OpenMP over GEMM rows); {args.steps} timed steps of "
+              f"{sec:.2f} s mean after {args.warmup} warm-up steps")
     line = {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * wl.T / v,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * sec,
+            "tokens_per_step": S, "ms_per_full_batch_extrapolated": 1000.0 * wl.T / v,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": _config(wl), "cpu_baseline": res,
+            "config": _config(wl),
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": _cores(), "kind": "oracle",
+                             "sample": sample},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -417,16 +481,54 @@ def run_ours(args, wl):
         for n in ["permute", "permute_standalone", "combine", "route_topk"]:
             g = kernels[n]["gbs"]
             kernels[n]["hbm_frac"] = g / peaks["hbm_gbs"] if g is not None else None
-        # the dominant kernel: the gate/up grouped GEMM (SwiGLU fused)
+        # The dominant kernel is the gate/up grouped GEMM (SwiGLU fused).  A
+        # step is a few ms and the timed region well under a second, so the
+        # burst bf16 peak is the denominator; the sustained figure (for
+        # kernels timed inside seconds-long runs) is kept beside it.
         achieved = tf(fl["gate_up"], avg["gemm_gate_up"])
-        # timed inside a long run of back-to-back steps under the 1000 W cap:
-        # the sustained bf16 peak is the denominator (burst fraction also given)
         roof = {"kernel": "grouped GEMM, gate/up + SwiGLU phase", "bound": "tensor",
-                "achieved": achieved, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops_sustained"],
-                "frac_of_burst": achieved / peaks["bf16_tflops"],
+                "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"],
+                "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
                 "traffic": _profile_traffic(wl), "algorithmic_flops_per_launch": fl["gate_up"],
-                "peak_source": peaks["source"] + " bf16 sustained (burst fraction also given)"}
+                "launch_us": avg["gemm_gate_up"] * 1e3,
+                "peak_source": peaks["source"] + " bf16 burst"}
+        # every other kernel against its own bound (same CUDA-event spans)
+        gb_w = traffic.gemm_phase_bytes(wl, rows, touched)
+        s8 = traffic.section8_bytes(wl, rows)
+        hbm = peaks["hbm_gbs"]
+
+        def hbm_entry(name, nbytes, us, what):
+            g = gbs(nbytes, us * 1e-3)
+            return {"kernel": name, "bound": "hbm", "achieved": g, "peak": hbm, "unit": "GB/s",
+                    "frac": g / hbm if g else None, "bytes": nbytes, "launch_us": us,
+                    "bytes_are": what}
+
+        others = [
+            {"kernel": "grouped GEMM, down phase", "bound": "tensor",
+             "achieved": tf(fl["down"], avg["gemm_down"]), "peak": peaks["bf16_tflops"],
+             "unit": "TFLOP/s", "frac": tf(fl["down"], avg["gemm_down"]) / peaks["bf16_tflops"],
+             "launch_us": avg["gemm_down"] * 1e3, "algorithmic_flops_per_launch": fl["down"],
+             "dram_bytes": gb_w["down"], "dram_gbs": gbs(gb_w["down"], avg["gemm_down"]),
+             "dram_frac": (gbs(gb_w["down"], avg["gemm_down"]) or 0) / hbm},
+            {"kernel": "grouped GEMM, gate/up + SwiGLU phase (DRAM view)", "bound": "hbm",
+             "achieved": gbs(gb_w["gate_up"], avg["gemm_gate_up"]), "peak": hbm, "unit": "GB/s",
+             "frac": (gbs(gb_w["gate_up"], avg["gemm_gate_up"]) or 0) / hbm,
+             "bytes": gb_w["gate_up"], "launch_us": avg["gemm_gate_up"] * 1e3},
+            {"kernel": "grouped GEMM, both phases", "bound": "tensor",
+             "achieved": tf(fl["total"], gemm_ms), "peak": peaks["bf16_tflops"],
+             "unit": "TFLOP/s", "frac": tf(fl["total"], gemm_ms) / peaks["bf16_tflops"],
+             "launch_us": gemm_ms * 1e3},
+            hbm_entry("permute (in the layer call)", kb["permute_layer"], avg["permute"] * 1e3,
+                      "bytes it moves"),
+            hbm_entry("permute (in the layer call)", s8["permute"], avg["permute"] * 1e3,
+                      "the send buffer's algorithmic bytes"),
+            hbm_entry("permute (standalone moe_permute)", kb["permute"], perm_alone_us,
+                      "the send buffer's algorithmic bytes"),
+            hbm_entry("combine", kb["combine"], avg["combine"] * 1e3, "bytes it moves"),
+            hbm_entry("combine", s8["combine"], avg["combine"] * 1e3,
+                      "algorithmic bytes with a bf16 (or the FP8) y"),
+        ]
         line = {
             "metric": METRIC, "value": whole_job_rate(wl.T, ws, ms), "unit": "tokens/s",
             "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -434,7 +536,7 @@ def run_ours(args, wl):
             "data": "synthetic", "config": dict(_config(wl), **_capacity_info(buf, dropped)),
             "layer_tokens_per_s": whole_job_rate(wl.T, ws, layer_ms),
             "layer_ms_excl_route": layer_ms,
-            "kernels": kernels, "roofline": roof,
+            "kernels": kernels, "roofline": roof, "roofline_other": others,
             "e2e": {"value": whole_job_rate(wl.T, ws, e2e), "unit": "tokens/s",
                     "h2d_bytes_per_step": h_logits.numel() * 4 + h_x.numel() * h_x.element_size(),
                     "d2h_bytes_per_step": h_out.numel() * h_out.element_size(),
@@ -443,7 +545,7 @@ def run_ours(args, wl):
                       "tokens_per_s": whole_job_rate(wl.T, ws, graph_us * 1e-3)},
             "gpu_launches": int(launches),
             "gpu_launches_per_step": int(launches) // max(args.steps, 1),
-            "clocks": clk.summary(),
+            "clocks": clk.summary(ms),
         }
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = oracle_sample(wl)
@@ -524,7 +626,10 @@ def main():
     ap.add_argument("--workload", default="dsv3", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ref-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-seconds", type=float, default=12.0,
+                    help="reference arm: at most this many seconds of oracle work per step")
+    ap.add_argument("--ref-budget", type=float, default=150.0,
+                    help="reference arm: about this many seconds for all warm-up and timed steps")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override T (smaller cases of the same kernels, for profiling)")
     ap.add_argument("--experts", type=int, default=None,

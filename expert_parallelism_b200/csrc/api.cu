@@ -42,6 +42,31 @@ static std::atomic<uint64_t> g_launches{0};
 void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 }  // namespace moe
 
+namespace moe {
+
+moe_status report_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return MOE_OK;
+    fprintf(stderr, "libmoe: CUDA error: %s\n", cudaGetErrorString(e));
+    return MOE_ERR_CUDA;
+}
+
+// The layout's argument rules, except for the caller workspace (shared by
+// every layout entry point).
+moe_status check_layout_args(const int32_t* topk_idx, int64_t T, int32_t k, int32_t E, int32_t W,
+                             const int32_t* expert_counts, const int32_t* expert_offsets,
+                             const int32_t* rank_offsets, const int32_t* slot_of_pair,
+                             const int32_t* pair_of_slot, const int32_t* dev_status) {
+    if (T < 0 || k < 1 || E < 1 || W < 1 || W > E || (E % W) != 0) return MOE_ERR_INVALID_ARG;
+    if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+    if (T * (int64_t)k >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
+    if (!expert_counts || !expert_offsets || !rank_offsets || !dev_status)
+        return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!topk_idx || !slot_of_pair || !pair_of_slot)) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+}  // namespace moe
+
 using namespace moe;
 
 namespace {
@@ -50,11 +75,7 @@ bool is_act_dtype(moe_dtype d) { return d == MOE_F32 || d == MOE_BF16; }
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
-moe_status cuda_status(cudaError_t e) {
-    if (e == cudaSuccess) return MOE_OK;
-    fprintf(stderr, "libmoe: CUDA error: %s\n", cudaGetErrorString(e));
-    return MOE_ERR_CUDA;
-}
+moe_status cuda_status(cudaError_t e) { return moe::report_cuda(e); }
 
 
 // Host-side validation of each step (no launch).  *noop is set when the
@@ -83,13 +104,11 @@ moe_status check_layout(const int32_t* topk_idx, int64_t T, int32_t k, int32_t E
                         const int32_t* rank_offsets, const int32_t* slot_of_pair,
                         const int32_t* pair_of_slot, const void* workspace,
                         size_t workspace_bytes, const int32_t* dev_status) {
-    if (T < 0 || k < 1 || E < 1 || W < 1 || W > E || (E % W) != 0) return MOE_ERR_INVALID_ARG;
-    if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
-    if (T * (int64_t)k >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
-    if (!expert_counts || !expert_offsets || !rank_offsets || !workspace || !dev_status)
-        return MOE_ERR_INVALID_ARG;
-    if (T > 0 && (!topk_idx || !slot_of_pair || !pair_of_slot)) return MOE_ERR_INVALID_ARG;
-    if (workspace_bytes < layout_workspace_bytes(T, k, E) || !aligned16(workspace))
+    const moe_status st = moe::check_layout_args(topk_idx, T, k, E, W, expert_counts,
+                                                 expert_offsets, rank_offsets, slot_of_pair,
+                                                 pair_of_slot, dev_status);
+    if (st != MOE_OK) return st;
+    if (!workspace || workspace_bytes < layout_workspace_bytes(T, k, E) || !aligned16(workspace))
         return MOE_ERR_INVALID_ARG;
     return MOE_OK;
 }
@@ -101,7 +120,9 @@ moe_status check_permute(const void* x, moe_dtype x_dtype, int64_t T, int32_t H,
     if (T < 0 || H < 1 || k < 1 || (H % 8) != 0) return MOE_ERR_INVALID_ARG;
     if (!is_act_dtype(x_dtype)) return MOE_ERR_INVALID_ARG;
     if (xp_dtype != x_dtype && xp_dtype != MOE_E4M3) return MOE_ERR_INVALID_ARG;
-    if (xp_dtype == MOE_E4M3 && ((H % 128) != 0 || !xp_scales)) return MOE_ERR_INVALID_ARG;
+    // the block scales leave the kernel as 16-byte vectors: 16-byte aligned
+    if (xp_dtype == MOE_E4M3 && ((H % 128) != 0 || !xp_scales || !aligned16(xp_scales)))
+        return MOE_ERR_INVALID_ARG;
     if (k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
     if (T == 0) return *noop = true, MOE_OK;
     if (!x || !slot_of_pair || !xp || !aligned16(x) || !aligned16(xp)) return MOE_ERR_INVALID_ARG;

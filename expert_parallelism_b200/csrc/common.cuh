@@ -138,4 +138,14 @@ struct gemm_gather {
 // Host-side count of kernel launches (reported by moe_launch_count).
 void note_launches(int n);
 
+// MOE_OK for cudaSuccess; otherwise prints the CUDA error and returns
+// MOE_ERR_CUDA (every entry point reports CUDA failures this way).
+moe_status report_cuda(cudaError_t e);
+
+// The dispatch layout's argument rules other than the caller workspace.
+moe_status check_layout_args(const int32_t* topk_idx, int64_t T, int32_t k, int32_t E, int32_t W,
+                             const int32_t* expert_counts, const int32_t* expert_offsets,
+                             const int32_t* rank_offsets, const int32_t* slot_of_pair,
+                             const int32_t* pair_of_slot, const int32_t* dev_status);
+
 }  // namespace moe

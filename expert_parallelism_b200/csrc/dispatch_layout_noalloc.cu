@@ -11,7 +11,10 @@
 // Every GPU that loads the library holds it until the process exits.  In
 // host code the array's name is only a host-side stand-in, not a device
 // address, so the set-up below asks the runtime for the real address once
-// per device (with that device current) and passes it to the kernels.
+// per device (with that device current), again if the device's current
+// context changes, and passes it to the kernels.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -32,19 +35,59 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
-void* g_scratch_ptr[kMaxDevices] = {};
 
-// Device address of g_layout_scratch on the current device (nullptr on error).
-void* scratch_on_current_device() {
+// What the set-up found on each device: the array's address, valid in the
+// context that was current when it was looked up.
+struct ScratchAddr {
+    CUcontext ctx;
+    void* ptr;
+};
+ScratchAddr g_scratch[kMaxDevices] = {};
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+// cuCtxGetCurrent from the driver, through the runtime (looked up once).
+CtxGetCurrentFn ctx_get_current() {
+    static const CtxGetCurrentFn fn = [] {
+        void* q = nullptr;
+        cudaDriverEntryPointQueryResult r;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &q, cudaEnableDefault, &r) ==
+                cudaSuccess &&
+            r == cudaDriverEntryPointSuccess)
+            return (CtxGetCurrentFn)q;
+        return (CtxGetCurrentFn) nullptr;
+    }();
+    return fn;
+}
+
+// Device address of g_layout_scratch on the current device, looked up (with
+// that device current) on the first call and again whenever the current
+// context is not the one of the last lookup (after cudaDeviceReset, or with
+// another context made current).  Returns the CUDA error of a failed lookup.
+cudaError_t scratch_on_current_device(void** out) {
+    *out = nullptr;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    const CtxGetCurrentFn get = ctx_get_current();
+    if (!get) return cudaErrorInitializationError;
+    CUcontext ctx = nullptr;
+    if (get(&ctx) != CUDA_SUCCESS) return cudaErrorInitializationError;
     std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (!g_scratch_ptr[dev]) {
+    ScratchAddr& s = g_scratch[dev];
+    if (!s.ptr || !ctx || s.ctx != ctx) {
+        // the lookup also brings up the runtime's context on this device
+        // when none is current yet; the context is read again after it
         void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_layout_scratch) != cudaSuccess) return nullptr;
-        g_scratch_ptr[dev] = p;
+        e = cudaGetSymbolAddress(&p, g_layout_scratch);
+        if (e != cudaSuccess) return e;
+        if (get(&ctx) != CUDA_SUCCESS || !ctx) return cudaErrorInitializationError;
+        s.ctx = ctx;
+        s.ptr = p;
     }
-    return g_scratch_ptr[dev];
+    *out = s.ptr;
+    return cudaSuccess;
 }
 
 }  // namespace
@@ -58,22 +101,21 @@ moe_status moe_dispatch_layout_noalloc(const int32_t* topk_idx, int64_t T, int32
                                        int32_t* expert_offsets, int32_t* rank_offsets,
                                        int32_t* slot_of_pair, int32_t* pair_of_slot,
                                        int32_t* dev_status, void* stream) {
-    if (T < 0 || k < 1 || E < 1 || W < 1 || W > E || (E % W) != 0) return MOE_ERR_INVALID_ARG;
-    if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
-    if (T * (int64_t)k >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
-    if (!expert_counts || !expert_offsets || !rank_offsets || !dev_status)
-        return MOE_ERR_INVALID_ARG;
-    if (T > 0 && (!topk_idx || !slot_of_pair || !pair_of_slot)) return MOE_ERR_INVALID_ARG;
+    const moe_status st = moe::check_layout_args(topk_idx, T, k, E, W, expert_counts,
+                                                 expert_offsets, rank_offsets, slot_of_pair,
+                                                 pair_of_slot, dev_status);
+    if (st != MOE_OK) return st;
     if (moe::layout_workspace_bytes(T, k, E) > kNoAllocScratchBytes) return MOE_ERR_UNSUPPORTED;
-    void* scratch = scratch_on_current_device();
-    if (!scratch) return MOE_ERR_CUDA;
+    void* scratch = nullptr;
+    cudaError_t e = scratch_on_current_device(&scratch);
     // The scratch keeps the previous call's contents; the first kernel of
     // the layout clears the look-back flags and the ticket itself, and the
     // rest is fully overwritten before it is read.
-    const cudaError_t e = moe::launch_dispatch_layout(
-        topk_idx, T, k, E, W, -1, expert_counts, expert_offsets, rank_offsets, slot_of_pair,
-        pair_of_slot, nullptr, scratch, dev_status, (cudaStream_t)stream);
-    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    if (e == cudaSuccess)
+        e = moe::launch_dispatch_layout(topk_idx, T, k, E, W, -1, expert_counts, expert_offsets,
+                                        rank_offsets, slot_of_pair, pair_of_slot, nullptr, scratch,
+                                        dev_status, (cudaStream_t)stream);
+    return moe::report_cuda(e);
 }
 
 }  // extern "C"

@@ -50,6 +50,7 @@
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
+#include "host_launch.cuh"
 #include "tcgen05.cuh"
 #include "tile_schedule.cuh"
 
@@ -373,65 +374,33 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
-    }
-    return fn;
-}
-
-// Tiled bf16 tensor map, 128-byte swizzle, zero fill out of bounds.
 static bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
                      const cuuint64_t* strides_bytes, const cuuint32_t* box) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint32_t elem[4] = {1, 1, 1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
-                    dims, strides_bytes, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    return make_bf16_map(m, base, rank, dims, strides_bytes, box);
 }
 
-static void cluster_attr(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr, int ncta) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)ncta;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-}
-
-// CTA groups of NCTA that fit on the device at once (one CTA per SM).
+// CTA groups of NCTA that fit on the current device at once (one CTA per
+// SM), cached per device.
 template <bool GLU, typename OutT, int NCTA>
 static int resident_units(size_t smem) {
-    static int cached = -1;
-    if (cached > 0) return cached;
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    int n = sms / NCTA;
-    if (NCTA > 1) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)(n * NCTA));
-        cfg.blockDim = dim3(kThreads);
-        cfg.dynamicSmemBytes = smem;
-        cudaLaunchAttribute attr[1];
-        cluster_attr(cfg, attr, NCTA);
-        int c = 0;
-        if (cudaOccupancyMaxActiveClusters(&c, grouped_gemm_tc_kernel<GLU, OutT, NCTA>, &cfg) ==
-                cudaSuccess &&
-            c > 0)
-            n = c;
-    }
-    cached = n;
-    return n;
+    struct Tag {};
+    return PerDeviceInt<Tag>::get([smem] {
+        int n = current_device_sm_count() / NCTA;
+        if (NCTA > 1) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3((unsigned)(n * NCTA));
+            cfg.blockDim = dim3(kThreads);
+            cfg.dynamicSmemBytes = smem;
+            cudaLaunchAttribute attr[1];
+            set_cluster_attr(cfg, attr, NCTA);
+            int c = 0;
+            if (cudaOccupancyMaxActiveClusters(&c, grouped_gemm_tc_kernel<GLU, OutT, NCTA>,
+                                               &cfg) == cudaSuccess &&
+                c > 0)
+                n = c;
+        }
+        return n;
+    });
 }
 
 template <bool GLU, typename OutT, int NCTA>
@@ -448,7 +417,7 @@ static cudaError_t launch_phase(const CUtensorMap& ma, const CUtensorMap& mb, co
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
-    cluster_attr(cfg, attr, NCTA);
+    set_cluster_attr(cfg, attr, NCTA);
     return cudaLaunchKernelEx(&cfg, kern, ma, mb, p);
 }
 

@@ -53,6 +53,7 @@
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
+#include "host_launch.cuh"
 #include "tcgen05.cuh"
 #include "tile_schedule.cuh"
 
@@ -615,62 +616,31 @@ __global__ void __launch_bounds__(threads_of<GATHER>(), 1)
 }
 
 // ---------------------------------------------------------------- host side
-static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void* q = nullptr;
-        cudaDriverEntryPointQueryResult r;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &q, cudaEnableDefault, &r) ==
-                cudaSuccess &&
-            r == cudaDriverEntryPointSuccess)
-            fn = (PFN_cuTensorMapEncodeTiled_v12000)q;
-    }
-    return fn;
-}
-
-// Tiled bf16 tensor map, 128-byte swizzle, zero fill out of bounds.
 static bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
                      const cuuint64_t* strides_bytes, const cuuint32_t* box) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint32_t elem[4] = {1, 1, 1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
-                    dims, strides_bytes, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    return make_bf16_map(m, base, rank, dims, strides_bytes, box);
 }
 
-static void pair_cluster(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-}
-
+// CTA pairs of this kernel that fit on the current device at once (one CTA
+// per SM), cached per device.
 template <bool GLU, typename OutT, bool GATHER>
 static int resident_pairs(size_t smem) {
-    static int cached = -1;
-    if (cached > 0) return cached;
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    int n = sms / 2;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(2 * n));
-    cfg.blockDim = dim3(threads_of<GATHER>());
-    cfg.dynamicSmemBytes = smem;
-    cudaLaunchAttribute attr[1];
-    pair_cluster(cfg, attr);
-    int c = 0;
-    if (cudaOccupancyMaxActiveClusters(&c, grouped_gemm_swap_kernel<GLU, OutT, GATHER>, &cfg) ==
-            cudaSuccess &&
-        c > 0)
-        n = c;
-    cached = n;
-    return n;
+    struct Tag {};
+    return PerDeviceInt<Tag>::get([smem] {
+        int n = current_device_sm_count() / 2;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(2 * n));
+        cfg.blockDim = dim3(threads_of<GATHER>());
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        set_cluster_attr(cfg, attr, 2);
+        int c = 0;
+        if (cudaOccupancyMaxActiveClusters(&c, grouped_gemm_swap_kernel<GLU, OutT, GATHER>,
+                                           &cfg) == cudaSuccess &&
+            c > 0)
+            n = c;
+        return n;
+    });
 }
 
 template <bool GLU, typename OutT, bool GATHER = false>
@@ -687,7 +657,7 @@ static cudaError_t launch_phase(const CUtensorMap& mw, const CUtensorMap* mt, co
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
-    pair_cluster(cfg, attr);
+    set_cluster_attr(cfg, attr, 2);
     return cudaLaunchKernelEx(&cfg, kern, mw, mt[0], mt[1], mt[2], p);
 }
 

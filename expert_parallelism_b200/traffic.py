@@ -60,3 +60,31 @@ def gemm_flops(wl: Workload, rows: int | None = None) -> dict:
 def touched_weight_bytes(wl: Workload, experts_touched: int) -> int:
     """Expert-weight bytes a pass must read at least once."""
     return experts_touched * 3 * wl.I * wl.H * ELEM_BYTES[wl.wdt]
+
+
+def section8_bytes(wl: Workload, rows: int | None = None) -> dict:
+    """The permute's and the combine's algorithmic bytes as the step table
+    counts them: the send buffer (x read once, the payload and its block
+    scales written once per routed row), and the combine reading each routed
+    row of y once in a 2-byte type (1 byte plus block scales for the FP8
+    combine payload) and writing out once.  Whatever y's storage dtype, the
+    combine's fraction of peak on these bytes is what the step's target
+    refers to."""
+    T, H, k = wl.T, wl.H, wl.k
+    N = wl.N if rows is None else rows
+    xb, pb = ELEM_BYTES[wl.act], ELEM_BYTES[wl.payload]
+    scales = N * (H // 128) * 4 if wl.payload == "e4m3" else 0
+    y_row = H + (H // 128) * 4 if wl.ydt == "e4m3" else 2 * H
+    return {"permute": T * H * xb + N * H * pb + scales,
+            "combine": N * y_row + T * H * xb}
+
+
+def gemm_phase_bytes(wl: Workload, rows: int, experts_touched: int) -> dict:
+    """DRAM bytes each GEMM phase must move at least: its weights once per
+    touched expert, its row operand once, its output once (h in the weight
+    dtype; y in its storage dtype, plus block scales for an FP8 y)."""
+    wb = ELEM_BYTES[wl.wdt]
+    H, I = wl.H, wl.I
+    y_row = H + (H // 128) * 4 if wl.ydt == "e4m3" else H * ELEM_BYTES[wl.ydt]
+    return {"gate_up": experts_touched * 2 * I * H * wb + rows * H * wb + rows * I * wb,
+            "down": experts_touched * H * I * wb + rows * I * wb + rows * y_row}

@@ -218,10 +218,15 @@ moe_status moe_dispatch_layout_capacity(const int32_t* topk_idx, int64_t T, int3
  *     MOE_ERR_UNSUPPORTED; moe_dispatch_layout handles those.
  *   - It allocates nothing.  The first call on each device looks up the
  *     array's device address (cudaGetSymbolAddress, with that device
- *     current); make that first call before any stream capture.
+ *     current), and looks it up again whenever the context current on the
+ *     device is not the one of the last lookup (after cudaDeviceReset, or
+ *     with another context made current); make the first call in each
+ *     context before any stream capture.  A CUDA error in the lookup or the
+ *     launch returns MOE_ERR_CUDA (and is printed, as for every entry point).
  *   - Every call shares the one array, so calls that overlap on the GPU
  *     (on different streams, or from different threads) race: serialise
  *     them, e.g. on one stream.  Nothing needs clearing between calls.
+ *   - Its argument rules are moe_dispatch_layout's (without the workspace).
  */
 size_t moe_dispatch_layout_noalloc_max_scratch_bytes(void);
 moe_status moe_dispatch_layout_noalloc(const int32_t* topk_idx, int64_t T, int32_t k, int32_t E,
@@ -246,9 +251,10 @@ moe_status moe_dispatch_layout_noalloc(const int32_t* topk_idx, int64_t T, int32
  *             row, scale = amax/448 (fp32 IEEE division; 1 if amax == 0)
  *             and q = e4m3(x/scale) (fp32 IEEE division, round to nearest
  *             even, saturating to +-448).  Requires H % 128 == 0.
- *   xp_scales [T*k, H/128] fp32, written for MOE_E4M3, else ignored (may
- *             be NULL).
- * Requires H % 8 == 0, H > 0, k >= 1.
+ *   xp_scales [T*k, H/128] fp32, written for MOE_E4M3 (16-byte aligned: a
+ *             slot's scales are stored as 16-byte vectors), else ignored
+ *             (may be NULL).
+ * Requires H % 8 == 0, H > 0, k >= 1; x and xp 16-byte aligned.
  */
 moe_status moe_permute(const void* x, moe_dtype x_dtype, int64_t T, int32_t H, int32_t k,
                        const int32_t* slot_of_pair, void* xp, moe_dtype xp_dtype,
@@ -436,7 +442,7 @@ typedef struct moe_layer_buffers {
     void* layout_workspace;  /* moe_dispatch_layout_workspace_bytes(T, k, E) */
     size_t layout_workspace_bytes;
     void* xp;                /* [S, H] payload */
-    float* xp_scales;        /* [S, H/128] (FP8 payload only) */
+    float* xp_scales;        /* [S, H/128] (FP8 payload only), 16-byte aligned */
     void* h;                 /* [S, I] in w_dtype */
     void* y;                 /* [S, H] in y_dtype */
     float* y_scales;         /* [S, H/128] (FP8 y only) */

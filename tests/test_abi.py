@@ -122,6 +122,10 @@ def test_permute_combine_gemm_reject_before_launch(lib):
     assert p(FAKE, moe.MOE_BF16, 10, 128, 2, FAKE, FAKE, moe.MOE_F32, None, None) == 1    # cast
     assert p(ctypes.c_void_p(4098), moe.MOE_BF16, 10, 128, 2, FAKE, FAKE, moe.MOE_BF16, None,
              None) == 1                                                                 # align
+    # FP8 block scales go out as 16-byte vectors: a scale buffer at an odd
+    # float offset (a sliced tensor, say) is refused instead of faulting
+    assert p(FAKE, moe.MOE_BF16, 10, 512, 2, FAKE, FAKE, moe.MOE_E4M3, ctypes.c_void_p(4100),
+             None) == 1
     c = lib.moe_combine
     assert c(FAKE, moe.MOE_E4M3, None, FAKE, FAKE, 10, 2, 128, FAKE, moe.MOE_BF16, None) == 1  # scales
     assert c(FAKE, moe.MOE_E4M3, FAKE, FAKE, FAKE, 10, 2, 136, FAKE, moe.MOE_BF16, None) == 1  # H%128
@@ -199,6 +203,19 @@ def test_all_reduce_form_calls_reject_before_launch(lib):
     assert lib.moe_layer_forward(FAKE, FAKE, moe.MOE_BF16, 10, 128, 8, 2, 2, 64, FAKE, FAKE,
                                  moe.MOE_BF16, moe.MOE_BF16, moe.MOE_F32, ctypes.byref(o),
                                  ctypes.byref(cb), FAKE, None, None) == 1
+
+
+def test_layer_call_rejects_misaligned_fp8_scales(lib):
+    """The layer call checks the permute's scale buffer as moe_permute does."""
+    T, H, E, k, W, I = 10, 512, 8, 2, 2, 64
+    lw = moe.moe_dispatch_layout_workspace_bytes(T, k, E)
+    gw = T * k * H * 2                                 # the FP8 payload's bf16 rows
+    fields = [FAKE] * 8 + [lw] + [FAKE] * 6 + [gw] + [FAKE, None, None]
+    fields[10] = ctypes.c_void_p(4100)                 # xp_scales, 4-byte aligned only
+    cb = moe.LayerBuffersC(*fields)
+    assert lib.moe_layer_forward(FAKE, FAKE, moe.MOE_BF16, T, H, E, k, W, I, FAKE, FAKE,
+                                 moe.MOE_BF16, moe.MOE_E4M3, moe.MOE_F32, None, ctypes.byref(cb),
+                                 FAKE, None, None) == 1
 
 
 def test_fused_gather_needs_one_workspace_row_per_token(lib):
