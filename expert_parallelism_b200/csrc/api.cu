@@ -35,6 +35,8 @@ cudaError_t launch_grouped_gemm_tc(const __nv_bfloat16*, const int32_t*, const i
 bool grouped_gemm_tc_uses_swap(int64_t n_rows, int n_experts, moe_dtype y_dtype);
 cudaError_t launch_quantize_tokens_e4m3(const void*, moe_dtype, int64_t, int, __nv_bfloat16*,
                                        cudaStream_t);
+size_t layout_wait_selftest_bytes();
+cudaError_t launch_layout_wait_selftest(void*, uint64_t, int32_t*, cudaStream_t);
 }  // namespace moe
 
 namespace moe {
@@ -524,6 +526,19 @@ moe_status moe_check_status(int32_t* dev_status, void* stream) {
 }
 
 uint64_t moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+size_t moe_diag_layout_wait_timeout_workspace_bytes(void) { return layout_wait_selftest_bytes(); }
+
+moe_status moe_diag_layout_wait_timeout(void* workspace, size_t workspace_bytes,
+                                        uint64_t wait_limit_ns, int32_t* dev_status,
+                                        void* stream) {
+    if (!workspace || !dev_status || !aligned16(workspace) ||
+        workspace_bytes < layout_wait_selftest_bytes())
+        return MOE_ERR_INVALID_ARG;
+    if (wait_limit_ns > kSpinLimitNs) return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_layout_wait_selftest(workspace, wait_limit_ns, dev_status,
+                                                   (cudaStream_t)stream));
+}
 
 const char* moe_status_str(moe_status s) {
     switch (s) {

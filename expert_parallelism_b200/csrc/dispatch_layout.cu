@@ -99,9 +99,12 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_hist_kernel(
     for (int e = threadIdx.x; e < E; e += blockDim.x) counts[(int64_t)e * nt + b] = hist[e];
 }
 
+// wait_limit_ns bounds each chunk's look-back wait (the library passes
+// kSpinLimitNs); a chunk number at or past nchunks does nothing.
 __global__ void __launch_bounds__(kScanThreads) layout_scan_kernel(
     const int32_t* __restrict__ counts, int32_t* __restrict__ base, int64_t L,
-    unsigned long long* status, int32_t* ticket, int32_t* dev_status) {
+    unsigned long long* status, int64_t nchunks, int32_t* ticket, int32_t* dev_status,
+    uint64_t wait_limit_ns) {
     __shared__ int32_t s_chunk, s_prefix;
     __shared__ int32_t s_warp[kScanThreads / kWarp];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -110,6 +113,7 @@ __global__ void __launch_bounds__(kScanThreads) layout_scan_kernel(
     if (tid == 0) s_chunk = atomicAdd(ticket, 1);
     __syncthreads();
     const int64_t c = s_chunk;
+    if (c >= nchunks) return;
     const int64_t i0 = c * kScanChunk + (int64_t)tid * kScanItems;
     int32_t v[kScanItems];
     int32_t mine = 0;
@@ -138,13 +142,13 @@ __global__ void __launch_bounds__(kScanThreads) layout_scan_kernel(
             atomicExch(&status[0], kFlagInclusive | (uint32_t)total);
         } else {
             atomicExch(&status[c], kFlagAggregate | (uint32_t)total);
-            const uint64_t deadline = global_timer_ns() + kSpinLimitNs;
+            const uint64_t deadline = global_timer_ns() + wait_limit_ns;
             int64_t j = c - 1;
             while (j >= 0) {
                 const unsigned long long st = *((volatile unsigned long long*)&status[j]);
                 const unsigned long long flag = st & 0xFFFFFFFF00000000ull;
                 if (flag == 0ull) {
-                    if (global_timer_ns() > deadline) {
+                    if (global_timer_ns() >= deadline) {
                         flag_status(dev_status, MOE_DEV_TIMEOUT);
                         break;
                     }
@@ -305,13 +309,47 @@ cudaError_t launch_dispatch_layout(const int32_t* idx, int64_t T, int k, int E, 
     }
     layout_hist_kernel<<<(unsigned)w.nt, kLayoutThreads, hist_smem, s>>>(
         idx, N, E, w.nt, w.counts, w.status, w.nchunks, w.ticket, dev_status);
-    layout_scan_kernel<<<(unsigned)w.nchunks, kScanThreads, 0, s>>>(w.counts, w.base, w.L,
-                                                                    w.status, w.ticket,
-                                                                    dev_status);
+    layout_scan_kernel<<<(unsigned)w.nchunks, kScanThreads, 0, s>>>(
+        w.counts, w.base, w.L, w.status, w.nchunks, w.ticket, dev_status, kSpinLimitNs);
     layout_scatter_kernel<<<(unsigned)w.nt, kLayoutThreads, scatter_smem, s>>>(
         idx, N, E, W, w.nt, w.counts, w.base, w.L, C, expert_counts, expert_offsets,
         rank_offsets, slot_of_pair, pair_of_slot, n_dropped);
     note_launches(3);
+    return cudaGetLastError();
+}
+
+// Look-back state of a two-chunk scan in which chunk 0 never runs: the
+// ticket starts at 1, so the one CTA launched becomes chunk 1 and waits for
+// status[0], which nothing sets.  Counts are zero.
+__global__ void layout_wait_selftest_init_kernel(unsigned long long* status, int32_t* ticket,
+                                                 int32_t* counts, int64_t L) {
+    for (int64_t i = threadIdx.x; i < L; i += blockDim.x) counts[i] = 0;
+    if (threadIdx.x < 2) status[threadIdx.x] = 0ull;
+    if (threadIdx.x == 0) *ticket = 1;
+}
+
+size_t layout_wait_selftest_bytes() {
+    const int64_t L = 2 * kScanChunk;
+    return align_up(2 * 8, 16) + 16 + 2 * align_up((size_t)L * 4, 16);
+}
+
+// The scan kernel itself, on that state, with the given wait limit: its
+// look-back wait runs out and MOE_DEV_TIMEOUT is OR-ed into dev_status.
+cudaError_t launch_layout_wait_selftest(void* workspace, uint64_t wait_limit_ns,
+                                        int32_t* dev_status, cudaStream_t s) {
+    const int64_t L = 2 * kScanChunk;
+    char* p = (char*)workspace;
+    unsigned long long* status = (unsigned long long*)p;
+    p += align_up(2 * 8, 16);
+    int32_t* ticket = (int32_t*)p;
+    p += 16;
+    int32_t* counts = (int32_t*)p;
+    p += align_up((size_t)L * 4, 16);
+    int32_t* base = (int32_t*)p;
+    layout_wait_selftest_init_kernel<<<1, 256, 0, s>>>(status, ticket, counts, L);
+    layout_scan_kernel<<<1, kScanThreads, 0, s>>>(counts, base, L, status, 2, ticket, dev_status,
+                                                  wait_limit_ns);
+    note_launches(2);
     return cudaGetLastError();
 }
 

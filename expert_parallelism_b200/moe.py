@@ -50,6 +50,8 @@ SIGNATURES = {
     "moe_check_status": ([_P, _P], _I),
     "moe_status_str": ([_I], ctypes.c_char_p),
     "moe_launch_count": ([], ctypes.c_uint64),
+    "moe_diag_layout_wait_timeout_workspace_bytes": ([], _SZ),
+    "moe_diag_layout_wait_timeout": ([_P, _SZ, ctypes.c_uint64, _P, _P], _I),
 }
 
 
@@ -218,6 +220,14 @@ def moe_reduce_partials(partials, out, stream=None):
 def moe_check_status(dev_status, stream=None) -> int:
     """Synchronises the stream; returns the raw status code (0 = OK)."""
     return int(load_library().moe_check_status(_ptr(dev_status), _stream(stream)))
+
+
+def moe_diag_layout_wait_timeout(workspace, wait_limit_ns, dev_status, stream=None):
+    """Runs the layout scan on a flag that nothing sets; its bounded wait
+    gives up after ``wait_limit_ns`` and records MOE_DEV_TIMEOUT."""
+    _check("moe_diag_layout_wait_timeout", load_library().moe_diag_layout_wait_timeout(
+        _ptr(workspace), workspace.numel() * workspace.element_size(), wait_limit_ns,
+        _ptr(dev_status), _stream(stream)))
 
 
 def moe_status_str(code: int) -> str:

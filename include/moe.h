@@ -491,6 +491,26 @@ const char* moe_status_str(moe_status s);
  * process (all devices, all streams), counted on the host at launch. */
 uint64_t moe_launch_count(void);
 
+/*
+ * moe_diag_layout_wait_timeout -- diagnostics for failure detection: runs
+ * the dispatch layout's scan kernel (the one moe_dispatch_layout launches)
+ * on a two-chunk look-back state in which the first chunk never publishes
+ * its count, so the second chunk's bounded wait on that flag can only run
+ * out.  After wait_limit_ns of device time (globaltimer) the kernel gives up,
+ * OR-s MOE_DEV_TIMEOUT into dev_status and returns; moe_check_status then
+ * reports MOE_ERR_TIMEOUT.  Nothing faults, traps or hangs, and the context
+ * stays usable.  The library's own calls bound this wait at 2 s; here the
+ * limit is the caller's, at most 2 s (MOE_ERR_INVALID_ARG above that).
+ *
+ *   workspace  device scratch of moe_diag_layout_wait_timeout_workspace_bytes()
+ *              bytes, 16-byte aligned, clobbered.
+ *   dev_status int32 device word.
+ */
+size_t moe_diag_layout_wait_timeout_workspace_bytes(void);
+moe_status moe_diag_layout_wait_timeout(void* workspace, size_t workspace_bytes,
+                                        uint64_t wait_limit_ns, int32_t* dev_status,
+                                        void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -99,10 +99,38 @@ class GpuLayer:
         return moe.moe_check_status(b.dev_status)
 
 
-def sample_rows(lay: dict, T: int, k: int, n_tokens: int, seed: int = 0):
-    """Slots of a seeded token sample (all kept pairs of each), plus the
-    first and last computed slot of every non-empty expert (the ragged
-    tails).  Works for the dropless and the fixed-capacity layouts."""
+def full_experts(lay: dict, n: int = 8, seed: int = 0):
+    """Experts whose every row a full-size check compares: the largest
+    expert; the largest one whose rows make one pass with a second chunk
+    (257..320 rows); the largest one that needs several passes (> 320 rows);
+    then seeded picks among the other non-empty experts, up to ``n``."""
+    cnt = lay["expert_counts"].numpy()
+    order = [int(e) for e in np.argsort(-cnt, kind="stable") if cnt[e] > 0]
+    chosen = []
+
+    def add(e):
+        if e is not None and e not in chosen and len(chosen) < n:
+            chosen.append(e)
+
+    if order:
+        add(order[0])
+    add(next((e for e in order if 256 < cnt[e] <= 320), None))
+    add(next((e for e in order if cnt[e] > 320), None))
+    rest = [e for e in order if e not in chosen]
+    rng = np.random.default_rng(seed + 1)
+    for e in rng.permutation(rest)[:max(0, n - len(chosen))]:
+        add(int(e))
+    return chosen
+
+
+def sample_rows(lay: dict, T: int, k: int, n_tokens: int, seed: int = 0, per_expert: int = 8,
+                n_full: int = 8):
+    """Slots a full-size check compares: every kept pair of a seeded token
+    sample; the first and last computed row of every non-empty expert (the
+    ragged tails) and ``per_expert`` more seeded rows of each; and every row
+    of ``n_full`` experts (``full_experts``).  Returns (tokens, slot mask,
+    those experts).  Works for the dropless and the fixed-capacity
+    layouts."""
     rng = np.random.default_rng(seed)
     toks = np.sort(rng.choice(T, size=min(n_tokens, T), replace=False))
     sop = lay["slot_of_pair"].numpy().reshape(T, k)
@@ -115,7 +143,11 @@ def sample_rows(lay: dict, T: int, k: int, n_tokens: int, seed: int = 0):
         if cnt[e] > 0:
             mask[off[e]] = True
             mask[off[e] + cnt[e] - 1] = True
-    return torch.from_numpy(toks), torch.from_numpy(mask)
+            mask[off[e] + rng.choice(cnt[e], size=min(per_expert, cnt[e]), replace=False)] = True
+    experts = full_experts(lay, n_full, seed)
+    for e in experts:
+        mask[off[e]:off[e] + cnt[e]] = True
+    return torch.from_numpy(toks), torch.from_numpy(mask), experts
 
 
 def oracle_gemm_rows(wl, xp, sc, offsets, mask, w13=None, w2=None, batch=16):

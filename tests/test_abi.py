@@ -231,6 +231,17 @@ def test_fused_gather_needs_one_workspace_row_per_token(lib):
                                  ctypes.byref(cb), FAKE, None, None) == 1
 
 
+def test_wait_timeout_diagnostic_rejects_before_launch(lib):
+    f = lib.moe_diag_layout_wait_timeout
+    n = lib.moe_diag_layout_wait_timeout_workspace_bytes()
+    assert n > 0 and n % 16 == 0
+    assert f(None, n, 1000, FAKE, None) == 1                    # no workspace
+    assert f(FAKE, n - 1, 1000, FAKE, None) == 1                # too small
+    assert f(ctypes.c_void_p(4100), n, 1000, FAKE, None) == 1   # misaligned
+    assert f(FAKE, n, 1000, None, None) == 1                    # no status word
+    assert f(FAKE, n, 3 * 10 ** 9, FAKE, None) == 1             # above the library's 2 s
+
+
 def test_grouped_route_rejects_before_launch(lib):
     f = lib.moe_route_topk_grouped
     assert f(FAKE, 10, 8, 2, 3, 1, FAKE, FAKE, None) == 1      # groups must divide E

@@ -99,8 +99,10 @@ def test_fp8_combine_layer_parity(name, cuda_device):
 
 @pytest.mark.gpu
 def test_fp8_combine_full_size_sampled(cuda_device):
-    """dsv3_fp8y at full size: sampled rows' codes and scales, and the
-    sampled tokens' out, against the oracle's exact rows."""
+    """dsv3_fp8y at full size: codes and scales of the sampled rows (every
+    row of 8 experts, 8 seeded rows and both ends of every other expert, and
+    all rows of the sampled tokens), and the sampled tokens' out, against the
+    oracle's exact rows."""
     wl = workloads.WORKLOADS["dsv3_fp8y"]
     g = GpuLayer(wl, cuda_device)
     assert g.run() == 0
@@ -108,7 +110,7 @@ def test_fp8_combine_full_size_sampled(cuda_device):
     idx_o, w_o = oracle.route_topk(g.inputs["logits"], wl.k)
     lay = oracle.dispatch_layout(idx_o, wl.E, wl.W)
     assert torch.equal(b.slot_of_pair.cpu(), lay["slot_of_pair"])
-    toks, mask = sample_rows(lay, wl.T, wl.k, 48)
+    toks, mask, _ = sample_rows(lay, wl.T, wl.k, 96)
     pos = lay["pair_of_slot"].clone()
     pos[~mask] = -1
     xp_o, sc_o = oracle.permute(g.inputs["x"], wl.k, pos, wl.payload)

@@ -3,10 +3,12 @@ the CPU oracle on the same seeded inputs.
 
 Small workloads (tiny and the extra ragged ones) are compared in full.
 The full-size workloads (mid, dsv3, skew, decode) are compared in full for
-routing, layout and the FP8/bf16 permute of a token sample, and on a
-seeded sample of rows for the GEMM and combine (all k rows of sampled
-tokens, plus the first and last row of every expert), with the same
-launches and sizes the benchmark times.  Full-size combine is also checked
+routing and layout, and on a seeded sample of rows for the permute, the
+GEMM and the combine, with the same launches and sizes the benchmark
+times: all k rows of sampled tokens; the first, the last and 8 more seeded
+rows of every expert; and every row of 8 experts, among them the largest
+one, one whose rows take a pass with a second chunk (257..320 rows) and one
+that takes several passes (parity_helpers.full_experts).  Full-size combine is also checked
 against a property that holds at any size: with identity experts it
 returns x bit for bit.
 """
@@ -81,7 +83,10 @@ def test_full_size_layer_sampled_parity(name, cuda_device):
     assert g.run() == 0
     idx_o, w_o, lay = _check_route_layout(wl, g)
     b = g.buf
-    toks, mask = sample_rows(lay, wl.T, wl.k, FULL[name])
+    toks, mask, experts = sample_rows(lay, wl.T, wl.k, FULL[name])
+    cnt = lay["expert_counts"]
+    assert all(int(mask[lay["expert_offsets"][e]:][:int(cnt[e])].sum()) == int(cnt[e])
+               for e in experts)
     # permute: the oracle writes only the sampled slots
     pos = lay["pair_of_slot"].clone()
     pos[~mask] = -1
