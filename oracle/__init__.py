@@ -67,6 +67,8 @@ def _load():
         lib.oracle_combine_rank.restype = I
         lib.oracle_reduce_partials.argtypes = [P, I, I32, I64, P, I]
         lib.oracle_reduce_partials.restype = I
+        lib.oracle_ep_plan.argtypes = [P, I32, I32, I32, P, P]
+        lib.oracle_ep_plan.restype = I64
         lib.oracle_e4m3_encode.argtypes = [P, I64, P]
         lib.oracle_e4m3_decode.argtypes = [P, I64, P]
         lib.oracle_bf16_round.argtypes = [P, I64, P]
@@ -340,3 +342,99 @@ def layer(wl, inputs, row_mask=None):
                     out=out, **lay)
     out = combine(y, lay["slot_of_pair"], w)
     return dict(topk_idx=idx, topk_w=w, xp=xp, xp_scales=sc, h=h, y=y, out=out, **lay)
+
+
+# ---------------------------------------------------------------- expert parallelism
+def ep_plan(counts_all: torch.Tensor, rank: int):
+    """The dispatch plan of rank ``rank`` from every rank's expert counts
+    ``counts_all`` [W, E] (the count exchange).  Returns (send_base [E]: the
+    row of each expert's owner's receive buffer where this rank's rows for
+    it begin; recv_offsets [E/W + 1]: where each local expert begins in this
+    rank's own receive buffer).  Receive order: expert by expert, inside an
+    expert by source rank, each source's rows in its slot order."""
+    c = counts_all.to(torch.int32).contiguous()
+    W, E = c.shape
+    send_base = torch.empty(E, dtype=torch.int32)
+    recv_offsets = torch.empty(E // W + 1, dtype=torch.int32)
+    if _load().oracle_ep_plan(_p(c), W, E, rank, _p(send_base), _p(recv_offsets)) < 0:
+        raise ValueError("ep_plan: W must divide E and rank lie in [0, W)")
+    return send_base, recv_offsets
+
+
+def ep_dest_rows(lay: dict, topk_idx: torch.Tensor, send_base: torch.Tensor, E: int, W: int):
+    """Where each of a rank's routed pairs lands: (owner rank [N], row of the
+    owner's receive buffer [N]); -1 for a skipped pair.  A pair in slot s of
+    the sender's own expert-major layout, routed to expert e, is the
+    (s - expert_offsets[e])-th row the sender sends to e."""
+    idx = topk_idx.reshape(-1).long()
+    sop = lay["slot_of_pair"].long()
+    ok = sop >= 0
+    e = idx.clamp(0, E - 1)
+    owner = torch.where(ok, e // (E // W), torch.full_like(e, -1))
+    row = torch.where(ok, send_base.long()[e] + sop - lay["expert_offsets"].long()[e],
+                      torch.full_like(e, -1))
+    return owner, row
+
+
+def ep_layer(wl, inputs_per_rank, w13, w2):
+    """The expert-parallel layer over W = len(inputs_per_rank) ranks, simulated
+    in one process: every rank routes its own tokens and lays them out
+    (route_topk, dispatch_layout), the counts are exchanged, each row is moved
+    to its owner's receive buffer by the plan, each owner runs its own
+    experts on what it received (grouped_gemm with w13/w2 rows
+    [r*E/W, (r+1)*E/W)), the rows travel back, and each rank combines its
+    tokens' k rows.  Returns per rank a dict with out (fp64, unrounded), the
+    plan and the receive buffer's offsets."""
+    W, E, k = len(inputs_per_rank), wl.E, wl.k
+    Er = E // W
+    per = []
+    for inp in inputs_per_rank:
+        idx, w = route_topk(inp["logits"], k)
+        per.append(dict(idx=idx, w=w, lay=dispatch_layout(idx, E, W), x=inp["x"]))
+    counts_all = torch.stack([p["lay"]["expert_counts"] for p in per])
+    for r, p in enumerate(per):
+        p["send_base"], p["recv_offsets"] = ep_plan(counts_all, r)
+        p["owner"], p["row"] = ep_dest_rows(p["lay"], p["idx"], p["send_base"], E, W)
+    # dispatch: each pair's payload row goes to (owner, row)
+    recv = []
+    for r in range(W):
+        n = int(per[r]["recv_offsets"][-1])
+        H = wl.H
+        if wl.payload == "e4m3":
+            buf = (torch.zeros(n, H, dtype=torch.uint8), torch.zeros(n, H // 128))
+        else:
+            buf = (torch.zeros(n, H, dtype=_TDT[wl.payload]), None)
+        recv.append(buf)
+    for s, p in enumerate(per):
+        xp, sc = permute(p["x"], k, p["lay"]["pair_of_slot"], wl.payload)
+        sop = p["lay"]["slot_of_pair"].long()
+        for q in torch.nonzero(p["owner"] >= 0).flatten().tolist():
+            r, row = int(p["owner"][q]), int(p["row"][q])
+            src = int(sop[q])
+            if wl.payload == "e4m3":
+                recv[r][0][row] = xp.view(torch.uint8)[src]
+                recv[r][1][row] = sc[src]
+            else:
+                recv[r][0][row] = xp[src]
+    # every owner runs its own experts on its receive buffer
+    ys = []
+    for r in range(W):
+        q, sc = recv[r]
+        if wl.payload == "e4m3":
+            q = q.view(torch.float8_e4m3fn)
+        _, y, _ = grouped_gemm(q, sc, per[r]["recv_offsets"], 0, Er,
+                               w13[r * Er:(r + 1) * Er].contiguous(),
+                               w2[r * Er:(r + 1) * Er].contiguous())
+        ys.append(y)
+    # combine: the rows come back to their sender's slots, then the k-way sum
+    outs = []
+    for s, p in enumerate(per):
+        N = p["lay"]["slot_of_pair"].numel()
+        y_home = torch.zeros(N, wl.H, dtype=torch.float64)
+        sop = p["lay"]["slot_of_pair"].long()
+        for q in torch.nonzero(p["owner"] >= 0).flatten().tolist():
+            y_home[sop[q]] = ys[int(p["owner"][q])][int(p["row"][q])]
+        outs.append(dict(out=combine(y_home, p["lay"]["slot_of_pair"], p["w"]),
+                         send_base=p["send_base"], recv_offsets=p["recv_offsets"],
+                         counts_all=counts_all, owner=p["owner"], row=p["row"]))
+    return outs

@@ -569,3 +569,53 @@ int oracle_reduce_partials(const void* partials, int p_dt, int32_t n, int64_t n_
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------ */
+/* Expert parallelism over W ranks: the dispatch plan                   */
+/* ------------------------------------------------------------------ */
+/* "Expert Parallelism" (aiwiki), "The two all-to-alls" and
+ * "Implementation": every rank sends each routed row to the owner of its
+ * expert, and a count exchange first tells every owner how many rows will
+ * arrive from each peer.  Rank r owns experts [r*Er, (r+1)*Er), Er = E/W
+ * ("Expert parallelism" (Transformers), "How the sizes combine").
+ *
+ * counts_all[s*E + e] is the number of rows rank s routes to expert e (its
+ * own layout's expert_counts, after the count exchange).  Reading of the
+ * receive order (the pages' all_to_all_single delivers one chunk per source
+ * rank; here the chunks are laid out so that each local expert's rows are
+ * one contiguous segment): an owner's receive buffer holds its experts one
+ * after the other; inside an expert, the rows of rank 0 come first, then
+ * rank 1's, and so on, each source's rows in its own slot order.  For
+ * rank `rank` this writes
+ *   send_base[e]      (e = 0..E-1) the row of owner(e)'s receive buffer at
+ *                     which rank's rows for expert e begin;
+ *   recv_offsets[j]   (j = 0..Er) the row at which local expert j begins
+ *                     in rank's own receive buffer (recv_offsets[Er] = the
+ *                     rows it receives),
+ * and returns the rows rank receives, or -1 for W not dividing E or a rank
+ * outside [0, W). */
+int64_t oracle_ep_plan(const int32_t* counts_all, int32_t W, int32_t E, int32_t rank,
+                       int32_t* send_base, int32_t* recv_offsets) {
+    if (W < 1 || E < 1 || E % W != 0 || rank < 0 || rank >= W) return -1;
+    int32_t Er = E / W;
+    int64_t mine = 0;
+    for (int32_t r = 0; r < W; ++r) {
+        int64_t row = 0;   /* rows of owner r's buffer filled so far */
+        for (int32_t j = 0; j < Er; ++j) {
+            int32_t e = r * Er + j;
+            int64_t before = 0, all = 0;
+            for (int32_t s = 0; s < W; ++s) {
+                if (s < rank) before += counts_all[(int64_t)s * E + e];
+                all += counts_all[(int64_t)s * E + e];
+            }
+            send_base[e] = (int32_t)(row + before);
+            if (r == rank) recv_offsets[j] = (int32_t)row;
+            row += all;
+        }
+        if (r == rank) {
+            recv_offsets[Er] = (int32_t)row;
+            mine = row;
+        }
+    }
+    return mine;
+}
