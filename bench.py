@@ -555,6 +555,87 @@ def run_ours(args, wl):
         torch.distributed.destroy_process_group()
 
 
+def run_ep(args, wl):
+    """Expert parallelism (``--ep``).  Under torchrun with N GPUs: N ranks,
+    each with its own T tokens and E/N experts, rows moved to their owners
+    through peer-mapped symmetric-memory buffers (DistributedEP); weak
+    scaling.  On one GPU: ``--ep-ranks`` W ranks emulated on the device, each
+    with T/W tokens (EmulatedEP), the same total batch as the plain step.
+    A step is one layer on every rank; the time is the max over ranks."""
+    from expert_parallelism_b200 import ep
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    moe.load_library()
+    stream = torch.cuda.current_stream()
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        W, Er = ws, wl.E // ws
+        wl_r = wl.replace(W=W, seed=wl.seed + 100 + rank)
+        w13 = torch.empty(Er, 2 * wl.I, wl.H, dtype=torch.bfloat16, device=dev)
+        w2 = torch.empty(Er, wl.H, wl.I, dtype=torch.bfloat16, device=dev)
+        workloads.fill_expert_weights(wl, w13, w2, experts=range(rank * Er, (rank + 1) * Er))
+        logits = workloads.router_logits(wl_r).to(dev)
+        x = workloads.hidden_states(wl_r).to(dev)
+        runner = ep.DistributedEP(wl.replace(W=W), device=dev)
+        step = lambda: runner.forward(logits, x, w13, w2)
+        tokens = wl.T
+        status = lambda: [moe.moe_check_status(runner.state.dev_status)]
+    else:
+        W = args.ep_ranks
+        wl_r = wl.replace(T=wl.T // W, W=W)
+        w13 = torch.empty(wl.E, 2 * wl.I, wl.H, dtype=torch.bfloat16, device=dev)
+        w2 = torch.empty(wl.E, wl.H, wl.I, dtype=torch.bfloat16, device=dev)
+        workloads.fill_expert_weights(wl, w13, w2)
+        lg = [workloads.router_logits(wl_r.replace(seed=wl.seed + 100 + r)).to(dev)
+              for r in range(W)]
+        xs = [workloads.hidden_states(wl_r.replace(seed=wl.seed + 100 + r)).to(dev)
+              for r in range(W)]
+        runner = ep.EmulatedEP(wl_r, W, dev)
+        step = lambda: runner.forward(lg, xs, w13, w2)
+        tokens = wl_r.T * W
+        status = runner.status
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if any(st != 0 for st in status()):
+        raise RuntimeError(f"device status after warm-up: {status()}")
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    if ws > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    launches0 = moe.load_library().moe_launch_count()
+    with ClockSampler(dev) as clk:
+        for a, b in evs:
+            a.record(stream)
+            step()
+            b.record(stream)
+        torch.cuda.synchronize()
+    launches = moe.load_library().moe_launch_count() - launches0
+    if ws > 1:
+        torch.distributed.barrier()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    (ms,) = max_over_ranks([ms], dev)
+    if rank == 0:
+        line = {"metric": METRIC, "value": whole_job_rate(tokens, ws, ms), "unit": "tokens/s",
+                "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic",
+                "config": dict(_config(wl_r), parallelism=(
+                    f"expert parallel over {W} GPUs (peer-mapped buffers)" if ws > 1 else
+                    f"expert parallel, {W} ranks emulated on one GPU"),
+                    tokens_per_rank=wl_r.T),
+                "gpu_launches": int(launches), "clocks": clk.summary(ms)}
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        del runner
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
 def _permute_alone_us(wl, x, buf, iters):
     """Mean device time of moe_permute on the step's routing (its send
     buffer, payload dtype of the workload), with a 512 MiB write before each
@@ -634,6 +715,10 @@ def main():
                     help="override T (smaller cases of the same kernels, for profiling)")
     ap.add_argument("--experts", type=int, default=None,
                     help="override E (must stay a multiple of the logical ranks)")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert parallelism: one rank per GPU under torchrun, or --ep-ranks "
+                         "ranks emulated on one GPU")
+    ap.add_argument("--ep-ranks", type=int, default=8)
     args = ap.parse_args()
     wl = workloads.WORKLOADS[args.workload]
     if args.tokens is not None or args.experts is not None:
@@ -641,6 +726,8 @@ def main():
                         name=f"{wl.name}[T={args.tokens or wl.T},E={args.experts or wl.E}]")
     if args.impl == "reference":
         run_reference(args, wl)
+    elif args.ep:
+        run_ep(args, wl)
     else:
         run_ours(args, wl)
 

@@ -521,6 +521,7 @@ moe_status moe_check_status(int32_t* dev_status, void* stream) {
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return cuda_status(e);
     if (v & MOE_DEV_TIMEOUT) return MOE_ERR_TIMEOUT;
+    if (v & MOE_DEV_OVERFLOW) return MOE_ERR_OVERFLOW;
     if (v & MOE_DEV_BAD_INDEX) return MOE_ERR_BAD_INDEX;
     return MOE_OK;
 }
@@ -548,6 +549,7 @@ const char* moe_status_str(moe_status s) {
         case MOE_ERR_BAD_INDEX: return "MOE_ERR_BAD_INDEX";
         case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
         case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+        case MOE_ERR_OVERFLOW: return "MOE_ERR_OVERFLOW";
     }
     return "MOE_ERR_UNKNOWN";
 }

@@ -104,26 +104,37 @@ struct Piece<uint8_t> {
 
 // rank_offsets null: every pick.  Otherwise only picks whose slot lies in
 // [rank_offsets[rank], rank_offsets[rank + 1]) (the others add nothing).
+// Pick j's row is found through `map` (the local slot of src.rows[0], or a
+// row of its expert's owner under an expert-parallel plan).
 template <typename TY, typename TO>
-__global__ void __launch_bounds__(256) combine_kernel(const TY* __restrict__ y,
-                                                      const float* __restrict__ y_scales,
+__global__ void __launch_bounds__(256) combine_kernel(const __grid_constant__ RankPtrs src,
                                                       const int32_t* __restrict__ slot_of_pair,
+                                                      const PairRows map,
                                                       const float* __restrict__ topk_w, int64_t T,
                                                       int k, int H, TO* __restrict__ out,
                                                       const int32_t* __restrict__ rank_offsets,
-                                                      int rank) {
+                                                      int rank, int32_t* dev_status) {
     using P = Piece<TY>;
     constexpr int EPT = P::N;
-    __shared__ int32_t s_slot[kCombineMaxTopK];
+    __shared__ int s_rank[kCombineMaxTopK];
+    __shared__ int64_t s_row[kCombineMaxTopK];
     __shared__ float s_w[kCombineMaxTopK];
     const int nchunk = H / EPT;
     const int32_t lo = rank_offsets ? __ldg(rank_offsets + rank) : INT32_MIN;
     const int32_t hi = rank_offsets ? __ldg(rank_offsets + rank + 1) : INT32_MAX;
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
         if (threadIdx.x < k) {
-            const int32_t sl = slot_of_pair[t * k + threadIdx.x];
-            s_slot[threadIdx.x] = (sl >= lo && sl < hi) ? sl : -1;
-            s_w[threadIdx.x] = topk_w[t * k + threadIdx.x];
+            const int64_t p = t * k + threadIdx.x;
+            const int32_t sl = slot_of_pair[p];
+            int r = -1;
+            int64_t row = -1;
+            if (sl >= lo && sl < hi && sl >= 0 && !pair_row(map, p, sl, r, row)) {
+                r = -1;
+                flag_status(dev_status, MOE_DEV_OVERFLOW);
+            }
+            s_rank[threadIdx.x] = (sl >= lo && sl < hi) ? r : -1;
+            s_row[threadIdx.x] = row;
+            s_w[threadIdx.x] = topk_w[p];
         }
         __syncthreads();
         for (int c = threadIdx.x; c < nchunk; c += blockDim.x) {
@@ -136,18 +147,19 @@ __global__ void __launch_bounds__(256) combine_kernel(const TY* __restrict__ y,
                 typename P::Raw v[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const int32_t s = s_slot[j + u];
-                    if (s >= 0) P::load(y, y_scales, s, H, c, v[u]);
+                    const int r = s_rank[j + u];
+                    if (r >= 0)
+                        P::load((const TY*)src.rows[r], src.scales[r], s_row[j + u], H, c, v[u]);
                 }
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
-                    if (s_slot[j + u] >= 0) P::add(acc, v[u], s_w[j + u]);
+                    if (s_rank[j + u] >= 0) P::add(acc, v[u], s_w[j + u]);
             }
             for (; j < k; ++j) {
-                const int32_t s = s_slot[j];
-                if (s < 0) continue;
+                const int r = s_rank[j];
+                if (r < 0) continue;
                 typename P::Raw v;
-                P::load(y, y_scales, s, H, c, v);
+                P::load((const TY*)src.rows[r], src.scales[r], s_row[j], H, c, v);
                 P::add(acc, v, s_w[j]);
             }
 #pragma unroll
@@ -165,20 +177,21 @@ static int64_t sm_grid_cap() {
     return (int64_t)sms * 8;   // 8 CTAs of <= 256 threads per SM
 }
 
+// The combine over rows found through `map` in the buffers of `src`.
 // rank_offsets (may be null): restrict to rank `rank`'s slab of slots.
-cudaError_t launch_combine(const void* y, moe_dtype ydt, const float* y_scales,
-                           const int32_t* slot_of_pair, const float* topk_w, int64_t T, int k,
-                           int H, void* out, moe_dtype odt, cudaStream_t s,
-                           const int32_t* rank_offsets, int rank) {
+cudaError_t launch_combine_from(const RankPtrs& src, moe_dtype ydt, const int32_t* slot_of_pair,
+                                const PairRows& map, const float* topk_w, int64_t T, int k, int H,
+                                void* out, moe_dtype odt, int32_t* dev_status, cudaStream_t s,
+                                const int32_t* rank_offsets, int rank) {
     if (T == 0) return cudaSuccess;
     const int64_t cap = sm_grid_cap();
     const unsigned grid = (unsigned)(T < cap ? T : cap);
     const int ept = ydt == MOE_E4M3 ? 16 : 8;
     int threads = ((H / ept + 31) / 32) * 32;
     threads = threads < 32 ? 32 : (threads > 256 ? 256 : threads);
-#define MOE_COMBINE(TY, TO)                                                               \
-    combine_kernel<TY, TO><<<grid, threads, 0, s>>>((const TY*)y, y_scales, slot_of_pair, \
-                                                    topk_w, T, k, H, (TO*)out, rank_offsets, rank)
+#define MOE_COMBINE(TY, TO)                                                                  \
+    combine_kernel<TY, TO><<<grid, threads, 0, s>>>(src, slot_of_pair, map, topk_w, T, k, H, \
+                                                    (TO*)out, rank_offsets, rank, dev_status)
     if (ydt == MOE_E4M3 && odt == MOE_BF16) MOE_COMBINE(uint8_t, __nv_bfloat16);
     else if (ydt == MOE_E4M3) MOE_COMBINE(uint8_t, float);
     else if (ydt == MOE_BF16 && odt == MOE_BF16) MOE_COMBINE(__nv_bfloat16, __nv_bfloat16);
@@ -188,6 +201,19 @@ cudaError_t launch_combine(const void* y, moe_dtype ydt, const float* y_scales,
 #undef MOE_COMBINE
     note_launches(1);
     return cudaGetLastError();
+}
+
+// The local layout: y rows at slot_of_pair's slots of y.
+cudaError_t launch_combine(const void* y, moe_dtype ydt, const float* y_scales,
+                           const int32_t* slot_of_pair, const float* topk_w, int64_t T, int k,
+                           int H, void* out, moe_dtype odt, cudaStream_t s,
+                           const int32_t* rank_offsets, int rank) {
+    RankPtrs src{};
+    src.rows[0] = const_cast<void*>(y);
+    src.scales[0] = const_cast<float*>(y_scales);
+    const PairRows local{nullptr, nullptr, nullptr, 1, 0};
+    return launch_combine_from(src, ydt, slot_of_pair, local, topk_w, T, k, H, out, odt, nullptr,
+                               s, rank_offsets, rank);
 }
 
 // out[i] = (((p[0][i] + p[1][i]) + p[2][i]) + ...) in fp32, rounded once to

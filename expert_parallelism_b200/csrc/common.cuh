@@ -135,6 +135,43 @@ struct gemm_gather {
     int top_k;
 };
 
+// Where a routed pair's row lives.  For the single-GPU layout (send_base
+// null) it is slot slot_of_pair[p] of the one local buffer (rank 0).  With an
+// expert-parallel plan it is row send_base[e] + (slot - expert_offsets[e]) of
+// the receive buffer of rank e / experts_per_rank, e = topk_idx[p]: the
+// sender's slots for expert e, in order, are consecutive rows of e's owner.
+struct PairRows {
+    const int32_t* topk_idx;        // [T*k]: expert of each pair (plan only)
+    const int32_t* expert_offsets;  // [E+1]: the sender's own layout (plan only)
+    const int32_t* send_base;       // [E]: the plan, or null for the local layout
+    int experts_per_rank;
+    int64_t rows_capacity;          // rows of every rank's receive buffer (plan only)
+};
+
+// Resolves pair p in slot `slot` (>= 0) to (rank, row); false when the row
+// would fall outside the receive buffer (the pair is then skipped).
+__device__ __forceinline__ bool pair_row(const PairRows& m, int64_t p, int32_t slot, int& rank,
+                                         int64_t& row) {
+    if (!m.send_base) {
+        rank = 0;
+        row = slot;
+        return true;
+    }
+    const int e = __ldg(m.topk_idx + p);
+    rank = e / m.experts_per_rank;
+    row = (int64_t)__ldg(m.send_base + e) + slot - __ldg(m.expert_offsets + e);
+    return row >= 0 && row < m.rows_capacity;
+}
+
+// Base pointers of every rank's buffer (rank 0 only for the local layout;
+// peer-mapped device pointers across W GPUs), passed by value as a
+// __grid_constant__ kernel parameter.
+constexpr int kMaxEpRanks = 64;
+struct RankPtrs {
+    void* rows[kMaxEpRanks];      // payload or y rows
+    float* scales[kMaxEpRanks];   // FP8 block scales, or null
+};
+
 // Host-side count of kernel launches (reported by moe_launch_count).
 void note_launches(int n);
 

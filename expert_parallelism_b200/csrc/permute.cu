@@ -18,22 +18,48 @@ namespace moe {
 
 constexpr int kMaxTopK = MOE_MAX_TOPK;
 
+// Destinations of token t's k pairs: the rank (-1: skipped) and the row in
+// that rank's buffer, into shared memory.  Flags MOE_DEV_OVERFLOW for a
+// plan row outside the receive buffers.
+__device__ __forceinline__ void token_dests(const int32_t* __restrict__ slot_of_pair,
+                                            const PairRows& map, int64_t t, int k,
+                                            int* s_rank, int64_t* s_row, int32_t* dev_status) {
+    if (threadIdx.x < k) {
+        const int64_t p = t * k + threadIdx.x;
+        const int32_t slot = slot_of_pair[p];
+        int rank = -1;
+        int64_t row = -1;
+        if (slot >= 0 && !pair_row(map, p, slot, rank, row)) {
+            rank = -1;
+            flag_status(dev_status, MOE_DEV_OVERFLOW);
+        }
+        s_rank[threadIdx.x] = rank;
+        s_row[threadIdx.x] = row;
+    }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) permute_copy_kernel(const T* __restrict__ x, int64_t T_,
                                                            int H, int k,
                                                            const int32_t* __restrict__ slot_of_pair,
-                                                           T* __restrict__ xp) {
-    __shared__ int32_t s_slot[kMaxTopK];
+                                                           const PairRows map,
+                                                           const __grid_constant__ RankPtrs dst,
+                                                           int32_t* dev_status) {
+    __shared__ int s_rank[kMaxTopK];
+    __shared__ int64_t s_row[kMaxTopK];
     const int nvec = H * (int)sizeof(T) / 16;
     for (int64_t t = blockIdx.x; t < T_; t += gridDim.x) {
-        if (threadIdx.x < k) s_slot[threadIdx.x] = slot_of_pair[t * k + threadIdx.x];
+        token_dests(slot_of_pair, map, t, k, s_rank, s_row, dev_status);
         __syncthreads();
         const char* src = reinterpret_cast<const char*>(x + t * H);
         for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
             const uint4 d = ld_nc_v4(src + (size_t)v * 16);
             for (int j = 0; j < k; ++j) {
-                const int32_t s = s_slot[j];
-                if (s >= 0) st_v4(reinterpret_cast<char*>(xp + (int64_t)s * H) + (size_t)v * 16, d);
+                const int r = s_rank[j];
+                if (r >= 0)
+                    st_v4(reinterpret_cast<char*>(reinterpret_cast<T*>(dst.rows[r]) + s_row[j] * H) +
+                              (size_t)v * 16,
+                          d);
             }
         }
         __syncthreads();
@@ -60,29 +86,31 @@ constexpr int kMaxBlocks = 64;           // scales staged in shared memory: H <=
 
 // FP8 payload: one CTA per token (grid-stride).  8 lanes own a 128-element
 // block (16 elements each): amax by shuffles, scale = amax / 448, and
-// 16-byte stores of codes to each of the token's k slots.  The token's
-// scales are staged in shared memory and written as 16-byte vectors per
-// slot once the row is done.  With `a` non-null (the layer call), the
-// kernel also writes what the grouped GEMM consumes, bf16(decode(q) *
-// scale) (an fp32 product rounded to bf16), to each slot's row of `a`,
-// so the GEMM needs no separate dequantisation pass.  With xp null (the
-// token-major form, for the GEMM's fused gather) only `a` is written, at
-// the token's own row t: each token is quantised once and its k copies are
-// the same row.
+// 16-byte stores of codes to each of the token's k destinations.  The
+// token's scales are staged in shared memory and written as 16-byte vectors
+// per destination once the row is done.  With `a` non-null (the layer call,
+// local layout), the kernel also writes what the grouped GEMM consumes,
+// bf16(decode(q) * scale) (an fp32 product rounded to bf16), to each slot's
+// row of `a`, so the GEMM needs no separate dequantisation pass.  With
+// dst.rows[0] null (the token-major form, for the GEMM's fused gather) only
+// `a` is written, at the token's own row t: each token is quantised once and
+// its k copies are the same row.
 template <typename T>
 __global__ void __launch_bounds__(kQuantThreads) permute_e4m3_kernel(
     const T* __restrict__ x, int64_t T_, int H, int k, const int32_t* __restrict__ slot_of_pair,
-    uint8_t* __restrict__ xp, float* __restrict__ xp_scales, __nv_bfloat16* __restrict__ a) {
-    __shared__ int32_t s_slot[kMaxTopK];
+    const PairRows map, const __grid_constant__ RankPtrs dst, __nv_bfloat16* __restrict__ a,
+    int32_t* dev_status) {
+    __shared__ int s_rank[kMaxTopK];
+    __shared__ int64_t s_row[kMaxTopK];
     __shared__ __align__(16) float s_scale[kMaxBlocks];
     const int nblk = H / 128;
     const int l8 = threadIdx.x & 7;                 // lane within the block's 8
     const int grp = threadIdx.x >> 3;               // block handled in this pass
     const int ngrp = blockDim.x >> 3;
-    const bool tok_major = xp == nullptr;
+    const bool tok_major = dst.rows[0] == nullptr;
     const bool vec_scales = !tok_major && (nblk % 4) == 0 && nblk <= kMaxBlocks;
     for (int64_t t = blockIdx.x; t < T_; t += gridDim.x) {
-        if (!tok_major && threadIdx.x < k) s_slot[threadIdx.x] = slot_of_pair[t * k + threadIdx.x];
+        if (!tok_major) token_dests(slot_of_pair, map, t, k, s_rank, s_row, dev_status);
         __syncthreads();
         const T* row = x + t * H;
         // whole warps iterate together so the 8-lane shuffles stay converged
@@ -113,8 +141,10 @@ __global__ void __launch_bounds__(kQuantThreads) permute_e4m3_kernel(
                                        quant4_e4m3(f[8], f[9], f[10], f[11], scale),
                                        quant4_e4m3(f[12], f[13], f[14], f[15], scale));
             for (int j = 0; j < k && !tok_major; ++j) {
-                const int32_t s = s_slot[j];
-                if (s >= 0) st_v4(xp + (int64_t)s * H + g * 128 + l8 * 16, q);
+                const int r = s_rank[j];
+                if (r >= 0)
+                    st_v4(reinterpret_cast<uint8_t*>(dst.rows[r]) + s_row[j] * H + g * 128 + l8 * 16,
+                          q);
             }
             if (a) {
                 // the GEMM's operand: each code decoded (exact) times the scale
@@ -130,16 +160,15 @@ __global__ void __launch_bounds__(kQuantThreads) permute_e4m3_kernel(
                 const uint4 b0 = make_uint4(bw[0], bw[1], bw[2], bw[3]);
                 const uint4 b1 = make_uint4(bw[4], bw[5], bw[6], bw[7]);
                 if (tok_major) {
-                    __nv_bfloat16* dst = a + t * H + g * 128 + l8 * 16;
-                    st_v4(dst, b0);
-                    st_v4(dst + 8, b1);
+                    __nv_bfloat16* d = a + t * H + g * 128 + l8 * 16;
+                    st_v4(d, b0);
+                    st_v4(d + 8, b1);
                 }
                 for (int j = 0; j < k && !tok_major; ++j) {
-                    const int32_t s = s_slot[j];
-                    if (s < 0) continue;
-                    __nv_bfloat16* dst = a + (int64_t)s * H + g * 128 + l8 * 16;
-                    st_v4(dst, b0);
-                    st_v4(dst + 8, b1);
+                    if (s_rank[j] < 0) continue;
+                    __nv_bfloat16* d = a + s_row[j] * H + g * 128 + l8 * 16;
+                    st_v4(d, b0);
+                    st_v4(d + 8, b1);
                 }
             }
             if (l8 == 0 && !tok_major) {
@@ -147,18 +176,18 @@ __global__ void __launch_bounds__(kQuantThreads) permute_e4m3_kernel(
                     s_scale[g] = scale;
                 } else {
                     for (int j = 0; j < k; ++j)
-                        if (s_slot[j] >= 0) xp_scales[(int64_t)s_slot[j] * nblk + g] = scale;
+                        if (s_rank[j] >= 0) dst.scales[s_rank[j]][s_row[j] * nblk + g] = scale;
                 }
             }
         }
         if (vec_scales) {
             __syncthreads();
-            const int nvec = nblk / 4;              // 16-byte pieces of one slot's scales
+            const int nvec = nblk / 4;              // 16-byte pieces of one row's scales
             for (int i = threadIdx.x; i < k * nvec; i += blockDim.x) {
                 const int j = i / nvec, v = i - j * nvec;
-                const int32_t s = s_slot[j];
-                if (s >= 0)
-                    st_v4(xp_scales + (int64_t)s * nblk + v * 4,
+                const int r = s_rank[j];
+                if (r >= 0)
+                    st_v4(dst.scales[r] + s_row[j] * nblk + v * 4,
                           *reinterpret_cast<const uint4*>(s_scale + v * 4));
             }
         }
@@ -174,29 +203,49 @@ static unsigned permute_grid(int64_t T) {
     return (unsigned)(T < cap ? T : cap);
 }
 
-// a_bf16 (may be null; FP8 payload only): also write the GEMM's bf16
-// operand bf16(decode(q) * scale) for every slot.
-cudaError_t launch_permute(const void* x, moe_dtype xdt, int64_t T, int H, int k,
-                           const int32_t* slot_of_pair, void* xp, moe_dtype xpdt,
-                           float* xp_scales, __nv_bfloat16* a_bf16, cudaStream_t s) {
+static RankPtrs one_rank(void* rows, float* scales) {
+    RankPtrs d{};
+    d.rows[0] = rows;
+    d.scales[0] = scales;
+    return d;
+}
+
+// Every routed pair's payload row to its destination: slot_of_pair's slot of
+// the local buffer (map.send_base null, dst.rows[0] = xp), or a row of its
+// expert's owner under an expert-parallel plan.  a_bf16 (may be null; FP8
+// payload, local layout only): also write the GEMM's bf16 operand
+// bf16(decode(q) * scale) for every slot.
+cudaError_t launch_permute_to(const void* x, moe_dtype xdt, int64_t T, int H, int k,
+                              const int32_t* slot_of_pair, const PairRows& map,
+                              const RankPtrs& dst, moe_dtype xpdt, __nv_bfloat16* a_bf16,
+                              int32_t* dev_status, cudaStream_t s) {
     if (T == 0) return cudaSuccess;
     const unsigned grid = permute_grid(T);
     if (xpdt == MOE_E4M3) {
         if (xdt == MOE_BF16)
             permute_e4m3_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-                (const __nv_bfloat16*)x, T, H, k, slot_of_pair, (uint8_t*)xp, xp_scales, a_bf16);
+                (const __nv_bfloat16*)x, T, H, k, slot_of_pair, map, dst, a_bf16, dev_status);
         else
-            permute_e4m3_kernel<float><<<grid, 256, 0, s>>>(
-                (const float*)x, T, H, k, slot_of_pair, (uint8_t*)xp, xp_scales, a_bf16);
+            permute_e4m3_kernel<float><<<grid, 256, 0, s>>>((const float*)x, T, H, k, slot_of_pair,
+                                                            map, dst, a_bf16, dev_status);
     } else if (xdt == MOE_BF16) {
         permute_copy_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-            (const __nv_bfloat16*)x, T, H, k, slot_of_pair, (__nv_bfloat16*)xp);
+            (const __nv_bfloat16*)x, T, H, k, slot_of_pair, map, dst, dev_status);
     } else {
         permute_copy_kernel<float><<<grid, 256, 0, s>>>((const float*)x, T, H, k, slot_of_pair,
-                                                        (float*)xp);
+                                                        map, dst, dev_status);
     }
     note_launches(1);
     return cudaGetLastError();
+}
+
+// The local layout: xp[slot_of_pair[t*k + j]] = x[t].
+cudaError_t launch_permute(const void* x, moe_dtype xdt, int64_t T, int H, int k,
+                           const int32_t* slot_of_pair, void* xp, moe_dtype xpdt,
+                           float* xp_scales, __nv_bfloat16* a_bf16, cudaStream_t s) {
+    const PairRows local{nullptr, nullptr, nullptr, 1, 0};
+    return launch_permute_to(x, xdt, T, H, k, slot_of_pair, local, one_rank(xp, xp_scales), xpdt,
+                             a_bf16, nullptr, s);
 }
 
 // Token-major FP8 round trip for the GEMM's fused gather: a[t] =
@@ -205,12 +254,14 @@ cudaError_t launch_quantize_tokens_e4m3(const void* x, moe_dtype xdt, int64_t T,
                                        __nv_bfloat16* a, cudaStream_t s) {
     if (T == 0) return cudaSuccess;
     const unsigned grid = permute_grid(T);
+    const PairRows local{nullptr, nullptr, nullptr, 1, 0};
+    const RankPtrs none = one_rank(nullptr, nullptr);
     if (xdt == MOE_BF16)
         permute_e4m3_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-            (const __nv_bfloat16*)x, T, H, 1, nullptr, nullptr, nullptr, a);
+            (const __nv_bfloat16*)x, T, H, 1, nullptr, local, none, a, nullptr);
     else
-        permute_e4m3_kernel<float><<<grid, 256, 0, s>>>((const float*)x, T, H, 1, nullptr,
-                                                        nullptr, nullptr, a);
+        permute_e4m3_kernel<float><<<grid, 256, 0, s>>>((const float*)x, T, H, 1, nullptr, local,
+                                                        none, a, nullptr);
     note_launches(1);
     return cudaGetLastError();
 }

@@ -19,9 +19,9 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe.so")
 
 MOE_F32, MOE_BF16, MOE_E4M3 = 0, 1, 2
-MOE_DEV_BAD_INDEX, MOE_DEV_TIMEOUT = 0x1, 0x2
+MOE_DEV_BAD_INDEX, MOE_DEV_TIMEOUT, MOE_DEV_OVERFLOW = 0x1, 0x2, 0x4
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_BAD_INDEX",
-          4: "MOE_ERR_TIMEOUT", 5: "MOE_ERR_CUDA"}
+          4: "MOE_ERR_TIMEOUT", 5: "MOE_ERR_CUDA", 6: "MOE_ERR_OVERFLOW"}
 _DT = {torch.float32: MOE_F32, torch.bfloat16: MOE_BF16, torch.float8_e4m3fn: MOE_E4M3}
 
 # exported symbols and their ctypes signatures (P = pointer, I64/I32 = ints)
@@ -50,6 +50,11 @@ SIGNATURES = {
     "moe_check_status": ([_P, _P], _I),
     "moe_status_str": ([_I], ctypes.c_char_p),
     "moe_launch_count": ([], ctypes.c_uint64),
+    "moe_ep_plan": ([_P, _I32, _I32, _I32, _P, _P, _P, _P], _I),
+    "moe_ep_dispatch": ([_P, _I, _I64, _I32, _I32, _P, _P, _P, _P, _I32, _I32, _P, _P, _I, _I64,
+                         _P, _P], _I),
+    "moe_ep_combine": ([_P, _P, _I, _P, _P, _P, _P, _P, _I64, _I32, _I32, _I32, _I32, _I64, _P,
+                        _I, _P, _P], _I),
     "moe_diag_layout_wait_timeout_workspace_bytes": ([], _SZ),
     "moe_diag_layout_wait_timeout": ([_P, _SZ, ctypes.c_uint64, _P, _P], _I),
 }
@@ -220,6 +225,50 @@ def moe_reduce_partials(partials, out, stream=None):
 def moe_check_status(dev_status, stream=None) -> int:
     """Synchronises the stream; returns the raw status code (0 = OK)."""
     return int(load_library().moe_check_status(_ptr(dev_status), _stream(stream)))
+
+
+def _ptr_array(ptrs):
+    """A host array of device pointers (ints or tensors; None -> NULL)."""
+    vals = [None if p is None else (p.data_ptr() if isinstance(p, torch.Tensor) else int(p))
+            for p in ptrs]
+    return (ctypes.c_void_p * len(vals))(*vals)
+
+
+def moe_ep_plan(counts_all, rank, send_base, recv_offsets, dev_status, stream=None):
+    """This rank's dispatch plan from every rank's expert counts [W, E]."""
+    W, E = counts_all.shape
+    _check("moe_ep_plan", load_library().moe_ep_plan(
+        _ptr(counts_all), W, E, rank, _ptr(send_base), _ptr(recv_offsets), _ptr(dev_status),
+        _stream(stream)))
+
+
+def moe_ep_dispatch(x, k, topk_idx, slot_of_pair, expert_offsets, send_base, recv_rows,
+                    recv_scales, payload_dtype, rows_capacity, dev_status, stream=None):
+    """Every routed row of this rank into its owner's receive buffer.
+    ``recv_rows``/``recv_scales``: one entry per rank (tensors on this GPU,
+    or raw peer-mapped device pointers)."""
+    T, H = x.shape
+    W = len(recv_rows)
+    E = expert_offsets.numel() - 1
+    sc = _ptr_array(recv_scales) if recv_scales is not None else None
+    _check("moe_ep_dispatch", load_library().moe_ep_dispatch(
+        _ptr(x), dtype_code(x), T, H, k, _ptr(topk_idx), _ptr(slot_of_pair),
+        _ptr(expert_offsets), _ptr(send_base), E, W, _ptr_array(recv_rows), sc,
+        _DT[payload_dtype], rows_capacity, _ptr(dev_status), _stream(stream)))
+
+
+def moe_ep_combine(y_rows, y_scales, y_dtype, topk_idx, slot_of_pair, expert_offsets, send_base,
+                   topk_w, rows_capacity, out, dev_status, stream=None):
+    """out[t] = sum_j w[t,j] * (pick j's output row in its owner's y)."""
+    T, k = topk_w.shape
+    H = out.shape[1]
+    W = len(y_rows)
+    E = expert_offsets.numel() - 1
+    sc = _ptr_array(y_scales) if y_scales is not None else None
+    _check("moe_ep_combine", load_library().moe_ep_combine(
+        _ptr_array(y_rows), sc, _DT[y_dtype], _ptr(topk_idx), _ptr(slot_of_pair),
+        _ptr(expert_offsets), _ptr(send_base), _ptr(topk_w), T, k, H, E, W, rows_capacity,
+        _ptr(out), dtype_code(out), _ptr(dev_status), _stream(stream)))
 
 
 def moe_diag_layout_wait_timeout(workspace, wait_limit_ns, dev_status, stream=None):

@@ -67,7 +67,8 @@ typedef enum moe_status {
     MOE_ERR_UNSUPPORTED = 2, /* valid but beyond the kernels' limits (E > 1024, k > 16) */
     MOE_ERR_BAD_INDEX = 3,   /* device: an expert id outside [0, E) was skipped */
     MOE_ERR_TIMEOUT = 4,     /* device: a bounded wait ran out; results invalid */
-    MOE_ERR_CUDA = 5         /* a CUDA runtime call or kernel launch failed */
+    MOE_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed */
+    MOE_ERR_OVERFLOW = 6     /* device: a row fell outside a receive buffer and was skipped */
 } moe_status;
 
 typedef enum moe_dtype {
@@ -79,6 +80,7 @@ typedef enum moe_dtype {
 /* Bits of the device status word. */
 #define MOE_DEV_BAD_INDEX 0x1
 #define MOE_DEV_TIMEOUT 0x2
+#define MOE_DEV_OVERFLOW 0x4
 
 /* Kernel limits (MOE_ERR_UNSUPPORTED beyond them). */
 #define MOE_MAX_EXPERTS 1024
@@ -380,6 +382,96 @@ moe_status moe_reduce_partials(const float* partials, int32_t n_partials, int64_
                                void* out, moe_dtype out_dtype, void* stream);
 
 /*
+ * Expert parallelism over W ranks (W GPUs of one NVLink domain, one process
+ * each; or W ranks run on one GPU).  Each rank holds its own T tokens and
+ * the weights of its E/W experts [r*E/W, (r+1)*E/W) ("Expert parallelism"
+ * (Transformers docs), "How the sizes combine").  One layer, per rank:
+ *   1. moe_route_topk and moe_dispatch_layout on its own tokens;
+ *   2. the count exchange: every rank's expert_counts gathered into
+ *      counts_all [W, E] on every rank (for example an all-gather over
+ *      NCCL) -- "Expert Parallelism" (aiwiki), "Implementation": peers must
+ *      know how much is coming;
+ *   3. moe_ep_plan: where this rank's rows land in each owner's receive
+ *      buffer, and where its own local experts start in its buffer;
+ *   4. moe_ep_dispatch: every routed row stored into its owner's receive
+ *      buffer (the dispatch all-to-all, "The two all-to-alls");
+ *   5. once every rank's dispatch has completed (a barrier across ranks):
+ *      moe_grouped_gemm on the local receive buffer, expert_offsets =
+ *      recv_offsets, expert_begin = 0, n_experts = E/W, the local weights;
+ *   6. once every rank's GEMM has completed: moe_ep_combine, which reads
+ *      each pick's output row from its owner's y buffer (the combine
+ *      all-to-all) and takes the router-weighted sum.
+ * Every routed row's result is the same as on one GPU: out equals
+ * moe_layer_forward's on the same tokens, bit for bit.
+ *
+ * Receive layout (a reading: the pages' all_to_all_single delivers one
+ * chunk per source rank): an owner's buffer holds its experts one after the
+ * other, and inside an expert the rows of rank 0, then rank 1, ..., each in
+ * the sender's slot order, so each local expert is one contiguous segment.
+ */
+
+/*
+ * moe_ep_plan -- this rank's dispatch plan from the exchanged counts.
+ *   counts_all   [W, E] int32, device: rows rank s routes to expert e.
+ *   send_base    [E] int32, device, written: the row of expert e's owner's
+ *                receive buffer where this rank's rows for e begin.
+ *   recv_offsets [E/W + 1] int32, device, written: where local expert j
+ *                begins in this rank's receive buffer; recv_offsets[E/W] is
+ *                the number of rows it receives.
+ *   dev_status   MOE_DEV_BAD_INDEX if a count is negative (read as 0).
+ * Requires W | E, 0 <= rank < W, W <= 64, E <= MOE_MAX_EXPERTS.
+ */
+moe_status moe_ep_plan(const int32_t* counts_all, int32_t W, int32_t E, int32_t rank,
+                       int32_t* send_base, int32_t* recv_offsets, int32_t* dev_status,
+                       void* stream);
+
+/*
+ * moe_ep_dispatch -- the dispatch all-to-all as stores: for each of this
+ * rank's routed pairs p = t*k + j (slot s = slot_of_pair[p] >= 0, expert e =
+ * topk_idx[p]), row x[t] (or its FP8 payload, by moe_permute's rule) is
+ * written to row send_base[e] + (s - expert_offsets[e]) of the receive
+ * buffer of rank e / (E/W).
+ *   x, x_dtype, T, H, k     as moe_permute.
+ *   topk_idx, slot_of_pair, expert_offsets   this rank's route and layout.
+ *   send_base               from moe_ep_plan.
+ *   recv_rows, recv_scales  HOST arrays of W device pointers: every rank's
+ *                           receive buffer [rows_capacity, H] in
+ *                           payload_dtype, and for MOE_E4M3 its block scales
+ *                           [rows_capacity, H/128] fp32 (16-byte aligned; may
+ *                           be NULL otherwise).  Across GPUs these are
+ *                           peer-mapped pointers.
+ *   rows_capacity           rows of every receive buffer; a row at or past
+ *                           it is skipped and MOE_DEV_OVERFLOW flagged.
+ * payload_dtype is x_dtype or MOE_E4M3.  The call only writes; the owners
+ * may read their buffers once every rank's dispatch has completed.
+ */
+moe_status moe_ep_dispatch(const void* x, moe_dtype x_dtype, int64_t T, int32_t H, int32_t k,
+                           const int32_t* topk_idx, const int32_t* slot_of_pair,
+                           const int32_t* expert_offsets, const int32_t* send_base, int32_t E,
+                           int32_t W, void* const* recv_rows, float* const* recv_scales,
+                           moe_dtype payload_dtype, int64_t rows_capacity, int32_t* dev_status,
+                           void* stream);
+
+/*
+ * moe_ep_combine -- the combine all-to-all as loads, fused with the
+ * weighted sum: out[t] = sum_j topk_w[t,j] * y_owner[row(p)], with row(p)
+ * as in moe_ep_dispatch and y_owner the owner's expert outputs (written by
+ * its moe_grouped_gemm at its receive rows), fp32 accumulation in j order,
+ * rounded once to out_dtype (moe_combine's rule).
+ *   y_rows, y_scales   HOST arrays of W device pointers: every rank's y
+ *                      [rows_capacity, H] in y_dtype (and its block scales
+ *                      for MOE_E4M3).
+ *   rows_capacity      rows of every y buffer (MOE_DEV_OVERFLOW past it).
+ * Other arguments as moe_ep_dispatch and moe_combine.
+ */
+moe_status moe_ep_combine(void* const* y_rows, float* const* y_scales, moe_dtype y_dtype,
+                          const int32_t* topk_idx, const int32_t* slot_of_pair,
+                          const int32_t* expert_offsets, const int32_t* send_base,
+                          const float* topk_w, int64_t T, int32_t k, int32_t H, int32_t E,
+                          int32_t W, int64_t rows_capacity, void* out, moe_dtype out_dtype,
+                          int32_t* dev_status, void* stream);
+
+/*
  * moe_layer_forward -- the whole hot path in one call: moe_route_topk,
  * moe_dispatch_layout, moe_permute, moe_grouped_gemm (every expert, local
  * expert j = global expert j) and moe_combine, in that order on `stream`,
@@ -479,8 +571,9 @@ moe_status moe_layer_forward_host(const float* logits_host, const void* x_host, 
 /*
  * moe_check_status -- synchronise `stream`, read the device status word,
  * clear it, and map it to a status: MOE_ERR_TIMEOUT if a wait ran out,
- * else MOE_ERR_BAD_INDEX if an id was skipped, else MOE_OK (MOE_ERR_CUDA if
- * the synchronisation itself failed).  The only call that blocks.
+ * else MOE_ERR_OVERFLOW if a row missed a receive buffer, else
+ * MOE_ERR_BAD_INDEX if an id was skipped, else MOE_OK (MOE_ERR_CUDA if the
+ * synchronisation itself failed).  The only call that blocks.
  */
 moe_status moe_check_status(int32_t* dev_status, void* stream);
 

@@ -242,6 +242,38 @@ def test_wait_timeout_diagnostic_rejects_before_launch(lib):
     assert f(FAKE, n, 3 * 10 ** 9, FAKE, None) == 1             # above the library's 2 s
 
 
+def test_ep_calls_reject_before_launch(lib):
+    W = 2
+    table = (ctypes.c_void_p * W)(4096, 8192)
+    bad_table = (ctypes.c_void_p * W)(4096, 4100)            # misaligned peer buffer
+    null_table = (ctypes.c_void_p * W)(4096, None)
+    pl = lib.moe_ep_plan
+    assert pl(FAKE, 3, 8, 0, FAKE, FAKE, FAKE, None) == 1       # W must divide E
+    assert pl(FAKE, 2, 8, 2, FAKE, FAKE, FAKE, None) == 1       # rank outside [0, W)
+    assert pl(FAKE, 128, 128, 0, FAKE, FAKE, FAKE, None) == 2   # more than 64 ranks
+    assert pl(None, 2, 8, 0, FAKE, FAKE, FAKE, None) == 1
+    d = lib.moe_ep_dispatch
+    args = lambda **kw: [FAKE, moe.MOE_BF16, 10, kw.get("H", 128), 2, FAKE, FAKE, FAKE, FAKE,
+                         kw.get("E", 8), W, kw.get("rows", table), kw.get("sc", None),
+                         kw.get("pd", moe.MOE_BF16), kw.get("cap", 100), FAKE, None]
+    assert d(*args(E=7)) == 1                                  # W does not divide E
+    assert d(*args(rows=bad_table)) == 1
+    assert d(*args(rows=null_table)) == 1
+    assert d(*args(pd=moe.MOE_E4M3)) == 1                      # FP8 needs the scale table
+    assert d(*args(pd=moe.MOE_E4M3, sc=table, H=136)) == 1     # and H % 128
+    assert d(*args(pd=moe.MOE_F32)) == 1                       # no dtype cast
+    assert d(*args(cap=-1)) == 1
+    assert d(*args(cap=1 << 31)) == 2
+    c = lib.moe_ep_combine
+    cargs = lambda **kw: [kw.get("rows", table), kw.get("sc", None), kw.get("yd", moe.MOE_F32),
+                          FAKE, FAKE, FAKE, FAKE, FAKE, 10, 2, 128, 8, W, 100,
+                          kw.get("out", FAKE), moe.MOE_BF16, FAKE, None]
+    assert c(*cargs(rows=null_table)) == 1
+    assert c(*cargs(yd=moe.MOE_E4M3)) == 1                     # FP8 y needs the scale table
+    assert c(*cargs(out=ctypes.c_void_p(4100))) == 1            # misaligned out
+    assert moe.moe_status_str(6) == "MOE_ERR_OVERFLOW"
+
+
 def test_grouped_route_rejects_before_launch(lib):
     f = lib.moe_route_topk_grouped
     assert f(FAKE, 10, 8, 2, 3, 1, FAKE, FAKE, None) == 1      # groups must divide E
