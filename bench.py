@@ -412,23 +412,46 @@ def run_ours(args, wl):
     layer_ms = ms - statistics.mean(per["route_topk"])      # dispatch + GEMM + combine
     ms, layer_ms = max_over_ranks([ms, layer_ms], dev)
 
-    # end to end through the C ABI with HOST buffers: the call copies logits
-    # and x from pinned host memory, runs the layer and copies out back
+    # end to end through the C ABI with HOST buffers: each call copies that
+    # step's logits and x from pinned host memory, runs the layer and copies
+    # out back.  Two steps are in flight on two streams with their own
+    # device buffers, so one step's host copies overlap the other's kernels
+    # (the copy engines and the SMs work at the same time); the time is the
+    # whole run of K steps, every copy included.
     h_logits = inp["logits"].pin_memory()
     h_x = inp["x"].pin_memory()
-    h_out = torch.empty(buf.out.shape, dtype=buf.out.dtype).pin_memory()
-    e2e_ms = []
-    for i in range(args.warmup + args.steps):
-        flush.fill_(1)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        moe.moe_layer_forward_host(wl, h_logits, h_x, h_out, logits, x, w13, w2, buf)
-        e1.record(stream)
+    sets = [(buf, logits, x), (moe.LayerBuffers(wl, dev), torch.empty_like(logits),
+                               torch.empty_like(x))]
+    h_outs = [torch.empty(buf.out.shape, dtype=buf.out.dtype).pin_memory() for _ in sets]
+    e2e_streams = [torch.cuda.Stream(dev), torch.cuda.Stream(dev)]
+
+    def e2e_run(n):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for st in e2e_streams:
+            st.wait_stream(stream)
+        for i in range(n):
+            bset, lg, xx = sets[i % 2]
+            st = e2e_streams[i % 2]
+            if _needs_flush(wl):
+                with torch.cuda.stream(st):
+                    flush.fill_(1)
+            moe.moe_layer_forward_host(wl, h_logits, h_x, h_outs[i % 2], lg, xx, w13, w2, bset,
+                                       stream=st)
+        for st in e2e_streams:
+            stream.wait_stream(st)
+        b.record(stream)
         torch.cuda.synchronize()
-        if i >= args.warmup:
-            e2e_ms.append(e0.elapsed_time(e1))
-    e2e = statistics.mean(e2e_ms)
+        return a.elapsed_time(b)
+
+    e2e_run(args.warmup)
+    e2e = e2e_run(args.steps) / args.steps
     (e2e,) = max_over_ranks([e2e], dev)
+    for bset, _, _ in sets:
+        st = moe.moe_check_status(bset.dev_status)
+        if st != 0:
+            raise RuntimeError(f"device status after the host-buffer steps: {moe.STATUS.get(st, st)}")
+    del sets[1]
     # the permute alone (moe_permute: the send buffer only, as a standalone
     # call), L2 flushed before each launch
     perm_alone_us = _permute_alone_us(wl, x, buf, 10)
@@ -539,8 +562,8 @@ def run_ours(args, wl):
             "kernels": kernels, "roofline": roof, "roofline_other": others,
             "e2e": {"value": whole_job_rate(wl.T, ws, e2e), "unit": "tokens/s",
                     "h2d_bytes_per_step": h_logits.numel() * 4 + h_x.numel() * h_x.element_size(),
-                    "d2h_bytes_per_step": h_out.numel() * h_out.element_size(),
-                    "ms_per_step": e2e},
+                    "d2h_bytes_per_step": h_outs[0].numel() * h_outs[0].element_size(),
+                    "ms_per_step": e2e, "steps_in_flight": 2},
             "graph": {"us_median_per_layer": graph_us, "replays": replays,
                       "tokens_per_s": whole_job_rate(wl.T, ws, graph_us * 1e-3)},
             "gpu_launches": int(launches),
