@@ -31,7 +31,10 @@ cudaError_t launch_grouped_gemm_simt_f32(const float*, const int32_t*, const int
 cudaError_t launch_grouped_gemm_tc(const __nv_bfloat16*, const int32_t*, const int32_t*, int, int,
                                    int64_t, int, int, const __nv_bfloat16*, const __nv_bfloat16*,
                                    __nv_bfloat16*, void*, moe_dtype, float*, int32_t*,
-                                   const gemm_gather*, cudaEvent_t, cudaStream_t);
+                                   const gemm_gather*, cudaEvent_t, cudaStream_t, bool);
+size_t packed_weights_bytes(int64_t E, int H, int I, int which);
+cudaError_t launch_pack_weights(const __nv_bfloat16*, const __nv_bfloat16*, int64_t, int, int,
+                                __nv_bfloat16*, __nv_bfloat16*, cudaStream_t);
 bool grouped_gemm_tc_uses_swap(int64_t n_rows, int n_experts, moe_dtype y_dtype);
 cudaError_t launch_quantize_tokens_e4m3(const void*, moe_dtype, int64_t, int, __nv_bfloat16*,
                                        cudaStream_t);
@@ -191,7 +194,7 @@ cudaError_t run_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_scales,
                      moe_dtype w_dtype, void* h, void* y, moe_dtype y_dtype, float* y_scales,
                      void* workspace, int32_t* dev_status, cudaStream_t s,
                      cudaEvent_t ev_a = nullptr, cudaEvent_t ev_b = nullptr,
-                     bool a_ready = false, const gemm_gather* g = nullptr) {
+                     bool a_ready = false, const gemm_gather* g = nullptr, bool packed = false) {
     cudaError_t e = cudaSuccess;
     if (w_dtype == MOE_F32) {
         if (ev_a) e = cudaEventRecord(ev_a, s);
@@ -216,7 +219,7 @@ cudaError_t run_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_scales,
                                   n_rows, H, I,
                                   (const __nv_bfloat16*)w13, (const __nv_bfloat16*)w2,
                                   (__nv_bfloat16*)h, y, y_dtype, y_scales, dev_status, g, ev_b,
-                                  s);
+                                  s, packed);
 }
 
 }  // namespace
@@ -319,6 +322,46 @@ moe_status moe_grouped_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_
                                 y_dtype, y_scales, workspace, dev_status, (cudaStream_t)stream));
 }
 
+size_t moe_packed_weights_bytes(int32_t E, int32_t H, int32_t I, int32_t which) {
+    if (E < 1 || H < 1 || I < 1 || (which != 0 && which != 1)) return 0;
+    return packed_weights_bytes(E, H, I, which);
+}
+
+moe_status moe_pack_expert_weights(const void* w13, const void* w2, int32_t E, int32_t H,
+                                   int32_t I, moe_dtype w_dtype, void* packed13, void* packed2,
+                                   void* stream) {
+    if (E < 1 || H < 1 || I < 1 || (H % 8) != 0 || (I % 8) != 0 || w_dtype != MOE_BF16)
+        return MOE_ERR_INVALID_ARG;
+    if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+    if (!w13 && !w2) return MOE_ERR_INVALID_ARG;
+    if ((w13 && (!packed13 || !aligned16(w13) || !aligned16(packed13))) ||
+        (w2 && (!packed2 || !aligned16(w2) || !aligned16(packed2))))
+        return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_pack_weights((const __nv_bfloat16*)w13, (const __nv_bfloat16*)w2, E,
+                                           H, I, (__nv_bfloat16*)packed13, (__nv_bfloat16*)packed2,
+                                           (cudaStream_t)stream));
+}
+
+moe_status moe_grouped_gemm_packed(const void* xp, moe_dtype xp_dtype, const float* xp_scales,
+                                   const int32_t* expert_offsets, const int32_t* expert_counts,
+                                   int32_t expert_begin, int32_t n_experts, int64_t n_rows,
+                                   int32_t H, int32_t I, const void* packed13,
+                                   const void* packed2, moe_dtype w_dtype, void* h, void* y,
+                                   moe_dtype y_dtype, float* y_scales, void* workspace,
+                                   size_t workspace_bytes, int32_t* dev_status, void* stream) {
+    if (w_dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+    bool noop;
+    const moe_status st =
+        check_gemm(xp, xp_dtype, xp_scales, expert_offsets, expert_begin, n_experts, n_rows, H,
+                   I, packed13, packed2, w_dtype, h, y, y_dtype, y_scales, workspace,
+                   workspace_bytes, dev_status, &noop);
+    if (st != MOE_OK || noop) return st;
+    return cuda_status(run_gemm(xp, xp_dtype, xp_scales, expert_offsets, expert_counts,
+                                expert_begin, n_experts, n_rows, H, I, packed13, packed2, w_dtype,
+                                h, y, y_dtype, y_scales, workspace, dev_status,
+                                (cudaStream_t)stream, nullptr, nullptr, false, nullptr, true));
+}
+
 moe_status moe_combine(const void* y, moe_dtype y_dtype, const float* y_scales,
                        const int32_t* slot_of_pair, const float* topk_w, int64_t T, int32_t k,
                        int32_t H, void* out, moe_dtype out_dtype, void* stream) {
@@ -361,7 +404,7 @@ static int64_t layer_slots(int64_t T, int32_t k, int32_t E, int32_t capacity) {
 }
 
 static moe_layer_options resolve(const moe_layer_options* o) {
-    return o ? *o : moe_layer_options{-1, 0, 0, 0, 0};
+    return o ? *o : moe_layer_options{-1, 0, 0, 0, 0, 0};
 }
 
 static moe_status check_layer(const float* logits, const void* x, moe_dtype x_dtype, int64_t T,
@@ -396,6 +439,8 @@ static moe_status check_layer(const float* logits, const void* x, moe_dtype x_dt
     // the all_reduce form: W fp32 partials of [T, H]
     if (st == MOE_OK && o.all_reduce_form != 0 && T > 0 && (!b->partials || !aligned16(b->partials)))
         st = MOE_ERR_INVALID_ARG;
+    // packed weights exist for bf16 weights only
+    if (st == MOE_OK && o.packed_weights != 0 && w_dtype != MOE_BF16) st = MOE_ERR_INVALID_ARG;
     // the fused gather's FP8 source, one bf16 row per token, lives in the
     // GEMM workspace
     if (st == MOE_OK && o.fused_gather != 0 && payload_dtype == MOE_E4M3 && T > 0 &&
@@ -416,7 +461,7 @@ static cudaError_t launch_layer(const float* logits, const void* x, moe_dtype x_
     // source (x itself for a bf16 payload; each token's FP8 round trip,
     // bf16(decode(q) * scale), for an FP8 payload) instead of a permuted copy.
     const bool gather = o.fused_gather != 0 && w_dtype == MOE_BF16 && n_slots > 0 &&
-                        grouped_gemm_tc_uses_swap(n_slots, E, y_dtype);
+                        (o.packed_weights != 0 || grouped_gemm_tc_uses_swap(n_slots, E, y_dtype));
     const gemm_gather gsrc{payload_dtype == MOE_E4M3 ? (const __nv_bfloat16*)b->gemm_workspace
                                                      : (const __nv_bfloat16*)x,
                            b->pair_of_slot, k};
@@ -448,7 +493,7 @@ static cudaError_t launch_layer(const float* logits, const void* x, moe_dtype x_
                      capacity < 0 ? nullptr : b->expert_counts, 0, E, n_slots, H, I, w13, w2,
                      w_dtype, b->h, b->y, y_dtype, b->y_scales, b->gemm_workspace, b->dev_status,
                      s, ev ? (cudaEvent_t)ev[4] : nullptr, ev ? (cudaEvent_t)ev[5] : nullptr,
-                     /*a_ready=*/true, gather ? &gsrc : nullptr);
+                     /*a_ready=*/true, gather ? &gsrc : nullptr, o.packed_weights != 0);
     } else if (e == cudaSuccess) {
         e = mark(4);
         if (e == cudaSuccess) e = mark(5);

@@ -474,7 +474,8 @@ cudaError_t launch_grouped_gemm_tc_swap(const __nv_bfloat16* a, const int32_t* o
                                         int64_t n_rows, int H, int I, const __nv_bfloat16* w13,
                                         const __nv_bfloat16* w2, __nv_bfloat16* h, void* y,
                                         moe_dtype y_dtype, float* y_scales, int32_t* dev_status,
-                                        const gemm_gather* g, cudaEvent_t ev_mid, cudaStream_t s);
+                                        const gemm_gather* g, cudaEvent_t ev_mid, cudaStream_t s,
+                                        bool packed);
 
 // Kernel choice, from the average rows per expert (known on the host
 // without reading the device offsets).  The operand-swapped pair kernel
@@ -501,16 +502,20 @@ bool grouped_gemm_tc_uses_swap(int64_t n_rows, int n_experts, moe_dtype y_dtype)
 // segment to its first counts[j] rows.  g (may be null; the operand-swapped
 // kernel only): the gate/up operand's rows are gathered from g->src instead
 // of read from A.  ev_mid (may be null) is recorded between the two phases.
+// packed: the weights are in pack_weights.cu's layout (operand-swapped
+// kernel).
 cudaError_t launch_grouped_gemm_tc(const __nv_bfloat16* a, const int32_t* offsets,
                                    const int32_t* counts, int expert_begin, int n_experts,
                                    int64_t n_rows, int H, int I, const __nv_bfloat16* w13,
                                    const __nv_bfloat16* w2, __nv_bfloat16* h, void* y,
                                    moe_dtype y_dtype, float* y_scales, int32_t* dev_status,
-                                   const gemm_gather* g, cudaEvent_t ev_mid, cudaStream_t s) {
-    if (grouped_gemm_tc_uses_swap(n_rows, n_experts, y_dtype))
+                                   const gemm_gather* g, cudaEvent_t ev_mid, cudaStream_t s,
+                                   bool packed) {
+    // packed weights: the operand-swapped kernel reads them at any size
+    if (packed || grouped_gemm_tc_uses_swap(n_rows, n_experts, y_dtype))
         return launch_grouped_gemm_tc_swap(a, offsets, counts, expert_begin, n_experts, n_rows, H,
                                            I, w13, w2, h, y, y_dtype, y_scales, dev_status, g,
-                                           ev_mid, s);
+                                           ev_mid, s, packed);
     if (g) return cudaErrorInvalidValue;
     return tc::run_gemm<1>(a, offsets, counts, expert_begin, n_experts, n_rows, H, I, w13, w2, h,
                            y, y_dtype == MOE_F32, dev_status, ev_mid, s);

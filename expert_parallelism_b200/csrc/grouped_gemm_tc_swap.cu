@@ -141,6 +141,9 @@ struct Params {
     const __nv_bfloat16* gather_src;
     const int32_t* pair_of_slot;
     int top_k;
+    // weights in the packed layout (pack_weights.cu): one contiguous 16 KB
+    // block per (expert, 64 or 128 weight rows, 64-column k-step)
+    int packed;
 };
 
 // Passes an expert with `rows` routed rows takes.
@@ -307,7 +310,10 @@ __global__ void __launch_bounds__(threads_of<GATHER>(), 1)
                 const uint32_t sw = sbase + Smem::w + stage * kWBytes;
                 const uint32_t st = sbase + Smem::t + stage * kTBytes;
                 const int k0 = kb * BK;
-                if (GLU)   // 64 gate rows, then the 64 matching up rows: one box
+                if (p.packed)   // this CTA's row block of the tile: one 16 KB block
+                    tma_load_3d<2>(sw, &tmap_w, cfb, 0, 0,
+                                   (ti.j * 2 * p.n_wtiles + 2 * ti.wt + (int)rank) * nk + kb);
+                else if (GLU)   // 64 gate rows, then the 64 matching up rows: one box
                     tma_load_4d<2>(sw, &tmap_w, cfb, k0, w_row(ti), 0, ti.j);
                 else
                     tma_load_3d<2>(sw, &tmap_w, cfb, k0, w_row(ti), ti.j);
@@ -681,17 +687,30 @@ static bool make_row_maps(CUtensorMap* m, const void* base, int K, int64_t n_row
 // each expert's segment to its first counts[j] rows.  ev_mid (may be null)
 // is recorded between the two phases.  With g (the fused gather) non-null,
 // A is not read: row s of the gate/up operand is row pair_of_slot[s] / k of
-// g.src [*, H] (16-byte aligned).
+// g.src [*, H] (16-byte aligned).  packed: w13 and w2 are in the packed
+// layout of pack_weights.cu.
 cudaError_t launch_grouped_gemm_tc_swap(const __nv_bfloat16* a, const int32_t* offsets,
                                         const int32_t* counts, int expert_begin, int n_experts,
                                         int64_t n_rows, int H, int I, const __nv_bfloat16* w13,
                                         const __nv_bfloat16* w2, __nv_bfloat16* h, void* y,
                                         moe_dtype y_dtype, float* y_scales, int32_t* dev_status,
                                         const gemm_gather* g, cudaEvent_t ev_mid,
-                                        cudaStream_t s) {
+                                        cudaStream_t s, bool packed) {
     using namespace tcs;
     CUtensorMap mw1, mt1[3], mw2, mt2[3];
-    {   // W13 as [E, 2, I, H]: a box of 64 gate rows and the 64 matching up rows
+    const int nwt1 = (I + kWRows - 1) / kWRows, nwt2 = (H + 2 * kWRows - 1) / (2 * kWRows);
+    // packed weights: [blocks][128 rows][64 columns], one 16 KB box per block
+    auto packed_map = [&](CUtensorMap* m, const void* base, int64_t blocks) {
+        const cuuint64_t dims[3] = {(cuuint64_t)BK, (cuuint64_t)kWRows, (cuuint64_t)blocks};
+        const cuuint64_t str[2] = {(cuuint64_t)BK * 2, (cuuint64_t)kWBytes};
+        const cuuint32_t box[3] = {BK, kWRows, 1};
+        return make_map(m, base, 3, dims, str, box);
+    };
+    if (packed) {
+        if (!packed_map(&mw1, w13, (int64_t)n_experts * 2 * nwt1 * ((H + BK - 1) / BK)) ||
+            !packed_map(&mw2, w2, (int64_t)n_experts * 2 * nwt2 * ((I + BK - 1) / BK)))
+            return cudaErrorInvalidValue;
+    } else {   // W13 as [E, 2, I, H]: a box of 64 gate rows and the 64 matching up rows
         const cuuint64_t dims[4] = {(cuuint64_t)H, (cuuint64_t)I, 2, (cuuint64_t)n_experts};
         const cuuint64_t str[3] = {(cuuint64_t)H * 2, (cuuint64_t)I * H * 2,
                                    (cuuint64_t)2 * I * H * 2};
@@ -699,7 +718,7 @@ cudaError_t launch_grouped_gemm_tc_swap(const __nv_bfloat16* a, const int32_t* o
         if (!make_map(&mw1, w13, 4, dims, str, box)) return cudaErrorInvalidValue;
     }
     if (!g && !make_row_maps(mt1, a, H, n_rows)) return cudaErrorInvalidValue;
-    {   // W2 as [E, H, I]: a box of 128 rows
+    if (!packed) {   // W2 as [E, H, I]: a box of 128 rows
         const cuuint64_t dims[3] = {(cuuint64_t)I, (cuuint64_t)H, (cuuint64_t)n_experts};
         const cuuint64_t str[2] = {(cuuint64_t)I * 2, (cuuint64_t)H * I * 2};
         const cuuint32_t box[3] = {BK, kWRows, 1};
@@ -707,8 +726,8 @@ cudaError_t launch_grouped_gemm_tc_swap(const __nv_bfloat16* a, const int32_t* o
     }
     if (!make_row_maps(mt2, h, I, n_rows)) return cudaErrorInvalidValue;
 
-    Params p1{offsets, counts, expert_begin, n_experts, H, I, (I + kWRows - 1) / kWRows,
-              (int)n_rows, h, nullptr, dev_status, nullptr, nullptr, 0};
+    Params p1{offsets, counts, expert_begin, n_experts, H, I, nwt1,
+              (int)n_rows, h, nullptr, dev_status, nullptr, nullptr, 0, packed ? 1 : 0};
     cudaError_t e;
     if (g) {
         p1.gather_src = g->src;
@@ -721,8 +740,8 @@ cudaError_t launch_grouped_gemm_tc_swap(const __nv_bfloat16* a, const int32_t* o
     }
     if (e == cudaSuccess && ev_mid) e = cudaEventRecord(ev_mid, s);
     if (e != cudaSuccess) return e;
-    Params p2{offsets, counts, expert_begin, n_experts, I, H, (H + 2 * kWRows - 1) / (2 * kWRows),
-              (int)n_rows, y, y_scales, dev_status, nullptr, nullptr, 0};
+    Params p2{offsets, counts, expert_begin, n_experts, I, H, nwt2,
+              (int)n_rows, y, y_scales, dev_status, nullptr, nullptr, 0, packed ? 1 : 0};
     e = y_dtype == MOE_F32    ? launch_phase<false, float>(mw2, mt2, p2, s)
         : y_dtype == MOE_BF16 ? launch_phase<false, __nv_bfloat16>(mw2, mt2, p2, s)
                               : launch_phase<false, uint8_t>(mw2, mt2, p2, s);

@@ -40,6 +40,10 @@ SIGNATURES = {
     "moe_grouped_gemm_workspace_bytes": ([_I64, _I32, _I32, _I, _I], _SZ),
     "moe_grouped_gemm": ([_P, _I, _P, _P, _P, _I32, _I32, _I64, _I32, _I32, _P, _P, _I, _P, _P,
                           _I, _P, _P, _SZ, _P, _P], _I),
+    "moe_packed_weights_bytes": ([_I32, _I32, _I32, _I32], _SZ),
+    "moe_pack_expert_weights": ([_P, _P, _I32, _I32, _I32, _I, _P, _P, _P], _I),
+    "moe_grouped_gemm_packed": ([_P, _I, _P, _P, _P, _I32, _I32, _I64, _I32, _I32, _P, _P, _I, _P,
+                                 _P, _I, _P, _P, _SZ, _P, _P], _I),
     "moe_combine": ([_P, _I, _P, _P, _P, _I64, _I32, _I32, _P, _I, _P], _I),
     "moe_combine_rank": ([_P, _I, _P, _P, _P, _I64, _I32, _I32, _P, _I32, _I32, _P, _P], _I),
     "moe_reduce_partials": ([_P, _I32, _I64, _I32, _P, _I, _P], _I),
@@ -63,7 +67,7 @@ SIGNATURES = {
 class LayerOptionsC(ctypes.Structure):
     """moe_layer_options (include/moe.h)."""
     _fields_ = [("capacity", _I32), ("route_groups", _I32), ("route_max_groups", _I32),
-                ("fused_gather", _I32), ("all_reduce_form", _I32)]
+                ("fused_gather", _I32), ("all_reduce_form", _I32), ("packed_weights", _I32)]
 
 
 class LayerBuffersC(ctypes.Structure):
@@ -194,6 +198,35 @@ def moe_grouped_gemm(xp, xp_scales, expert_offsets, expert_begin, n_experts, w13
         n_experts, n_rows, H, I, _ptr(w13), _ptr(w2), dtype_code(w13), _ptr(h), _ptr(y),
         dtype_code(y), _ptr(y_scales), _ptr(workspace), ws_bytes, _ptr(dev_status),
         _stream(stream)))
+
+
+def packed_weight_tensors(E, H, I, device):
+    """Empty uint8 buffers for the packed W13 and W2 of E experts."""
+    lib = load_library()
+    return (torch.empty(lib.moe_packed_weights_bytes(E, H, I, 0), dtype=torch.uint8,
+                        device=device),
+            torch.empty(lib.moe_packed_weights_bytes(E, H, I, 1), dtype=torch.uint8,
+                        device=device))
+
+
+def moe_pack_expert_weights(w13, w2, packed13, packed2, stream=None):
+    """Re-lay stacked bf16 weights [E, 2I, H] / [E, H, I] into 16 KB blocks."""
+    E, H, I = w2.shape
+    _check("moe_pack_expert_weights", load_library().moe_pack_expert_weights(
+        _ptr(w13), _ptr(w2), E, H, I, dtype_code(w2), _ptr(packed13), _ptr(packed2),
+        _stream(stream)))
+
+
+def moe_grouped_gemm_packed(xp, xp_scales, expert_offsets, expert_begin, n_experts, packed13,
+                            packed2, H, I, h, y, workspace, dev_status, stream=None,
+                            expert_counts=None, y_scales=None):
+    n_rows = xp.shape[0]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("moe_grouped_gemm_packed", load_library().moe_grouped_gemm_packed(
+        _ptr(xp), dtype_code(xp), _ptr(xp_scales), _ptr(expert_offsets), _ptr(expert_counts),
+        expert_begin, n_experts, n_rows, H, I, _ptr(packed13), _ptr(packed2), MOE_BF16,
+        _ptr(h), _ptr(y), dtype_code(y), _ptr(y_scales), _ptr(workspace), ws_bytes,
+        _ptr(dev_status), _stream(stream)))
 
 
 def moe_combine(y, slot_of_pair, topk_w, out, stream=None, y_scales=None):
@@ -369,7 +402,8 @@ def _events(step_events, stream=None):
 
 def layer_options(wl, buf: "LayerBuffers") -> LayerOptionsC:
     return LayerOptionsC(buf.capacity, wl.route_groups, wl.route_max_groups,
-                         1 if wl.fused_gather else 0, 1 if wl.all_reduce_form else 0)
+                         1 if wl.fused_gather else 0, 1 if wl.all_reduce_form else 0,
+                         1 if getattr(wl, "packed_weights", False) else 0)
 
 
 def moe_layer_forward(wl, logits, x, w13, w2, buf: "LayerBuffers", step_events=None,

@@ -64,6 +64,7 @@ class Workload:
     route_max_groups: int = 0              # M: groups a token may reach (with route_groups)
     fused_gather: bool = False             # the gate/up GEMM gathers rows from x (no xp copy)
     all_reduce_form: bool = False          # combine as W per-rank partials summed over ranks
+    packed_weights: bool = False           # expert weights re-laid out in 16 KB blocks
 
     @property
     def N(self) -> int:
@@ -110,6 +111,15 @@ WORKLOADS = {
                                "bf16", all_reduce_form=True),
     "decode_allreduce": Workload("decode_allreduce", 64, 7168, 256, 8, 2048, 8, "bf16", "bf16",
                                  "bf16", all_reduce_form=True),
+    # expert weights re-laid out once (moe_pack_expert_weights) into 16 KB blocks
+    "dsv3_packed": Workload("dsv3_packed", 8192, 7168, 256, 8, 2048, 8, "bf16", "e4m3", "bf16",
+                            packed_weights=True),
+    "mid_packed": Workload("mid_packed", 4096, 2048, 64, 6, 1408, 4, "bf16", "bf16", "bf16",
+                           packed_weights=True),
+    "skew_packed": Workload("skew_packed", 16384, 2880, 128, 4, 2880, 8, "bf16", "bf16", "bf16",
+                            router="zipf", packed_weights=True),
+    "decode_packed": Workload("decode_packed", 64, 7168, 256, 8, 2048, 8, "bf16", "bf16", "bf16",
+                              packed_weights=True),
 }
 
 TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16,

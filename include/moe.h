@@ -323,6 +323,44 @@ moe_status moe_grouped_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_
                             size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /*
+ * moe_pack_expert_weights -- one-time re-layout of the stacked expert
+ * weights (W13 [E, 2I, H], W2 [E, H, I], bf16) into blocks of 128 rows x
+ * 64 columns, each 16 KB block contiguous, in the order the grouped GEMM
+ * reads them: W13 block (e, f, c) holds gate features [64f, 64f+64) and the
+ * matching up features of columns [64c, 64c+64); W2 block (e, r, c) rows
+ * [128r, 128r+128) of columns [64c, 64c+64).  Rows and columns past the
+ * matrices are zero.  In the stacked layout a 128-row tile of one k-step is
+ * 128 pieces of 128 bytes, H*2 (or I*2) bytes apart; packed, it is one
+ * contiguous read.  The values are unchanged: moe_grouped_gemm_packed on the
+ * packed weights computes exactly moe_grouped_gemm's results.
+ *   w13, w2             stacked weights (either may be NULL to pack only
+ *                       the other), 16-byte aligned, device.
+ *   packed13, packed2   outputs of moe_packed_weights_bytes(E, H, I, 0) and
+ *                       (..., 1) bytes, 16-byte aligned, device.
+ * Requires w_dtype MOE_BF16, H % 8 == 0, I % 8 == 0.  A shard of experts
+ * [a, b) packs from the stacked shard w13[a:b], w2[a:b] with E = b - a.
+ */
+size_t moe_packed_weights_bytes(int32_t E, int32_t H, int32_t I, int32_t which);
+moe_status moe_pack_expert_weights(const void* w13, const void* w2, int32_t E, int32_t H,
+                                   int32_t I, moe_dtype w_dtype, void* packed13, void* packed2,
+                                   void* stream);
+
+/*
+ * moe_grouped_gemm_packed -- moe_grouped_gemm with the expert weights in
+ * moe_pack_expert_weights' layout (bf16 weights; the tensor-core kernel
+ * with the weights as the MMA's M operand runs at every size).  Arguments
+ * and results as moe_grouped_gemm, with packed13 / packed2 in place of
+ * w13 / w2 (packed for the n_experts local experts).
+ */
+moe_status moe_grouped_gemm_packed(const void* xp, moe_dtype xp_dtype, const float* xp_scales,
+                                   const int32_t* expert_offsets, const int32_t* expert_counts,
+                                   int32_t expert_begin, int32_t n_experts, int64_t n_rows,
+                                   int32_t H, int32_t I, const void* packed13,
+                                   const void* packed2, moe_dtype w_dtype, void* h, void* y,
+                                   moe_dtype y_dtype, float* y_scales, void* workspace,
+                                   size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
  * moe_combine -- un-permute plus the router-weighted sum of each token's k
  * expert outputs into its home row:
  *     out[t] = sum_{j=0..k-1} topk_w[t,j] * y[slot_of_pair[t*k+j]],
@@ -485,7 +523,7 @@ moe_status moe_ep_combine(void* const* y_rows, float* const* y_scales, moe_dtype
  *   owned); b->xp is in payload_dtype (x_dtype or MOE_E4M3), b->y in
  *   y_dtype.
  *   opts (may be NULL: capacity -1, route_groups 0, fused_gather 0,
- *   all_reduce_form 0):
+ *   all_reduce_form 0, packed_weights 0):
  *     capacity: -1 for the dropless layout (moe_dispatch_layout; the
  *     permuted buffers have T*k rows), or C >= 0 for fixed slabs of C rows
  *     per expert (moe_dispatch_layout_capacity; E*C rows, dropped pairs
@@ -501,6 +539,8 @@ moe_status moe_ep_combine(void* const* y_rows, float* const* y_scales, moe_dtype
  *     moe_permute's payload dequantises to), written once per token into
  *     b->gemm_workspace.  h, y and out are the same; b->xp and b->xp_scales
  *     are not written.  Elsewhere the flag is ignored.
+ *     packed_weights: 1 when w13 and w2 hold moe_pack_expert_weights'
+ *     output (bf16 weights; the GEMM then runs as moe_grouped_gemm_packed).
  *     all_reduce_form: 0 runs moe_combine.  1 runs the combine of the
  *     all_reduce form on the W logical ranks: moe_combine_rank for r = 0..W-1
  *     into b->partials[r], then moe_reduce_partials into out (the same sum,
@@ -521,6 +561,7 @@ typedef struct moe_layer_options {
     int32_t route_max_groups;  /* M: groups each token may reach (with route_groups) */
     int32_t fused_gather;      /* 0: permute, then the GEMM; 1: the GEMM gathers the rows */
     int32_t all_reduce_form;   /* 0: one combine; 1: W per-rank partials, then their sum */
+    int32_t packed_weights;    /* 0: w13/w2 stacked; 1: in moe_pack_expert_weights' layout */
 } moe_layer_options;
 
 typedef struct moe_layer_buffers {

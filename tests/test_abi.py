@@ -274,6 +274,26 @@ def test_ep_calls_reject_before_launch(lib):
     assert moe.moe_status_str(6) == "MOE_ERR_OVERFLOW"
 
 
+def test_pack_calls_reject_before_launch(lib):
+    assert lib.moe_packed_weights_bytes(256, 7168, 2048, 0) == 256 * 32 * 112 * 16384
+    assert lib.moe_packed_weights_bytes(256, 7168, 2048, 1) == 256 * 56 * 32 * 16384
+    assert lib.moe_packed_weights_bytes(128, 2880, 2880, 1) == 128 * 24 * 45 * 16384
+    assert lib.moe_packed_weights_bytes(4, 256, 64, 2) == 0
+    f = lib.moe_pack_expert_weights
+    assert f(FAKE, FAKE, 4, 256, 64, moe.MOE_F32, FAKE, FAKE, None) == 1     # bf16 only
+    assert f(FAKE, FAKE, 4, 250, 64, moe.MOE_BF16, FAKE, FAKE, None) == 1    # H % 8
+    assert f(FAKE, FAKE, 4, 256, 64, moe.MOE_BF16, None, FAKE, None) == 1    # no output
+    assert f(None, None, 4, 256, 64, moe.MOE_BF16, FAKE, FAKE, None) == 1    # nothing to pack
+    assert f(ctypes.c_void_p(4100), None, 4, 256, 64, moe.MOE_BF16, FAKE, None, None) == 1
+    g = lib.moe_grouped_gemm_packed
+    base = [FAKE, moe.MOE_BF16, None, FAKE, None, 0, 8, 100, 256, 64, FAKE, FAKE, moe.MOE_BF16,
+            FAKE, FAKE, moe.MOE_F32, None, None, 0, FAKE, None]
+    bad = list(base); bad[12] = moe.MOE_F32            # packed weights are bf16
+    assert g(*bad) == 1
+    bad = list(base); bad[9] = 60                      # I % 8
+    assert g(*bad) == 1
+
+
 def test_grouped_route_rejects_before_launch(lib):
     f = lib.moe_route_topk_grouped
     assert f(FAKE, 10, 8, 2, 3, 1, FAKE, FAKE, None) == 1      # groups must divide E
