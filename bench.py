@@ -662,7 +662,7 @@ def run_ep(args, wl):
                 "gpu_launches": int(launches), "clocks": clk.summary(ms)}
         print(json.dumps(line), flush=True)
     if ws > 1:
-        del runner
+        runner.close()
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
 

@@ -22,6 +22,9 @@
 // ranks are run on one device.  No TMA and no cluster multicast touch
 // another GPU's memory; the grouped GEMM reads only the local receive
 // buffer.
+#include <cuda.h>
+#include <string.h>
+
 #include "common.cuh"
 
 namespace moe {
@@ -183,6 +186,78 @@ moe_status moe_ep_combine(void* const* y_rows, float* const* y_scales, moe_dtype
     return moe::report_cuda(moe::launch_combine_from(src, y_dtype, slot_of_pair, map, topk_w, T,
                                                      k, H, out, out_dtype, dev_status,
                                                      (cudaStream_t)stream, nullptr, 0));
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- buffer sharing
+// A rank hands its receive and output buffers to the other processes as
+// CUDA IPC handles (the allocation's handle plus the buffer's offset inside
+// it), and maps theirs the same way; the mapped addresses fill the buffer
+// tables of moe_ep_dispatch and moe_ep_combine.  No multicast object is
+// created.
+
+namespace {
+
+struct IpcRecord {
+    cudaIpcMemHandle_t handle;
+    uint64_t offset;
+};
+
+using MemGetAddressRangeFn = CUresult (*)(CUdeviceptr*, size_t*, CUdeviceptr);
+
+MemGetAddressRangeFn mem_get_address_range() {
+    static const MemGetAddressRangeFn fn = [] {
+        void* q = nullptr;
+        cudaDriverEntryPointQueryResult r;
+        if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &q, cudaEnableDefault, &r) ==
+                cudaSuccess &&
+            r == cudaDriverEntryPointSuccess)
+            return (MemGetAddressRangeFn)q;
+        return (MemGetAddressRangeFn) nullptr;
+    }();
+    return fn;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_ipc_handle_bytes(void) { return sizeof(IpcRecord); }
+
+moe_status moe_ipc_export(const void* ptr, void* record) {
+    if (!ptr || !record) return MOE_ERR_INVALID_ARG;
+    const MemGetAddressRangeFn range = mem_get_address_range();
+    if (!range) return moe::report_cuda(cudaErrorInitializationError);
+    CUdeviceptr base = 0;
+    size_t size = 0;
+    if (range(&base, &size, (CUdeviceptr)ptr) != CUDA_SUCCESS)
+        return moe::report_cuda(cudaErrorInvalidValue);
+    IpcRecord rec{};
+    const cudaError_t e = cudaIpcGetMemHandle(&rec.handle, (void*)base);
+    if (e != cudaSuccess) return moe::report_cuda(e);
+    rec.offset = (uint64_t)((CUdeviceptr)ptr - base);
+    memcpy(record, &rec, sizeof(rec));
+    return MOE_OK;
+}
+
+moe_status moe_ipc_import(const void* record, void** ptr) {
+    if (!record || !ptr) return MOE_ERR_INVALID_ARG;
+    IpcRecord rec;
+    memcpy(&rec, record, sizeof(rec));
+    void* base = nullptr;
+    const cudaError_t e =
+        cudaIpcOpenMemHandle(&base, rec.handle, cudaIpcMemLazyEnablePeerAccess);
+    if (e != cudaSuccess) return moe::report_cuda(e);
+    *ptr = (char*)base + rec.offset;
+    return MOE_OK;
+}
+
+moe_status moe_ipc_close(const void* record, void* ptr) {
+    if (!record || !ptr) return MOE_ERR_INVALID_ARG;
+    IpcRecord rec;
+    memcpy(&rec, record, sizeof(rec));
+    return moe::report_cuda(cudaIpcCloseMemHandle((char*)ptr - rec.offset));
 }
 
 }  // extern "C"

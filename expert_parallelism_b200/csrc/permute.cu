@@ -64,6 +64,9 @@ __global__ void __launch_bounds__(256) permute_copy_kernel(const T* __restrict__
         }
         __syncthreads();
     }
+    // rows stored into other GPUs' buffers: make them visible system-wide
+    // before the kernel ends (the owners read them after a barrier)
+    if (map.send_base) __threadfence_system();
 }
 
 // 8 consecutive elements of a row as fp32.
@@ -193,6 +196,7 @@ __global__ void __launch_bounds__(kQuantThreads) permute_e4m3_kernel(
         }
         __syncthreads();
     }
+    if (map.send_base) __threadfence_system();
 }
 
 static unsigned permute_grid(int64_t T) {

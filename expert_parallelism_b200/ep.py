@@ -22,15 +22,14 @@ Two ways to run the W ranks:
     The kernels of different ranks never wait for one another (stream
     order is the only synchronisation), so this is an exact stand-in for
     the data flow, not for its timing.
-  - ``DistributedEP``: one process per GPU of an NVLink domain.  The
-    receive and output buffers are symmetric-memory allocations whose peer
-    pointers the dispatch stores to and the combine loads from; the count
-    exchange is an all-gather; the barriers are the symmetric-memory
-    barrier.  No TMA or cluster multicast reads another GPU's memory.
+  - ``DistributedEP``: one process per GPU of an NVLink domain.  Each
+    rank maps the other ranks' receive and output buffers through CUDA IPC
+    records; the dispatch stores to them and the combine loads from them
+    (peer memory over NVLink); the count exchange is an all-gather; the
+    barriers are stream-ordered collectives.  No TMA or cluster multicast
+    reads another GPU's memory.
 """
 from __future__ import annotations
-
-import os
 
 import torch
 
@@ -151,44 +150,74 @@ class EmulatedEP:
 
 def exchange_counts(expert_counts: torch.Tensor, counts_all: torch.Tensor, group=None):
     """The count exchange: counts_all[s] = rank s's expert_counts on every
-    rank (an all-gather; NCCL on GPUs, gloo on CPU)."""
+    rank (an all-gather: NCCL on GPU tensors; a gloo group takes the counts
+    through host memory)."""
     import torch.distributed as dist
+    if expert_counts.is_cuda and dist.get_backend(group) != "nccl":
+        host = torch.empty(counts_all.shape, dtype=counts_all.dtype)
+        dist.all_gather(list(host.unbind(0)), expert_counts.cpu(), group=group)
+        counts_all.copy_(host)
+        return counts_all
     dist.all_gather(list(counts_all.unbind(0)), expert_counts.contiguous(), group=group)
     return counts_all
 
 
 class DistributedEP:
-    """One expert-parallel rank per process and GPU.  Receive and output
-    buffers live in symmetric memory, so every rank holds device pointers to
-    every other rank's buffers (peer-mapped over NVLink); multicast objects
-    are not requested."""
+    """One expert-parallel rank per process.  Every rank exports its receive
+    and output buffers as CUDA IPC records (moe_ipc_export), gathers the
+    others' records, and maps them (moe_ipc_import): the tables that the
+    dispatch stores through and the combine loads through then hold the
+    peers' buffers (peer memory over NVLink between GPUs).  No multicast
+    object is created and no TMA load reads a peer's memory.
+
+    Barriers: with NCCL, a one-element all-reduce on the compute stream
+    (ordered after this rank's kernels and before its next ones); with gloo
+    (several processes sharing one GPU, as in the tests), the device is
+    synchronised and the host group meets."""
 
     def __init__(self, wl, group=None, device=None):
         import torch.distributed as dist
-        import torch.distributed._symmetric_memory as symm
-        os.environ.setdefault("TORCH_SYMM_MEM_DISABLE_MULTICAST", "1")
+        self.dist = dist
         self.group = group or dist.group.WORLD
         self.world = dist.get_world_size(self.group)
         self.rank = dist.get_rank(self.group)
+        self.nccl = dist.get_backend(self.group) == "nccl"
         self.wl = wl
         dev = device or torch.device("cuda", torch.cuda.current_device())
         self.cap = recv_capacity_rows(wl, self.world)
-        self.handles = []
+        self.state = RankState(wl, self.world, dev, self.cap)
+        self._tick = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.imported = []
+        S = self.state
+        self.recv_rows = self._share(S.recv)
+        self.recv_scales = self._share(S.recv_scales)
+        self.y_rows = self._share(S.y)
+        self.y_scales = self._share(S.y_scales)
 
-        def alloc(shape, dtype):
-            t = symm.empty(*shape, dtype=dtype, device=dev)
-            self.handles.append((t, symm.rendezvous(t, self.group)))
-            return t
-
-        self.state = RankState(wl, self.world, dev, self.cap, alloc=alloc)
-        by_ptr = {t.data_ptr(): h for t, h in self.handles}
-        ptrs = lambda t: None if t is None else list(by_ptr[t.data_ptr()].buffer_ptrs)
-        self.recv_rows, self.recv_scales = ptrs(self.state.recv), ptrs(self.state.recv_scales)
-        self.y_rows, self.y_scales = ptrs(self.state.y), ptrs(self.state.y_scales)
-        self.barrier_handle = self.handles[0][1]
+    def _share(self, t):
+        """Every rank's address of the buffer ``t`` of each rank (its own
+        pointer at its own index)."""
+        if t is None:
+            return None
+        rec = moe.moe_ipc_export(t)
+        recs = [None] * self.world
+        self.dist.all_gather_object(recs, rec, group=self.group)
+        ptrs = []
+        for r, other in enumerate(recs):
+            if r == self.rank:
+                ptrs.append(t.data_ptr())
+            else:
+                p = moe.moe_ipc_import(other)
+                self.imported.append((other, p))
+                ptrs.append(p)
+        return ptrs
 
     def barrier(self):
-        self.barrier_handle.barrier(channel=0)
+        if self.nccl:
+            self.dist.all_reduce(self._tick, group=self.group)
+        else:
+            torch.cuda.synchronize()
+            self.dist.barrier(group=self.group)
 
     def forward(self, logits, x, w13_local, w2_local, stream=None):
         S = self.state
@@ -202,3 +231,10 @@ class DistributedEP:
         S.combine(self.y_rows, self.y_scales, stream=stream)
         self.barrier()                       # nobody reads this rank's y any more
         return S.out
+
+    def close(self):
+        """Unmaps the peers' buffers (every rank, after its last forward)."""
+        torch.cuda.synchronize()
+        for rec, p in self.imported:
+            moe.moe_ipc_close(rec, p)
+        self.imported = []

@@ -59,6 +59,10 @@ SIGNATURES = {
                          _P, _P], _I),
     "moe_ep_combine": ([_P, _P, _I, _P, _P, _P, _P, _P, _I64, _I32, _I32, _I32, _I32, _I64, _P,
                         _I, _P, _P], _I),
+    "moe_ipc_handle_bytes": ([], _SZ),
+    "moe_ipc_export": ([_P, _P], _I),
+    "moe_ipc_import": ([_P, ctypes.POINTER(ctypes.c_void_p)], _I),
+    "moe_ipc_close": ([_P, _P], _I),
     "moe_diag_layout_wait_timeout_workspace_bytes": ([], _SZ),
     "moe_diag_layout_wait_timeout": ([_P, _SZ, ctypes.c_uint64, _P, _P], _I),
 }
@@ -265,6 +269,29 @@ def _ptr_array(ptrs):
     vals = [None if p is None else (p.data_ptr() if isinstance(p, torch.Tensor) else int(p))
             for p in ptrs]
     return (ctypes.c_void_p * len(vals))(*vals)
+
+
+def moe_ipc_export(t: torch.Tensor) -> bytes:
+    """IPC record (handle of the allocation + the tensor's offset) of a
+    device tensor, as bytes to send to another process."""
+    lib = load_library()
+    rec = ctypes.create_string_buffer(lib.moe_ipc_handle_bytes())
+    _check("moe_ipc_export", lib.moe_ipc_export(_ptr(t), rec))
+    return rec.raw
+
+
+def moe_ipc_import(record: bytes) -> int:
+    """Device address, in this process, of the buffer another process
+    exported."""
+    lib = load_library()
+    out = ctypes.c_void_p()
+    _check("moe_ipc_import", lib.moe_ipc_import(ctypes.c_char_p(record), ctypes.byref(out)))
+    return int(out.value)
+
+
+def moe_ipc_close(record: bytes, ptr: int):
+    _check("moe_ipc_close", load_library().moe_ipc_close(ctypes.c_char_p(record),
+                                                          ctypes.c_void_p(ptr)))
 
 
 def moe_ep_plan(counts_all, rank, send_base, recv_offsets, dev_status, stream=None):

@@ -510,6 +510,30 @@ moe_status moe_ep_combine(void* const* y_rows, float* const* y_scales, moe_dtype
                           int32_t* dev_status, void* stream);
 
 /*
+ * Buffer sharing between processes for the expert-parallel tables: a rank
+ * exports each receive / output buffer as a record of
+ * moe_ipc_handle_bytes() bytes (the CUDA IPC handle of the allocation that
+ * holds it, and the buffer's offset inside that allocation), sends the
+ * records to the other ranks by any host means, and every rank maps the
+ * others' buffers with moe_ipc_import; the mapped addresses (peer memory
+ * over NVLink) go into the W-entry tables.  moe_ipc_close unmaps.  The
+ * buffer must come from cudaMalloc (for example PyTorch's default caching
+ * allocator, not its expandable segments); no multicast object is created.
+ *   moe_ipc_export: ptr a device pointer of this process; record written
+ *                   (host memory).
+ *   moe_ipc_import: record from another process; *ptr receives the mapped
+ *                   address of the same buffer (cudaIpcOpenMemHandle, peer
+ *                   access enabled lazily).  A record of this same process
+ *                   cannot be imported (CUDA refuses it).
+ *   moe_ipc_close:  the record and the address moe_ipc_import gave.
+ * CUDA failures return MOE_ERR_CUDA.
+ */
+size_t moe_ipc_handle_bytes(void);
+moe_status moe_ipc_export(const void* ptr, void* record);
+moe_status moe_ipc_import(const void* record, void** ptr);
+moe_status moe_ipc_close(const void* record, void* ptr);
+
+/*
  * moe_layer_forward -- the whole hot path in one call: moe_route_topk,
  * moe_dispatch_layout, moe_permute, moe_grouped_gemm (every expert, local
  * expert j = global expert j) and moe_combine, in that order on `stream`,

@@ -272,6 +272,11 @@ def test_ep_calls_reject_before_launch(lib):
     assert c(*cargs(yd=moe.MOE_E4M3)) == 1                     # FP8 y needs the scale table
     assert c(*cargs(out=ctypes.c_void_p(4100))) == 1            # misaligned out
     assert moe.moe_status_str(6) == "MOE_ERR_OVERFLOW"
+    rec = ctypes.create_string_buffer(lib.moe_ipc_handle_bytes())
+    assert lib.moe_ipc_handle_bytes() >= 64
+    assert lib.moe_ipc_export(None, rec) == 1
+    assert lib.moe_ipc_import(None, ctypes.byref(ctypes.c_void_p())) == 1
+    assert lib.moe_ipc_close(rec, None) == 1
 
 
 def test_pack_calls_reject_before_launch(lib):
