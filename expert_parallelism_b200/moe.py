@@ -427,6 +427,13 @@ def _events(step_events, stream=None):
     return ctypes.cast(arr, ctypes.c_void_p), arr
 
 
+def _weight_code(wl) -> int:
+    """The weights' dtype code from the workload (packed weights live in byte
+    buffers, so their tensors do not carry it)."""
+    from .workloads import TORCH_DTYPE
+    return _DT[TORCH_DTYPE[wl.wdt]]
+
+
 def layer_options(wl, buf: "LayerBuffers") -> LayerOptionsC:
     return LayerOptionsC(buf.capacity, wl.route_groups, wl.route_max_groups,
                          1 if wl.fused_gather else 0, 1 if wl.all_reduce_form else 0,
@@ -442,7 +449,7 @@ def moe_layer_forward(wl, logits, x, w13, w2, buf: "LayerBuffers", step_events=N
     ev = _events(step_events, stream)
     _check("moe_layer_forward", load_library().moe_layer_forward(
         _ptr(logits), _ptr(x), dtype_code(x), wl.T, wl.H, wl.E, wl.k, wl.W, wl.I, _ptr(w13),
-        _ptr(w2), dtype_code(w13), dtype_code(buf.xp), dtype_code(buf.y),
+        _ptr(w2), _weight_code(wl), dtype_code(buf.xp), dtype_code(buf.y),
         ctypes.byref(layer_options(wl, buf)), ctypes.byref(cb), _ptr(buf.out),
         ev[0] if ev else None, _stream(stream)))
     return buf.out
@@ -456,7 +463,7 @@ def moe_layer_forward_host(wl, logits_host, x_host, out_host, logits_dev, x_dev,
     _check("moe_layer_forward_host", load_library().moe_layer_forward_host(
         _ptr(logits_host), _ptr(x_host), _ptr(out_host), _ptr(logits_dev), _ptr(x_dev),
         _ptr(buf.out), dtype_code(x_dev), wl.T, wl.H, wl.E, wl.k, wl.W, wl.I, _ptr(w13), _ptr(w2),
-        dtype_code(w13), dtype_code(buf.xp), dtype_code(buf.y),
+        _weight_code(wl), dtype_code(buf.xp), dtype_code(buf.y),
         ctypes.byref(layer_options(wl, buf)), ctypes.byref(cb), ev[0] if ev else None,
         _stream(stream)))
 

@@ -35,8 +35,11 @@ def _rank_main(rank, world, port, payload, q):
     import oracle
     from expert_parallelism_b200 import ep, moe, workloads
     from parity_helpers import BF16_TOL, bits, rowwise_ok
+    import datetime
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
-    dist.init_process_group("gloo", rank=rank, world_size=world)
+    # a short group timeout: a rank that fails ends the other's next collective
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
     try:
         dev = torch.device("cuda:0")
         torch.cuda.set_device(dev)
@@ -80,7 +83,11 @@ def test_expert_parallel_processes_over_ipc(payload, cuda_device):
         p.start()
     for p in procs:
         p.join(300)
-        assert p.exitcode == 0
+    for p in procs:
+        if p.exitcode is None:
+            p.terminate()
+            p.join(10)
+    assert [p.exitcode for p in procs] == [0] * world
     res = sorted(q.get(timeout=10) for _ in range(world))
     for rank, st, same, ok, worst in res:
         assert st == 0, (rank, st)
