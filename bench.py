@@ -347,6 +347,7 @@ def _config(wl):
                if wl.route_groups else {}),
             "fused_gather": wl.fused_gather,
             **({"packed_weights": True} if wl.packed_weights else {}),
+            **({"weights_in_gemm": True} if wl.weights_in_gemm else {}),
             **({"all_reduce_form": True} if wl.all_reduce_form else {}),
             "parallelism": "replicas (one independent layer per GPU)"}
 

@@ -31,7 +31,8 @@ cudaError_t launch_grouped_gemm_simt_f32(const float*, const int32_t*, const int
 cudaError_t launch_grouped_gemm_tc(const __nv_bfloat16*, const int32_t*, const int32_t*, int, int,
                                    int64_t, int, int, const __nv_bfloat16*, const __nv_bfloat16*,
                                    __nv_bfloat16*, void*, moe_dtype, float*, int32_t*,
-                                   const gemm_gather*, cudaEvent_t, cudaStream_t, bool);
+                                   const gemm_gather*, cudaEvent_t, cudaStream_t, bool,
+                                   const float*, const int32_t*);
 size_t packed_weights_bytes(int64_t E, int H, int I, int which);
 cudaError_t launch_pack_weights(const __nv_bfloat16*, const __nv_bfloat16*, int64_t, int, int,
                                 __nv_bfloat16*, __nv_bfloat16*, cudaStream_t);
@@ -179,7 +180,8 @@ moe_status check_combine(const void* y, moe_dtype y_dtype, const float* y_scales
     if (y_dtype == MOE_E4M3 && ((H % 128) != 0 || !y_scales)) return MOE_ERR_INVALID_ARG;
     if (k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
     if (T == 0) return *noop = true, MOE_OK;
-    if (!y || !slot_of_pair || !topk_w || !out || !aligned16(y) || !aligned16(out))
+    // topk_w may be null: unit weights (outputs that already carry them)
+    if (!y || !slot_of_pair || !out || !aligned16(y) || !aligned16(out))
         return MOE_ERR_INVALID_ARG;
     return MOE_OK;
 }
@@ -194,7 +196,8 @@ cudaError_t run_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_scales,
                      moe_dtype w_dtype, void* h, void* y, moe_dtype y_dtype, float* y_scales,
                      void* workspace, int32_t* dev_status, cudaStream_t s,
                      cudaEvent_t ev_a = nullptr, cudaEvent_t ev_b = nullptr,
-                     bool a_ready = false, const gemm_gather* g = nullptr, bool packed = false) {
+                     bool a_ready = false, const gemm_gather* g = nullptr, bool packed = false,
+                     const float* row_weights = nullptr, const int32_t* weight_pairs = nullptr) {
     cudaError_t e = cudaSuccess;
     if (w_dtype == MOE_F32) {
         if (ev_a) e = cudaEventRecord(ev_a, s);
@@ -219,7 +222,7 @@ cudaError_t run_gemm(const void* xp, moe_dtype xp_dtype, const float* xp_scales,
                                   n_rows, H, I,
                                   (const __nv_bfloat16*)w13, (const __nv_bfloat16*)w2,
                                   (__nv_bfloat16*)h, y, y_dtype, y_scales, dev_status, g, ev_b,
-                                  s, packed);
+                                  s, packed, row_weights, weight_pairs);
 }
 
 }  // namespace
@@ -404,7 +407,7 @@ static int64_t layer_slots(int64_t T, int32_t k, int32_t E, int32_t capacity) {
 }
 
 static moe_layer_options resolve(const moe_layer_options* o) {
-    return o ? *o : moe_layer_options{-1, 0, 0, 0, 0, 0};
+    return o ? *o : moe_layer_options{-1, 0, 0, 0, 0, 0, 0};
 }
 
 static moe_status check_layer(const float* logits, const void* x, moe_dtype x_dtype, int64_t T,
@@ -439,8 +442,9 @@ static moe_status check_layer(const float* logits, const void* x, moe_dtype x_dt
     // the all_reduce form: W fp32 partials of [T, H]
     if (st == MOE_OK && o.all_reduce_form != 0 && T > 0 && (!b->partials || !aligned16(b->partials)))
         st = MOE_ERR_INVALID_ARG;
-    // packed weights exist for bf16 weights only
-    if (st == MOE_OK && o.packed_weights != 0 && w_dtype != MOE_BF16) st = MOE_ERR_INVALID_ARG;
+    // packed weights and router weights in the GEMM: bf16 weights only
+    if (st == MOE_OK && (o.packed_weights != 0 || o.weights_in_gemm != 0) && w_dtype != MOE_BF16)
+        st = MOE_ERR_INVALID_ARG;
     // the fused gather's FP8 source, one bf16 row per token, lives in the
     // GEMM workspace
     if (st == MOE_OK && o.fused_gather != 0 && payload_dtype == MOE_E4M3 && T > 0 &&
@@ -493,21 +497,25 @@ static cudaError_t launch_layer(const float* logits, const void* x, moe_dtype x_
                      capacity < 0 ? nullptr : b->expert_counts, 0, E, n_slots, H, I, w13, w2,
                      w_dtype, b->h, b->y, y_dtype, b->y_scales, b->gemm_workspace, b->dev_status,
                      s, ev ? (cudaEvent_t)ev[4] : nullptr, ev ? (cudaEvent_t)ev[5] : nullptr,
-                     /*a_ready=*/true, gather ? &gsrc : nullptr, o.packed_weights != 0);
+                     /*a_ready=*/true, gather ? &gsrc : nullptr, o.packed_weights != 0,
+                     o.weights_in_gemm != 0 ? b->topk_w : nullptr,
+                     o.weights_in_gemm != 0 ? b->pair_of_slot : nullptr);
     } else if (e == cudaSuccess) {
         e = mark(4);
         if (e == cudaSuccess) e = mark(5);
     }
     if (e == cudaSuccess) e = mark(6);
+    // with the router weights applied in the GEMM, the combine is a plain sum
+    const float* comb_w = o.weights_in_gemm != 0 ? nullptr : b->topk_w;
     if (e == cudaSuccess && T > 0 && o.all_reduce_form != 0) {
         // each logical rank's partial over its own slab, then their sum in
         // rank order (on W GPUs: the all-reduce) rounded once
         for (int r = 0; r < W && e == cudaSuccess; ++r)
-            e = launch_combine(b->y, y_dtype, b->y_scales, b->slot_of_pair, b->topk_w, T, k, H,
+            e = launch_combine(b->y, y_dtype, b->y_scales, b->slot_of_pair, comb_w, T, k, H,
                                b->partials + (int64_t)r * T * H, MOE_F32, s, b->rank_offsets, r);
         if (e == cudaSuccess) e = launch_reduce_partials(b->partials, W, T * H, out, x_dtype, s);
     } else if (e == cudaSuccess && T > 0) {
-        e = launch_combine(b->y, y_dtype, b->y_scales, b->slot_of_pair, b->topk_w, T, k, H, out,
+        e = launch_combine(b->y, y_dtype, b->y_scales, b->slot_of_pair, comb_w, T, k, H, out,
                            x_dtype, s);
     }
     if (e == cudaSuccess) e = mark(7);

@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(kCombineMaxThreads, 2) combine_kernel(const __
             }
             s_rank[threadIdx.x] = (sl >= lo && sl < hi) ? r : -1;
             s_row[threadIdx.x] = row;
-            s_w[threadIdx.x] = topk_w[p];
+            s_w[threadIdx.x] = topk_w ? topk_w[p] : 1.0f;   // null: unit weights
         }
         __syncthreads();
         for (int c = threadIdx.x; c < nchunk; c += blockDim.x) {

@@ -475,7 +475,8 @@ cudaError_t launch_grouped_gemm_tc_swap(const __nv_bfloat16* a, const int32_t* o
                                         const __nv_bfloat16* w2, __nv_bfloat16* h, void* y,
                                         moe_dtype y_dtype, float* y_scales, int32_t* dev_status,
                                         const gemm_gather* g, cudaEvent_t ev_mid, cudaStream_t s,
-                                        bool packed);
+                                        bool packed, const float* row_weights,
+                                        const int32_t* weight_pairs);
 
 // Kernel choice, from the average rows per expert (known on the host
 // without reading the device offsets).  The operand-swapped pair kernel
@@ -503,19 +504,21 @@ bool grouped_gemm_tc_uses_swap(int64_t n_rows, int n_experts, moe_dtype y_dtype)
 // kernel only): the gate/up operand's rows are gathered from g->src instead
 // of read from A.  ev_mid (may be null) is recorded between the two phases.
 // packed: the weights are in pack_weights.cu's layout (operand-swapped
-// kernel).
+// kernel).  row_weights (may be null; operand-swapped kernel): y row s is
+// scaled by row_weights[weight_pairs[s]].
 cudaError_t launch_grouped_gemm_tc(const __nv_bfloat16* a, const int32_t* offsets,
                                    const int32_t* counts, int expert_begin, int n_experts,
                                    int64_t n_rows, int H, int I, const __nv_bfloat16* w13,
                                    const __nv_bfloat16* w2, __nv_bfloat16* h, void* y,
                                    moe_dtype y_dtype, float* y_scales, int32_t* dev_status,
                                    const gemm_gather* g, cudaEvent_t ev_mid, cudaStream_t s,
-                                   bool packed) {
-    // packed weights: the operand-swapped kernel reads them at any size
-    if (packed || grouped_gemm_tc_uses_swap(n_rows, n_experts, y_dtype))
+                                   bool packed, const float* row_weights,
+                                   const int32_t* weight_pairs) {
+    // packed weights and row weights: the operand-swapped kernel, at any size
+    if (packed || row_weights || grouped_gemm_tc_uses_swap(n_rows, n_experts, y_dtype))
         return launch_grouped_gemm_tc_swap(a, offsets, counts, expert_begin, n_experts, n_rows, H,
                                            I, w13, w2, h, y, y_dtype, y_scales, dev_status, g,
-                                           ev_mid, s, packed);
+                                           ev_mid, s, packed, row_weights, weight_pairs);
     if (g) return cudaErrorInvalidValue;
     return tc::run_gemm<1>(a, offsets, counts, expert_begin, n_experts, n_rows, H, I, w13, w2, h,
                            y, y_dtype == MOE_F32, dev_status, ev_mid, s);

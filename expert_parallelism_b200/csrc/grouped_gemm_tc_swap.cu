@@ -144,7 +144,19 @@ struct Params {
     // weights in the packed layout (pack_weights.cu): one contiguous 16 KB
     // block per (expert, 64 or 128 weight rows, 64-column k-step)
     int packed;
+    // phase 2 only, may be null: y row s is multiplied by
+    // row_weights[pair_of_slot[s]] (0 for a slot holding no pair)
+    const float* row_weights;
+    const int32_t* weight_pairs;
 };
+
+// Router weight of routed row `row` (phase 2 with row weights), 0 past the
+// pass or for a slot holding no pair.
+__device__ __forceinline__ float row_weight(const Params& p, int64_t row, int row_end) {
+    if (row >= row_end) return 0.0f;
+    const int32_t pr = __ldg(p.weight_pairs + row);
+    return pr >= 0 ? __ldg(p.row_weights + pr) : 0.0f;
+}
 
 // Passes an expert with `rows` routed rows takes.
 struct PassesOf {
@@ -527,6 +539,11 @@ __global__ void __launch_bounds__(threads_of<GATHER>(), 1)
                         // then takes chunk row l: its amax over this warp's 32
                         // outputs, the block amax over the group's four warps, and
                         // 32 codes (32 bytes) of the row's 128-wide block
+                        if (p.row_weights) {   // the routed row's router weight, first
+                            const float wl = row_weight(p, crow0 + col + lane, row_end);
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) v[i] *= __shfl_sync(0xffffffffu, wl, i);
+                        }
 #pragma unroll
                         for (int i = 0; i < 32; ++i) out_stage[i * kOutPitch + lane] = v[i];
                         __syncwarp();
@@ -570,6 +587,11 @@ __global__ void __launch_bounds__(threads_of<GATHER>(), 1)
                         __syncwarp();
                     } else {
                         // this warp: 32 outputs (its lanes) x 32 chunk rows (v)
+                        if (p.row_weights) {   // y row = router weight x expert output
+                            const float wl = row_weight(p, crow0 + col + lane, row_end);
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) v[i] *= __shfl_sync(0xffffffffu, wl, i);
+                        }
 #pragma unroll
                         for (int i = 0; i < 32; ++i) out_stage[i * kOutPitch + lane] = v[i];
                         __syncwarp();
@@ -688,14 +710,16 @@ static bool make_row_maps(CUtensorMap* m, const void* base, int K, int64_t n_row
 // is recorded between the two phases.  With g (the fused gather) non-null,
 // A is not read: row s of the gate/up operand is row pair_of_slot[s] / k of
 // g.src [*, H] (16-byte aligned).  packed: w13 and w2 are in the packed
-// layout of pack_weights.cu.
+// layout of pack_weights.cu.  row_weights (may be null): y row s is written
+// as row_weights[weight_pairs[s]] times the expert's output.
 cudaError_t launch_grouped_gemm_tc_swap(const __nv_bfloat16* a, const int32_t* offsets,
                                         const int32_t* counts, int expert_begin, int n_experts,
                                         int64_t n_rows, int H, int I, const __nv_bfloat16* w13,
                                         const __nv_bfloat16* w2, __nv_bfloat16* h, void* y,
                                         moe_dtype y_dtype, float* y_scales, int32_t* dev_status,
                                         const gemm_gather* g, cudaEvent_t ev_mid,
-                                        cudaStream_t s, bool packed) {
+                                        cudaStream_t s, bool packed, const float* row_weights,
+                                        const int32_t* weight_pairs) {
     using namespace tcs;
     CUtensorMap mw1, mt1[3], mw2, mt2[3];
     const int nwt1 = (I + kWRows - 1) / kWRows, nwt2 = (H + 2 * kWRows - 1) / (2 * kWRows);
@@ -727,7 +751,8 @@ cudaError_t launch_grouped_gemm_tc_swap(const __nv_bfloat16* a, const int32_t* o
     if (!make_row_maps(mt2, h, I, n_rows)) return cudaErrorInvalidValue;
 
     Params p1{offsets, counts, expert_begin, n_experts, H, I, nwt1,
-              (int)n_rows, h, nullptr, dev_status, nullptr, nullptr, 0, packed ? 1 : 0};
+              (int)n_rows, h, nullptr, dev_status, nullptr, nullptr, 0, packed ? 1 : 0,
+              nullptr, nullptr};
     cudaError_t e;
     if (g) {
         p1.gather_src = g->src;
@@ -741,7 +766,8 @@ cudaError_t launch_grouped_gemm_tc_swap(const __nv_bfloat16* a, const int32_t* o
     if (e == cudaSuccess && ev_mid) e = cudaEventRecord(ev_mid, s);
     if (e != cudaSuccess) return e;
     Params p2{offsets, counts, expert_begin, n_experts, I, H, nwt2,
-              (int)n_rows, y, y_scales, dev_status, nullptr, nullptr, 0, packed ? 1 : 0};
+              (int)n_rows, y, y_scales, dev_status, nullptr, nullptr, 0, packed ? 1 : 0,
+              row_weights, weight_pairs};
     e = y_dtype == MOE_F32    ? launch_phase<false, float>(mw2, mt2, p2, s)
         : y_dtype == MOE_BF16 ? launch_phase<false, __nv_bfloat16>(mw2, mt2, p2, s)
                               : launch_phase<false, uint8_t>(mw2, mt2, p2, s);

@@ -38,8 +38,10 @@ __device__ __forceinline__ void token_dests(const int32_t* __restrict__ slot_of_
     }
 }
 
+constexpr int kPermuteMaxThreads = 512;
+
 template <typename T>
-__global__ void __launch_bounds__(256) permute_copy_kernel(const T* __restrict__ x, int64_t T_,
+__global__ void __launch_bounds__(kPermuteMaxThreads) permute_copy_kernel(const T* __restrict__ x, int64_t T_,
                                                            int H, int k,
                                                            const int32_t* __restrict__ slot_of_pair,
                                                            const PairRows map,
@@ -84,7 +86,6 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&f)[8]) {
     unpack16(ld_nc_v4(p), f);
 }
 
-constexpr int kQuantThreads = 256;
 constexpr int kMaxBlocks = 64;           // scales staged in shared memory: H <= 8192
 
 // FP8 payload: one CTA per token (grid-stride).  8 lanes own a 128-element
@@ -99,7 +100,7 @@ constexpr int kMaxBlocks = 64;           // scales staged in shared memory: H <=
 // `a` is written, at the token's own row t: each token is quantised once and
 // its k copies are the same row.
 template <typename T>
-__global__ void __launch_bounds__(kQuantThreads) permute_e4m3_kernel(
+__global__ void __launch_bounds__(kPermuteMaxThreads) permute_e4m3_kernel(
     const T* __restrict__ x, int64_t T_, int H, int k, const int32_t* __restrict__ slot_of_pair,
     const PairRows map, const __grid_constant__ RankPtrs dst, __nv_bfloat16* __restrict__ a,
     int32_t* dev_status) {
@@ -199,6 +200,16 @@ __global__ void __launch_bounds__(kQuantThreads) permute_e4m3_kernel(
     if (map.send_base) __threadfence_system();
 }
 
+// Threads per CTA for `units` equal pieces of work per token (16-byte
+// vectors, or 8 threads per 128-element FP8 block): as few equal rounds as
+// a CTA of at most 512 threads allows, so no thread idles in the last one.
+static int permute_threads(int units, int per_unit) {
+    const int work = units * per_unit;
+    const int rounds = (work + kPermuteMaxThreads - 1) / kPermuteMaxThreads;
+    const int t = ((work + rounds - 1) / rounds + 31) / 32 * 32;
+    return t < 32 ? 32 : t;
+}
+
 static unsigned permute_grid(int64_t T) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -226,18 +237,19 @@ cudaError_t launch_permute_to(const void* x, moe_dtype xdt, int64_t T, int H, in
     if (T == 0) return cudaSuccess;
     const unsigned grid = permute_grid(T);
     if (xpdt == MOE_E4M3) {
+        const int th = permute_threads(H / 128, 8);
         if (xdt == MOE_BF16)
-            permute_e4m3_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+            permute_e4m3_kernel<__nv_bfloat16><<<grid, th, 0, s>>>(
                 (const __nv_bfloat16*)x, T, H, k, slot_of_pair, map, dst, a_bf16, dev_status);
         else
-            permute_e4m3_kernel<float><<<grid, 256, 0, s>>>((const float*)x, T, H, k, slot_of_pair,
-                                                            map, dst, a_bf16, dev_status);
+            permute_e4m3_kernel<float><<<grid, th, 0, s>>>((const float*)x, T, H, k, slot_of_pair,
+                                                           map, dst, a_bf16, dev_status);
     } else if (xdt == MOE_BF16) {
-        permute_copy_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+        permute_copy_kernel<__nv_bfloat16><<<grid, permute_threads(H * 2 / 16, 1), 0, s>>>(
             (const __nv_bfloat16*)x, T, H, k, slot_of_pair, map, dst, dev_status);
     } else {
-        permute_copy_kernel<float><<<grid, 256, 0, s>>>((const float*)x, T, H, k, slot_of_pair,
-                                                        map, dst, dev_status);
+        permute_copy_kernel<float><<<grid, permute_threads(H * 4 / 16, 1), 0, s>>>(
+            (const float*)x, T, H, k, slot_of_pair, map, dst, dev_status);
     }
     note_launches(1);
     return cudaGetLastError();
@@ -260,12 +272,13 @@ cudaError_t launch_quantize_tokens_e4m3(const void* x, moe_dtype xdt, int64_t T,
     const unsigned grid = permute_grid(T);
     const PairRows local{nullptr, nullptr, nullptr, 1, 0};
     const RankPtrs none = one_rank(nullptr, nullptr);
+    const int th = permute_threads(H / 128, 8);
     if (xdt == MOE_BF16)
-        permute_e4m3_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+        permute_e4m3_kernel<__nv_bfloat16><<<grid, th, 0, s>>>(
             (const __nv_bfloat16*)x, T, H, 1, nullptr, local, none, a, nullptr);
     else
-        permute_e4m3_kernel<float><<<grid, 256, 0, s>>>((const float*)x, T, H, 1, nullptr, local,
-                                                        none, a, nullptr);
+        permute_e4m3_kernel<float><<<grid, th, 0, s>>>((const float*)x, T, H, 1, nullptr, local,
+                                                       none, a, nullptr);
     note_launches(1);
     return cudaGetLastError();
 }

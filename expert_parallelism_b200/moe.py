@@ -71,7 +71,8 @@ SIGNATURES = {
 class LayerOptionsC(ctypes.Structure):
     """moe_layer_options (include/moe.h)."""
     _fields_ = [("capacity", _I32), ("route_groups", _I32), ("route_max_groups", _I32),
-                ("fused_gather", _I32), ("all_reduce_form", _I32), ("packed_weights", _I32)]
+                ("fused_gather", _I32), ("all_reduce_form", _I32), ("packed_weights", _I32),
+                ("weights_in_gemm", _I32)]
 
 
 class LayerBuffersC(ctypes.Structure):
@@ -437,7 +438,8 @@ def _weight_code(wl) -> int:
 def layer_options(wl, buf: "LayerBuffers") -> LayerOptionsC:
     return LayerOptionsC(buf.capacity, wl.route_groups, wl.route_max_groups,
                          1 if wl.fused_gather else 0, 1 if wl.all_reduce_form else 0,
-                         1 if getattr(wl, "packed_weights", False) else 0)
+                         1 if getattr(wl, "packed_weights", False) else 0,
+                         1 if getattr(wl, "weights_in_gemm", False) else 0)
 
 
 def moe_layer_forward(wl, logits, x, w13, w2, buf: "LayerBuffers", step_events=None,

@@ -65,6 +65,7 @@ class Workload:
     fused_gather: bool = False             # the gate/up GEMM gathers rows from x (no xp copy)
     all_reduce_form: bool = False          # combine as W per-rank partials summed over ranks
     packed_weights: bool = False           # expert weights re-laid out in 16 KB blocks
+    weights_in_gemm: bool = False          # router weights applied in the down GEMM's epilogue
 
     @property
     def N(self) -> int:
@@ -120,6 +121,12 @@ WORKLOADS = {
                             router="zipf", packed_weights=True),
     "decode_packed": Workload("decode_packed", 64, 7168, 256, 8, 2048, 8, "bf16", "bf16", "bf16",
                               packed_weights=True),
+    # the router weights applied in the down GEMM's epilogue; the combine sums
+    "dsv3_wgemm": Workload("dsv3_wgemm", 8192, 7168, 256, 8, 2048, 8, "bf16", "e4m3", "bf16",
+                           weights_in_gemm=True),
+    # both halves of the fused row: the gather and the weights in the GEMM
+    "dsv3_fused_wgemm": Workload("dsv3_fused_wgemm", 8192, 7168, 256, 8, 2048, 8, "bf16", "e4m3",
+                                 "bf16", fused_gather=True, weights_in_gemm=True),
 }
 
 TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16,

@@ -377,7 +377,8 @@ moe_status moe_grouped_gemm_packed(const void* xp, moe_dtype xp_dtype, const flo
  *   y_scales     [>= max slot + 1, H/128] fp32 when y_dtype == MOE_E4M3
  *                (H % 128 == 0), else ignored (may be NULL).
  *   slot_of_pair [T*k] int32, device.
- *   topk_w       [T, k] fp32, device.
+ *   topk_w       [T, k] fp32, device; or NULL for unit weights (rows that
+ *                already carry their router weight: out = the k-way sum).
  *   out          [T, H] in out_dtype (MOE_F32 / MOE_BF16), device, written.
  * Requires H % 8 == 0, k >= 1.
  */
@@ -547,7 +548,7 @@ moe_status moe_ipc_close(const void* record, void* ptr);
  *   owned); b->xp is in payload_dtype (x_dtype or MOE_E4M3), b->y in
  *   y_dtype.
  *   opts (may be NULL: capacity -1, route_groups 0, fused_gather 0,
- *   all_reduce_form 0, packed_weights 0):
+ *   all_reduce_form 0, packed_weights 0, weights_in_gemm 0):
  *     capacity: -1 for the dropless layout (moe_dispatch_layout; the
  *     permuted buffers have T*k rows), or C >= 0 for fixed slabs of C rows
  *     per expert (moe_dispatch_layout_capacity; E*C rows, dropped pairs
@@ -565,6 +566,12 @@ moe_status moe_ipc_close(const void* record, void* ptr);
  *     are not written.  Elsewhere the flag is ignored.
  *     packed_weights: 1 when w13 and w2 hold moe_pack_expert_weights'
  *     output (bf16 weights; the GEMM then runs as moe_grouped_gemm_packed).
+ *     weights_in_gemm: 1 (bf16 weights) applies each routed row's router
+ *     weight in the down GEMM's epilogue (y row s = topk_w[pair_of_slot[s]]
+ *     times the expert's output, fp32 product) and makes the combine a plain
+ *     k-way sum in j order (moe_combine with topk_w NULL); out differs from
+ *     the default by the rounding of that product (each pick's w*y is
+ *     rounded to fp32 before the sum instead of fused into it).
  *     all_reduce_form: 0 runs moe_combine.  1 runs the combine of the
  *     all_reduce form on the W logical ranks: moe_combine_rank for r = 0..W-1
  *     into b->partials[r], then moe_reduce_partials into out (the same sum,
@@ -586,6 +593,7 @@ typedef struct moe_layer_options {
     int32_t fused_gather;      /* 0: permute, then the GEMM; 1: the GEMM gathers the rows */
     int32_t all_reduce_form;   /* 0: one combine; 1: W per-rank partials, then their sum */
     int32_t packed_weights;    /* 0: w13/w2 stacked; 1: in moe_pack_expert_weights' layout */
+    int32_t weights_in_gemm;   /* 0: combine weights the rows; 1: the down GEMM does */
 } moe_layer_options;
 
 typedef struct moe_layer_buffers {
