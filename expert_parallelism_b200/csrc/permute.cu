@@ -66,9 +66,6 @@ __global__ void __launch_bounds__(kPermuteMaxThreads) permute_copy_kernel(const 
         }
         __syncthreads();
     }
-    // rows stored into other GPUs' buffers: make them visible system-wide
-    // before the kernel ends (the owners read them after a barrier)
-    if (map.send_base) __threadfence_system();
 }
 
 // 8 consecutive elements of a row as fp32.
@@ -197,7 +194,6 @@ __global__ void __launch_bounds__(kPermuteMaxThreads) permute_e4m3_kernel(
         }
         __syncthreads();
     }
-    if (map.send_base) __threadfence_system();
 }
 
 // Threads per CTA for `units` equal pieces of work per token (16-byte

@@ -68,8 +68,8 @@ def test_weights_in_gemm_with_fused_gather(cuda_device):
 @pytest.mark.gpu
 def test_weights_in_gemm_full_size_dsv3(cuda_device):
     """dsv3 at full size: every y row is the default fp32 y row times its
-    router weight, bit for bit; out is the default layer's out or one bf16
-    ulp from it."""
+    router weight, bit for bit; out differs from the default layer's out by
+    at most one bf16 rounding plus the fp32 roundings of the k terms."""
     wl = workloads.WORKLOADS["dsv3"]
     g = GpuLayer(wl, cuda_device)
     assert g.run() == 0
@@ -79,7 +79,13 @@ def test_weights_in_gemm_full_size_dsv3(cuda_device):
     n = wl.N
     w = _weights_of_slots(wb, n).to(cuda_device)
     assert torch.equal(bits(wb.y), bits(y0 * w[:, None]))
-    # the two fp32 sums differ by a few fp32 ulps; rounded to bf16 they are
-    # equal or one bf16 ulp apart (at most 2^-7 of the value)
+    # the two fp32 sums (of fl(w*y) terms, and of fused w*y + acc steps)
+    # differ by a few fp32 roundings of the terms; each is then rounded to
+    # bf16 once: |d| <= one bf16 ulp of out (2^-7 |out|) + 2^-20 sum_j |w_j y_j|
+    sop = wb.slot_of_pair.view(wl.T, wl.k).long()
+    tw = wb.topk_w.view(wl.T, wl.k)
+    mag = torch.zeros(wl.T, wl.H, device=cuda_device)
+    for j in range(wl.k):
+        mag += (tw[:, j:j + 1] * y0[sop[:, j]]).abs()
     d = (wb.out.float() - out0.float()).abs()
-    assert bool((d <= 2.0 ** -7 * out0.float().abs() + 1e-30).all())
+    assert bool((d <= 2.0 ** -7 * out0.float().abs() + 2.0 ** -20 * mag).all())
