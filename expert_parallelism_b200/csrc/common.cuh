@@ -86,13 +86,6 @@ __device__ __forceinline__ void st_v4(void* p, const uint4& v) {
                  "r"(v.z), "r"(v.w)
                  : "memory");
 }
-// The same store with the streaming (evict-first) cache hint, for outputs
-// that nothing reads soon.
-__device__ __forceinline__ void st_v4_cs(void* p, const uint4& v) {
-    asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y),
-                 "r"(v.z), "r"(v.w)
-                 : "memory");
-}
 
 // The FP8 payload rule, shared by the dispatch payload (permute) and the
 // combine payload (the down GEMM's epilogue): for a block with largest
