@@ -9,7 +9,7 @@ import torch
 
 from expert_parallelism_b200 import moe, workloads
 
-from parity_helpers import GpuLayer, bits
+from parity_helpers import GpuLayer
 
 CASES = {
     "cap_bf16": workloads.Workload("cap_p", 600, 256, 8, 2, 192, 2, "bf16", "bf16", "bf16",
