@@ -14,7 +14,9 @@
 // With the FP8 combine payload ("Expert parallelism and all-to-all",
 // "Traffic math": 1-byte activations both ways) y holds e4m3 codes with one
 // fp32 scale per 128 elements; a piece is 16 codes (one 16-byte load) and
-// its block's scale, used as decode(q) * scale, an fp32 product.
+// its block's scale.  A code q adds (w * scale) * decode(q): the pick's
+// weight times the block scale is one fp32 product per piece, then each
+// decoded code (exact in fp32) goes in with a fused multiply-add.
 //
 // The all_reduce form of the layer (Transformers docs, "Expert
 // parallelism", "Choosing an implementation": no token moves, every rank
@@ -59,8 +61,8 @@ __device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&f)[8]) {
 // loads are issued before any sum), add() folds w * piece into the fp32
 // accumulators in element order.  fp32 / bf16 y: 8 elements (16 bytes),
 // converted at load.  e4m3 y: 16 codes (16 bytes) and the block's scale,
-// kept raw until add() (decode(q) * scale, an fp32 product), so four picks
-// in flight hold 4 x 5 registers instead of 4 x 16.
+// kept raw until add(), so four picks in flight hold 4 x 5 registers
+// instead of 4 x 16.
 template <typename TY>
 struct Piece {
     static constexpr int N = 8;
@@ -89,16 +91,20 @@ struct Piece<uint8_t> {
         r.q = ld_nc_v4(y + s * H + c * 16);
         r.sc = __ldg(y_scales + s * (H / 128) + (c * 16) / 128);
     }
+    // The pick's weight times the block's scale (one fp32 product per 16
+    // codes), then one fused multiply-add per code: an FP8-y combine of dsv3
+    // ran 143 us this way against 158 us with a product per code.
     static __device__ __forceinline__ void add(float (&acc)[16], const Raw& r, float w) {
         const uint32_t q[4] = {r.q.x, r.q.y, r.q.z, r.q.w};
+        const float ws = __fmul_rn(w, r.sc);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const float2 a = decode2_e4m3((uint16_t)(q[i] & 0xFFFFu));
             const float2 b = decode2_e4m3((uint16_t)(q[i] >> 16));
-            acc[4 * i + 0] = fmaf(w, __fmul_rn(a.x, r.sc), acc[4 * i + 0]);
-            acc[4 * i + 1] = fmaf(w, __fmul_rn(a.y, r.sc), acc[4 * i + 1]);
-            acc[4 * i + 2] = fmaf(w, __fmul_rn(b.x, r.sc), acc[4 * i + 2]);
-            acc[4 * i + 3] = fmaf(w, __fmul_rn(b.y, r.sc), acc[4 * i + 3]);
+            acc[4 * i + 0] = fmaf(ws, a.x, acc[4 * i + 0]);
+            acc[4 * i + 1] = fmaf(ws, a.y, acc[4 * i + 1]);
+            acc[4 * i + 2] = fmaf(ws, b.x, acc[4 * i + 2]);
+            acc[4 * i + 3] = fmaf(ws, b.y, acc[4 * i + 3]);
         }
     }
 };

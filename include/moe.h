@@ -372,8 +372,10 @@ moe_status moe_grouped_gemm_packed(const void* xp, moe_dtype xp_dtype, const flo
  * expert output for each token).
  *
  *   y            [>= max slot + 1, H] in y_dtype (MOE_F32 / MOE_BF16, or MOE_E4M3
- *                codes: each element used as decode(q) * scale of its
- *                128-element block, an fp32 product), device.
+ *                codes with one scale per 128-element block: a code adds
+ *                (topk_w * scale) * decode(q), the weight-scale product in
+ *                fp32 once per 16 codes, then a fused multiply-add per
+ *                code), device.
  *   y_scales     [>= max slot + 1, H/128] fp32 when y_dtype == MOE_E4M3
  *                (H % 128 == 0), else ignored (may be NULL).
  *   slot_of_pair [T*k] int32, device.
