@@ -590,7 +590,7 @@ def run_ours(args, wl):
 def run_ep(args, wl):
     """Expert parallelism (``--ep``).  Under torchrun with N GPUs: N ranks,
     each with its own T tokens and E/N experts, rows moved to their owners
-    through peer-mapped symmetric-memory buffers (DistributedEP); weak
+    through peer buffers mapped with CUDA IPC (DistributedEP); weak
     scaling.  On one GPU: ``--ep-ranks`` W ranks emulated on the device, each
     with T/W tokens (EmulatedEP), the same total batch as the plain step.
     A step is one layer on every rank; the time is the max over ranks."""

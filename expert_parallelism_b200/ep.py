@@ -220,15 +220,20 @@ class DistributedEP:
             self.dist.barrier(group=self.group)
 
     def forward(self, logits, x, w13_local, w2_local, stream=None):
+        """One layer on this rank.  With ``stream`` given, the kernels and the
+        collectives (count exchange, barriers) are all ordered on it."""
+        if stream is not None:
+            with torch.cuda.stream(stream):
+                return self.forward(logits, x, w13_local, w2_local)
         S = self.state
-        S.route_and_layout(logits, stream=stream)
+        S.route_and_layout(logits)
         exchange_counts(S.expert_counts, S.counts_all, self.group)
-        S.plan(self.rank, stream=stream)
-        S.dispatch(x, self.recv_rows, self.recv_scales, stream=stream)
+        S.plan(self.rank)
+        S.dispatch(x, self.recv_rows, self.recv_scales)
         self.barrier()                       # every rank's rows have landed
-        S.experts(w13_local, w2_local, stream=stream)
+        S.experts(w13_local, w2_local)
         self.barrier()                       # every owner's y is written
-        S.combine(self.y_rows, self.y_scales, stream=stream)
+        S.combine(self.y_rows, self.y_scales)
         self.barrier()                       # nobody reads this rank's y any more
         return S.out
 
