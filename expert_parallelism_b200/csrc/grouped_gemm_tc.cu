@@ -341,9 +341,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_before();
             if constexpr (NCTA == 2)
-                mbar_arrive_cluster(map_to_rank(tempty_bar(acc), 0));   // the leader's barrier
+                mbar_arrive_signal(map_to_rank(tempty_bar(acc), 0));   // the leader's barrier
             else
-                mbar_arrive_cluster(tempty_bar(acc));
+                mbar_arrive_signal(tempty_bar(acc));
             if (++acc == 2) {
                 acc = 0;
                 acc_phase ^= 1u;

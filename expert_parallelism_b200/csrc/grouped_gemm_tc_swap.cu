@@ -622,7 +622,7 @@ __global__ void __launch_bounds__(threads_of<GATHER>(), 1)
                     }
                 }
                 tc_fence_before();
-                mbar_arrive_cluster(map_to_rank(tempty_bar(nslot & 1), 0));   // leader's barrier
+                mbar_arrive_signal(map_to_rank(tempty_bar(nslot & 1), 0));   // leader's barrier
             }
         }
     }

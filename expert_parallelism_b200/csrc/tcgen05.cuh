@@ -39,10 +39,25 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
 
-// Arrive on a barrier given by its cluster-window address (own or peer CTA).
+// Arrive on a barrier given by its cluster-window address (own or peer CTA)
+// with a cluster-scope release: this thread's earlier memory writes (shared
+// memory the peer CTA's MMA will read) are visible to whoever acquires the
+// phase.  Costly: on B200 each such arrive stalls the thread for about half a
+// microsecond (a load-stream probe whose consumer released its stages this
+// way ran at 2.8 instead of 6.6 TB/s), so it is kept off per-k-step paths
+// that publish no data.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cbar) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cbar)
                  : "memory");
+}
+
+// Arrive on a barrier given by its cluster-window address with the default
+// (CTA-scope) release: a pure signal.  Used where the ordering that matters
+// is that of tcgen05 operations, carried by tcgen05.fence::before_thread_sync
+// before the arrive and tcgen05.fence::after_thread_sync after the wait (an
+// epilogue's tensor-memory reads against the next MMA into that memory).
+__device__ __forceinline__ void mbar_arrive_signal(uint32_t cbar) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cbar) : "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
