@@ -40,22 +40,14 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
 }
 
 // Arrive on a barrier given by its cluster-window address (own or peer CTA)
-// with a cluster-scope release: this thread's earlier memory writes (shared
-// memory the peer CTA's MMA will read) are visible to whoever acquires the
-// phase.  Costly: on B200 each such arrive stalls the thread for about half a
-// microsecond (a load-stream probe whose consumer released its stages this
-// way ran at 2.8 instead of 6.6 TB/s), so it is kept off per-k-step paths
-// that publish no data.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cbar) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cbar)
-                 : "memory");
-}
-
-// Arrive on a barrier given by its cluster-window address with the default
-// (CTA-scope) release: a pure signal.  Used where the ordering that matters
-// is that of tcgen05 operations, carried by tcgen05.fence::before_thread_sync
-// before the arrive and tcgen05.fence::after_thread_sync after the wait (an
-// epilogue's tensor-memory reads against the next MMA into that memory).
+// with the default, CTA-scope release: a signal.  What it orders is carried
+// by the operations around it: tcgen05.fence::before_thread_sync before the
+// arrive and tcgen05.fence::after_thread_sync after the wait (an epilogue's
+// tensor-memory reads against the next MMA into that memory), or copies
+// already complete in shared memory and fenced to the async proxy (the fused
+// gather).  A cluster-scope release (.release.cluster) would stall the thread
+// about half a microsecond per arrive on B200: a load-stream probe whose
+// consumer released its stages that way ran at 2.8 instead of 6.6 TB/s.
 __device__ __forceinline__ void mbar_arrive_signal(uint32_t cbar) {
     asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cbar) : "memory");
 }
