@@ -235,6 +235,13 @@ __device__ __forceinline__ void load_rows(uint32_t dst, const CUtensorMap* m128,
     tma_load_2d<2>(dst, b == 128 ? m128 : b == 32 ? m32 : m8, bar, k0, r0);
 }
 
+// Clock record, summed over launches: per phase (gate/up, down), the SM
+// cycles (clock64) and the nanoseconds (globaltimer) CTA 0 spent from its
+// first instruction to its last.  Their ratio is the SM clock the kernel ran
+// at, which the power cap can hold well below the nominal maximum while the
+// tensor cores and the weight stream are both busy.
+__device__ unsigned long long g_swap_clock[4];
+
 template <bool GLU, typename OutT, bool GATHER>
 __global__ void __launch_bounds__(threads_of<GATHER>(), 1)
     grouped_gemm_swap_kernel(const __grid_constant__ CUtensorMap tmap_w,
@@ -248,6 +255,9 @@ __global__ void __launch_bounds__(threads_of<GATHER>(), 1)
     const uint32_t rank = cluster_ctarank();   // 0 = leader
     const bool leader = rank == 0;
     const int unit = blockIdx.x / 2, n_units = gridDim.x / 2;
+    const bool clock_cta = blockIdx.x == 0 && threadIdx.x == 0;
+    const long long clk0 = clock_cta ? clock64() : 0;
+    const uint64_t ns0 = clock_cta ? global_timer_ns() : 0;
 
     const uint32_t bar0 = sbase + Smem::bars;
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
@@ -649,6 +659,10 @@ __global__ void __launch_bounds__(threads_of<GATHER>(), 1)
         asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                      "r"(kTmemCols)
                      : "memory");
+    if (clock_cta) {
+        atomicAdd(&g_swap_clock[GLU ? 0 : 2], (unsigned long long)(clock64() - clk0));
+        atomicAdd(&g_swap_clock[GLU ? 1 : 3], (unsigned long long)(global_timer_ns() - ns0));
+    }
 }
 
 // ---------------------------------------------------------------- host side
@@ -784,3 +798,14 @@ cudaError_t launch_grouped_gemm_tc_swap(const __nv_bfloat16* a, const int32_t* o
 }
 
 }  // namespace moe
+
+extern "C" moe_status moe_diag_gemm_clock(uint64_t* out, int32_t reset) {
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess && out)
+        e = cudaMemcpyFromSymbol(out, moe::tcs::g_swap_clock, sizeof(moe::tcs::g_swap_clock));
+    if (e == cudaSuccess && reset) {
+        const unsigned long long zero[4] = {0, 0, 0, 0};
+        e = cudaMemcpyToSymbol(moe::tcs::g_swap_clock, zero, sizeof(zero));
+    }
+    return moe::report_cuda(e);
+}

@@ -65,6 +65,7 @@ SIGNATURES = {
     "moe_ipc_close": ([_P, _P], _I),
     "moe_diag_layout_wait_timeout_workspace_bytes": ([], _SZ),
     "moe_diag_layout_wait_timeout": ([_P, _SZ, ctypes.c_uint64, _P, _P], _I),
+    "moe_diag_gemm_clock": ([_P, ctypes.c_int32], _I),
 }
 
 
@@ -330,6 +331,15 @@ def moe_ep_combine(y_rows, y_scales, y_dtype, topk_idx, slot_of_pair, expert_off
         _ptr_array(y_rows), sc, _DT[y_dtype], _ptr(topk_idx), _ptr(slot_of_pair),
         _ptr(expert_offsets), _ptr(send_base), _ptr(topk_w), T, k, H, E, W, rows_capacity,
         _ptr(out), dtype_code(out), _ptr(dev_status), _stream(stream)))
+
+
+def moe_diag_gemm_clock(reset=False):
+    """The grouped GEMM's clock record: {"gate_up": (cycles, ns), "down":
+    (cycles, ns)} summed over launches since the last reset (synchronises the
+    device); with reset, clears it afterwards."""
+    out = (ctypes.c_uint64 * 4)()
+    _check("moe_diag_gemm_clock", load_library().moe_diag_gemm_clock(out, 1 if reset else 0))
+    return {"gate_up": (int(out[0]), int(out[1])), "down": (int(out[2]), int(out[3]))}
 
 
 def moe_diag_layout_wait_timeout(workspace, wait_limit_ns, dev_status, stream=None):

@@ -660,6 +660,20 @@ const char* moe_status_str(moe_status s);
 uint64_t moe_launch_count(void);
 
 /*
+ * moe_diag_gemm_clock -- diagnostics: the SM clock the operand-swapped
+ * grouped GEMM ran at (the bf16 tensor-core kernel moe_grouped_gemm and the
+ * layer use from 16 routed rows per expert on average, or with an FP8 y,
+ * packed weights or router weights in the GEMM; below that, the token-major
+ * kernel runs and records nothing).  Every launch adds, for CTA 0, the SM cycles (clock64) and the
+ * nanoseconds (globaltimer) from its first instruction to its last into a
+ * per-device record: out[0], out[1] for the gate/up phase, out[2], out[3]
+ * for the down phase; cycles / ns is the mean clock in GHz.  Synchronises
+ * the current device, then copies the record to out (4 uint64, host; may be
+ * NULL) and, with reset non-zero, clears it.  MOE_ERR_CUDA if a copy fails.
+ */
+moe_status moe_diag_gemm_clock(uint64_t* out, int32_t reset);
+
+/*
  * moe_diag_layout_wait_timeout -- diagnostics for failure detection: runs
  * the dispatch layout's scan kernel (the one moe_dispatch_layout launches)
  * on a two-chunk look-back state in which the first chunk never publishes
