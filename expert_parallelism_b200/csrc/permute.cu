@@ -85,9 +85,15 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&f)[8]) {
 
 constexpr int kMaxBlocks = 64;           // scales staged in shared memory: H <= 8192
 
+__device__ __forceinline__ void st_v2(void* p, uint32_t x, uint32_t y) {
+    asm volatile("st.global.v2.u32 [%0], {%1,%2};" ::"l"(p), "r"(x), "r"(y) : "memory");
+}
+
 // FP8 payload: one CTA per token (grid-stride).  8 lanes own a 128-element
-// block (16 elements each): amax by shuffles, scale = amax / 448, and
-// 16-byte stores of codes to each of the token's k destinations.  The
+// block, lane i its elements 8i..8i+7 and 64+8i..64+8i+7, so every store
+// instruction of the 8 lanes covers whole 32-byte sectors (64 bytes of codes,
+// 128 bytes of bf16): amax by shuffles, scale = amax / 448, and 8-byte
+// stores of codes to each of the token's k destinations.  The
 // token's scales are staged in shared memory and written as 16-byte vectors
 // per destination once the row is done.  With `a` non-null (the layer call,
 // local layout), the kernel also writes what the grouped GEMM consumes,
@@ -122,8 +128,8 @@ __global__ void __launch_bounds__(kPermuteMaxThreads) permute_e4m3_kernel(
             float amax = 0.0f;
             if (live) {
                 float a8[8], b8[8];
-                load8(row + g * 128 + l8 * 16, a8);
-                load8(row + g * 128 + l8 * 16 + 8, b8);
+                load8(row + g * 128 + l8 * 8, a8);         // elements 8 l8 ..
+                load8(row + g * 128 + 64 + l8 * 8, b8);    // elements 64 + 8 l8 ..
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     f[i] = a8[i];
@@ -143,9 +149,11 @@ __global__ void __launch_bounds__(kPermuteMaxThreads) permute_e4m3_kernel(
                                        quant4_e4m3(f[12], f[13], f[14], f[15], scale));
             for (int j = 0; j < k && !tok_major; ++j) {
                 const int r = s_rank[j];
-                if (r >= 0)
-                    st_v4(reinterpret_cast<uint8_t*>(dst.rows[r]) + s_row[j] * H + g * 128 + l8 * 16,
-                          q);
+                if (r >= 0) {
+                    uint8_t* d = reinterpret_cast<uint8_t*>(dst.rows[r]) + s_row[j] * H + g * 128;
+                    st_v2(d + l8 * 8, q.x, q.y);
+                    st_v2(d + 64 + l8 * 8, q.z, q.w);
+                }
             }
             if (a) {
                 // the GEMM's operand: each code decoded (exact) times the scale
@@ -161,15 +169,15 @@ __global__ void __launch_bounds__(kPermuteMaxThreads) permute_e4m3_kernel(
                 const uint4 b0 = make_uint4(bw[0], bw[1], bw[2], bw[3]);
                 const uint4 b1 = make_uint4(bw[4], bw[5], bw[6], bw[7]);
                 if (tok_major) {
-                    __nv_bfloat16* d = a + t * H + g * 128 + l8 * 16;
-                    st_v4(d, b0);
-                    st_v4(d + 8, b1);
+                    __nv_bfloat16* d = a + t * H + g * 128;
+                    st_v4(d + l8 * 8, b0);
+                    st_v4(d + 64 + l8 * 8, b1);
                 }
                 for (int j = 0; j < k && !tok_major; ++j) {
                     if (s_rank[j] < 0) continue;
-                    __nv_bfloat16* d = a + s_row[j] * H + g * 128 + l8 * 16;
-                    st_v4(d, b0);
-                    st_v4(d + 8, b1);
+                    __nv_bfloat16* d = a + s_row[j] * H + g * 128;
+                    st_v4(d + l8 * 8, b0);
+                    st_v4(d + 64 + l8 * 8, b1);
                 }
             }
             if (l8 == 0 && !tok_major) {
