@@ -24,7 +24,8 @@ def _counts(W, E, seed, hi=6):
     return c
 
 
-@pytest.mark.parametrize("W,E,seed", [(1, 5, 0), (2, 4, 1), (3, 6, 2), (4, 8, 3), (4, 4, 4)])
+@pytest.mark.parametrize("W,E,seed", [(1, 5, 0), (2, 4, 1), (3, 6, 2), (4, 8, 3), (4, 4, 4),
+                                       (8, 16, 5), (8, 64, 6)])
 def test_plan_tiles_every_owner_buffer_in_expert_then_source_order(W, E, seed):
     """Brute force over every (source, expert) chunk: for each owner the
     chunks [send_base, send_base + count) are disjoint, cover [0, total)
@@ -98,7 +99,7 @@ def test_dest_rows_are_a_bijection_onto_each_owner_buffer():
     assert all(bool((h == 1).all()) for h in hits)
 
 
-@pytest.mark.parametrize("W,payload", [(2, "bf16"), (4, "bf16"), (2, "e4m3")])
+@pytest.mark.parametrize("W,payload", [(2, "bf16"), (4, "bf16"), (2, "e4m3"), (8, "e4m3")])
 def test_expert_parallel_layer_equals_the_single_rank_layer(W, payload):
     """Moving rows to their owners and back changes nothing: every rank's out
     equals the single-GPU layer on its own tokens, bit for bit (fp64, each
