@@ -32,7 +32,8 @@
  *    where a call says otherwise).  Index arrays are int32.
  *  - The caller allocates and owns every buffer, including workspaces and
  *    the device status word.  The library allocates nothing, frees
- *    nothing and never synchronises, except moe_check_status.
+ *    nothing and never synchronises, except moe_check_status and the
+ *    diagnostic moe_diag_gemm_clock.
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
  *    call only enqueues work on it and returns; the chain of calls has no
  *    host synchronisation, so it can be captured in a CUDA graph.
